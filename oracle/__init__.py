@@ -1,0 +1,2 @@
+"""fp64 CPU oracle (test infrastructure; never imported by the product path)."""
+from . import isloss_oracle  # noqa: F401
