@@ -1,0 +1,485 @@
+// bi_api.cu -- the C ABI declared in include/bi_isloss.h: argument checks, workspace layout,
+// tensor maps and the fixed launch sequence.  Nothing here allocates device memory.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <array>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/bi_isloss.h"
+#include "kernels_bwd.cuh"
+#include "kernels_fwd.cuh"
+#include "kernels_small.cuh"
+
+namespace {
+
+using bi::Ctrl;
+using bi::RedPart;
+
+constexpr uint64_t kWaitLimitNs = 4000000000ull;  // 4 s for any single in-kernel wait
+constexpr int kMaxSms = 160;                      // upper bound used to size the dZ scratch
+constexpr int kDzSlotsMax = 2 * kMaxSms;          // clusters * C * slots-per-CTA <= 2 * SMs
+
+thread_local uint64_t g_force_timeout_ns = 0;
+
+// ---------------------------------------------------------------------------------------------
+// optional per-kernel timing (events around each launch; measurement tools only)
+// ---------------------------------------------------------------------------------------------
+enum KernelKind : int { kKPrep, kKRowmap, kKZeroRows, kKGather, kKFwd, kKCombineLp, kKCombineIs, kKReduce,
+                        kKBwdDH, kKBwdDW, kKD3Partial, kNumKinds };
+const char* const kKindNames[kNumKinds] = {"k_prep", "k_rowmap", "k_zero_prompt_rows", "k_gather_rows",
+                                           "k_fwd_logits", "k_combine_logprob", "k_combine_is",
+                                           "k_reduce_parts", "k_bwd_dh", "k_bwd_dw", "k_d3_partial"};
+struct Pending {
+  int kind;
+  cudaEvent_t a, b;
+};
+struct Profiler {
+  bool on = false;
+  bool failed = false;
+  std::vector<Pending> pending;
+  std::vector<cudaEvent_t> pool;
+  double ms[kNumKinds] = {};
+  int64_t n[kNumKinds] = {};
+  cudaEvent_t get() {
+    if (!pool.empty()) {
+      cudaEvent_t e = pool.back();
+      pool.pop_back();
+      return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) failed = true;
+    return e;
+  }
+};
+thread_local Profiler g_prof;
+
+struct ProfScope {  // records an event pair around one launch when profiling is on
+  int kind;
+  cudaStream_t s;
+  cudaEvent_t a = nullptr;
+  ProfScope(int k, cudaStream_t st) : kind(k), s(st) {
+    if (g_prof.on) {
+      a = g_prof.get();
+      if (a) cudaEventRecord(a, s);
+    }
+  }
+  ~ProfScope() {
+    if (g_prof.on && a) {
+      cudaEvent_t b = g_prof.get();
+      if (b) {
+        cudaEventRecord(b, s);
+        g_prof.pending.push_back({kind, a, b});
+      }
+    }
+  }
+};
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct WsLayout {
+  size_t ctrl, part_m, part_s, part_zy, lse_c, g_c, y_c, logmu_c, rowmap, respof, coef, cprefix, red, hc, dz, total;
+  int nred;
+};
+
+WsLayout ws_layout(int64_t T, int32_t H, int32_t R) {
+  WsLayout L{};
+  const size_t t = static_cast<size_t>(T > 0 ? T : 1);
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o = align_up(o + bytes, 256);
+    return at;
+  };
+  L.ctrl = take(256);
+  L.part_m = take(bi::kMaxVChunks * t * 4);
+  L.part_s = take(bi::kMaxVChunks * t * 4);
+  L.part_zy = take(bi::kMaxVChunks * t * 4);
+  L.lse_c = take(t * 4);
+  L.g_c = take(t * 4);
+  L.y_c = take(t * 4);
+  L.logmu_c = take(t * 4);
+  L.rowmap = take(t * 4);
+  L.respof = take(t * 4);
+  L.coef = take(static_cast<size_t>(R > 0 ? R : 1) * 8);
+  L.cprefix = take(static_cast<size_t>(R + 1) * 8);
+  L.nred = static_cast<int>((t + bi::kRedBlock - 1) / bi::kRedBlock);
+  L.red = take(static_cast<size_t>(L.nred) * sizeof(RedPart));
+  L.hc = take(R > 0 ? t * static_cast<size_t>(H) * 2 : 0);
+  L.dz = take(static_cast<size_t>(kDzSlotsMax) * 128 * 128 * 2);
+  L.total = o;
+  return L;
+}
+
+// Split of H over a cluster: smallest C in {1, 2, 4, 8} with H / C <= 384 and a multiple of 64.
+int cluster_split(int32_t H) {
+  for (int c : {1, 2, 4, 8})
+    if (H % c == 0 && (H / c) % 64 == 0 && H / c <= 384) return c;
+  return 0;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---------------------------------------------------------------------------------------------
+// tensor maps (driver entry point fetched through the runtime; no libcuda link dependency)
+// ---------------------------------------------------------------------------------------------
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 row-major tensor [rows][cols], box {64 columns, box_rows rows}, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows) {
+  EncodeTiledFn f = encode_fn();
+  if (!f) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows > 0 ? rows : 1)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+  const cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1u, 1u};
+  return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------------------------------------
+// per-device set-up (kernel attributes, SM count, cluster occupancy), done once per device
+// ---------------------------------------------------------------------------------------------
+struct DevInfo {
+  bool ready = false;
+  bool ok = false;
+  int sms = 0;
+  int max_clusters[2][9] = {};  // [mode][C]
+};
+std::mutex g_dev_mu;
+std::array<DevInfo, 64> g_dev;
+
+template <int kMode>
+int query_clusters(int C) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(C, 1, 1);
+  cfg.blockDim = dim3(bi::kBwdThreads, 1, 1);
+  cfg.dynamicSmemBytes = bi::kBwdSmemBytes;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, bi::k_bwd_cluster<kMode>, &cfg) != cudaSuccess) return 0;
+  return n;
+}
+
+const DevInfo* device_info() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= static_cast<int>(g_dev.size())) return nullptr;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DevInfo& d = g_dev[dev];
+  if (d.ready) return d.ok ? &d : nullptr;
+  d.ready = true;
+  if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return nullptr;
+  if (cudaFuncSetAttribute(bi::k_fwd_logits, cudaFuncAttributeMaxDynamicSharedMemorySize, bi::kFwdSmemBytes) !=
+          cudaSuccess ||
+      cudaFuncSetAttribute(bi::k_bwd_cluster<bi::kModeDH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           bi::kBwdSmemBytes) != cudaSuccess ||
+      cudaFuncSetAttribute(bi::k_bwd_cluster<bi::kModeDW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           bi::kBwdSmemBytes) != cudaSuccess)
+    return nullptr;
+  for (int c : {1, 2, 4, 8}) {
+    d.max_clusters[0][c] = query_clusters<bi::kModeDH>(c);
+    d.max_clusters[1][c] = query_clusters<bi::kModeDW>(c);
+  }
+  cudaGetLastError();
+  d.ok = d.sms > 0 && d.sms <= kMaxSms;
+  return d.ok ? &d : nullptr;
+}
+
+int nchunks_for(int nvt) { return nvt < bi::kMaxVChunks ? nvt : bi::kMaxVChunks; }
+
+bi_status launch_fwd(const uint16_t* hidden, int64_t T, const int64_t* d_rows, const uint16_t* w, int32_t H,
+                     int32_t V, const int32_t* targets, const WsLayout& L, uint8_t* ws, int32_t* dev_status,
+                     const DevInfo* di, cudaStream_t s, uint64_t force_timeout_ns) {
+  CUtensorMap tm_h, tm_w;
+  if (!make_map(&tm_h, hidden, T, H, bi::kFwdBM) || !make_map(&tm_w, w, V, H, bi::kFwdBN)) return BI_ERR_CUDA;
+  bi::FwdArgs a{};
+  a.T = T;
+  a.d_rows = d_rows;
+  a.H = H;
+  a.V = V;
+  a.nvt = (V + bi::kFwdBN - 1) / bi::kFwdBN;
+  a.nchunks = nchunks_for(a.nvt);
+  a.targets = targets;
+  a.part_m = reinterpret_cast<float*>(ws + L.part_m);
+  a.part_s = reinterpret_cast<float*>(ws + L.part_s);
+  a.part_zy = reinterpret_cast<float*>(ws + L.part_zy);
+  a.status = dev_status;
+  a.limit_ns = kWaitLimitNs;
+  a.force_timeout_ns = force_timeout_ns;
+  const int64_t units = ((T + bi::kFwdBM - 1) / bi::kFwdBM) * a.nchunks;
+  const int grid = static_cast<int>(units < di->sms ? units : di->sms);
+  ProfScope ps(kKFwd, s);
+  bi::k_fwd_logits<<<grid, bi::kFwdThreads, bi::kFwdSmemBytes, s>>>(tm_h, tm_w, a);
+  return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+}
+
+template <int kMode>
+bi_status launch_bwd(const CUtensorMap& tm_stat, const CUtensorMap& tm_stream, const CUtensorMap& tm_dz,
+                     const bi::BwdArgs& a, int64_t units_upper, const DevInfo* di, cudaStream_t s) {
+  const int maxc = di->max_clusters[kMode][a.C];
+  if (maxc <= 0) return BI_ERR_CUDA;
+  int64_t ncl = units_upper < maxc ? units_upper : maxc;
+  if (ncl < 1) ncl = 1;
+  if (ncl * a.C * bi::kSlotsPerCta > kDzSlotsMax) return BI_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(ncl * a.C), 1, 1);
+  cfg.blockDim = dim3(bi::kBwdThreads, 1, 1);
+  cfg.dynamicSmemBytes = bi::kBwdSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = a.C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  ProfScope ps(kMode == bi::kModeDH ? kKBwdDH : kKBwdDW, s);
+  return cudaLaunchKernelEx(&cfg, bi::k_bwd_cluster<kMode>, tm_stat, tm_stream, tm_dz, a) == cudaSuccess
+             ? BI_OK
+             : BI_ERR_CUDA;
+}
+
+unsigned blocks_for(int64_t n, int per) { return static_cast<unsigned>((n + per - 1) / per); }
+
+}  // namespace
+
+extern "C" {
+
+int32_t bi_version(void) { return 100; }
+
+const char* bi_status_string(bi_status s) {
+  switch (s) {
+    case BI_OK: return "BI_OK";
+    case BI_ERR_INVALID_ARG: return "BI_ERR_INVALID_ARG";
+    case BI_ERR_UNSUPPORTED_SHAPE: return "BI_ERR_UNSUPPORTED_SHAPE";
+    case BI_ERR_WORKSPACE: return "BI_ERR_WORKSPACE";
+    case BI_ERR_CUDA: return "BI_ERR_CUDA";
+    case BI_ERR_TIMEOUT: return "BI_ERR_TIMEOUT";
+    case BI_ERR_BAD_TARGET: return "BI_ERR_BAD_TARGET";
+    case BI_ERR_NONFINITE: return "BI_ERR_NONFINITE";
+    case BI_ERR_BAD_OFFSETS: return "BI_ERR_BAD_OFFSETS";
+  }
+  return "BI_UNKNOWN";
+}
+
+void bi_debug_force_timeout_once(uint64_t limit_ns) { g_force_timeout_ns = limit_ns; }
+
+void bi_profile_enable(int32_t on) { g_prof.on = on != 0; }
+
+void bi_profile_reset(void) {
+  for (int k = 0; k < kNumKinds; ++k) {
+    g_prof.ms[k] = 0.0;
+    g_prof.n[k] = 0;
+  }
+}
+
+int32_t bi_profile_read(const char** names_out, double* ms_out, int64_t* launches_out, int32_t max_kernels) {
+  for (const Pending& p : g_prof.pending) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(p.b) != cudaSuccess || cudaEventElapsedTime(&ms, p.a, p.b) != cudaSuccess)
+      g_prof.failed = true;
+    g_prof.ms[p.kind] += ms;
+    g_prof.n[p.kind] += 1;
+    g_prof.pool.push_back(p.a);
+    g_prof.pool.push_back(p.b);
+  }
+  g_prof.pending.clear();
+  if (g_prof.failed) return -1;
+  int32_t m = 0;
+  for (int k = 0; k < kNumKinds && m < max_kernels; ++k) {
+    if (names_out) names_out[m] = kKindNames[k];
+    if (ms_out) ms_out[m] = g_prof.ms[k];
+    if (launches_out) launches_out[m] = g_prof.n[k];
+    ++m;
+  }
+  return m;
+}
+
+size_t bi_workspace_bytes(int64_t T, int32_t H, int32_t V, int32_t R) {
+  (void)V;
+  if (T < 0 || H <= 0 || R < 0) return 0;
+  return ws_layout(T, H, R).total;
+}
+
+bi_status bi_logprob_fwd(const uint16_t* hidden, const uint16_t* w_lm, const int32_t* targets, int64_t T, int32_t H,
+                         int32_t V, float* logprob, float* lse, int32_t* dev_status, void* ws, size_t ws_bytes,
+                         void* stream) {
+  const uint64_t force = g_force_timeout_ns;
+  g_force_timeout_ns = 0;
+  if (T < 0 || T >= (int64_t(1) << 31) || H <= 0 || V <= 0) return BI_ERR_INVALID_ARG;
+  if (!dev_status || (T > 0 && (!hidden || !w_lm || !targets || !logprob))) return BI_ERR_INVALID_ARG;
+  if (T > 0 && (!aligned16(hidden) || !aligned16(w_lm))) return BI_ERR_INVALID_ARG;
+  if (H % 64 != 0 || cluster_split(H) == 0) return BI_ERR_UNSUPPORTED_SHAPE;
+  const WsLayout L = ws_layout(T, H, 0);
+  if (!ws || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) return BI_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const DevInfo* di = device_info();
+  if (!di) return BI_ERR_CUDA;
+  if (cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s) != cudaSuccess) return BI_ERR_CUDA;
+  if (T == 0) return BI_OK;
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  bi_status st = launch_fwd(hidden, T, nullptr, w_lm, H, V, targets, L, w8, dev_status, di, s, force);
+  if (st != BI_OK) return st;
+  const int nvt = (V + bi::kFwdBN - 1) / bi::kFwdBN;
+  ProfScope ps(kKCombineLp, s);
+  bi::k_combine_logprob<<<blocks_for(T, 256), 256, 0, s>>>(
+      reinterpret_cast<float*>(w8 + L.part_m), reinterpret_cast<float*>(w8 + L.part_s),
+      reinterpret_cast<float*>(w8 + L.part_zy), T, nchunks_for(nvt), nvt, V, targets, logprob, lse, dev_status);
+  return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+}
+
+bi_status bi_is_loss_fwd_bwd(const uint16_t* hidden, const uint16_t* w_lm, const int32_t* targets,
+                             const float* rollout_logprob, const float* rewards, const int64_t* resp_offsets,
+                             const int32_t* group_offsets, const int32_t* prompt_lens, int32_t R, int32_t G,
+                             double resp_normalizer, int64_t T, int32_t H, int32_t V, float* loss, float* logprob,
+                             float* is_weight, float* token_loss, bi_d3* d3, uint16_t* grad_hidden, float* grad_w,
+                             int32_t* dev_status, void* ws, size_t ws_bytes, void* stream) {
+  if (T < 0 || T >= (int64_t(1) << 31) || H <= 0 || V <= 0 || R < 1 || G < 1 || G > R) return BI_ERR_INVALID_ARG;
+  if (!(resp_normalizer >= 0.0)) return BI_ERR_INVALID_ARG;
+  if (!dev_status || !w_lm || !rewards || !resp_offsets || !group_offsets || !loss || !grad_w)
+    return BI_ERR_INVALID_ARG;
+  if (T > 0 && (!hidden || !targets || !rollout_logprob || !logprob || !grad_hidden)) return BI_ERR_INVALID_ARG;
+  if (!aligned16(w_lm) || !aligned16(grad_w) || (T > 0 && (!aligned16(hidden) || !aligned16(grad_hidden))))
+    return BI_ERR_INVALID_ARG;
+  if (H % 64 != 0) return BI_ERR_UNSUPPORTED_SHAPE;
+  const int C = cluster_split(H);
+  if (C == 0) return BI_ERR_UNSUPPORTED_SHAPE;
+  const WsLayout L = ws_layout(T, H, R);
+  if (!ws || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) return BI_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const DevInfo* di = device_info();
+  if (!di) return BI_ERR_CUDA;
+  if (cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s) != cudaSuccess) return BI_ERR_CUDA;
+
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  Ctrl* ctrl = reinterpret_cast<Ctrl*>(w8 + L.ctrl);
+  const int64_t* d_rows = &ctrl->n_scored;
+  auto F = [&](size_t o) { return reinterpret_cast<float*>(w8 + o); };
+  auto I = [&](size_t o) { return reinterpret_cast<int32_t*>(w8 + o); };
+  const double rstar = resp_normalizer > 0.0 ? resp_normalizer : static_cast<double>(R);
+
+  { ProfScope ps(kKPrep, s);
+  bi::k_prep<<<1, 1024, 0, s>>>(rewards, resp_offsets, group_offsets, prompt_lens, R, G, rstar, T,
+                                reinterpret_cast<double*>(w8 + L.coef), reinterpret_cast<int64_t*>(w8 + L.cprefix),
+                                ctrl, dev_status);
+  }
+  if (T > 0) {
+    ProfScope ps(kKRowmap, s);
+    bi::k_rowmap<<<blocks_for(T, 256), 256, 0, s>>>(resp_offsets, prompt_lens, R, T,
+                                                    reinterpret_cast<int64_t*>(w8 + L.cprefix), ctrl, targets,
+                                                    rollout_logprob, I(L.rowmap), I(L.respof), I(L.y_c),
+                                                    F(L.logmu_c), logprob, is_weight, token_loss);
+  }
+  const uint16_t* hc = hidden;
+  if (T > 0 && prompt_lens) {
+    {
+      ProfScope ps(kKZeroRows, s);
+      bi::k_zero_prompt_rows<<<blocks_for(T * 32, 256), 256, 0, s>>>(resp_offsets, prompt_lens, R, T, H, ctrl,
+                                                                      grad_hidden);
+    }
+    uint16_t* hcw = reinterpret_cast<uint16_t*>(w8 + L.hc);
+    ProfScope ps(kKGather, s);
+    bi::k_gather_rows<<<blocks_for(T * 32, 256), 256, 0, s>>>(hidden, T, H, ctrl, I(L.rowmap), hcw);
+    hc = hcw;
+  }
+  if (cudaGetLastError() != cudaSuccess) return BI_ERR_CUDA;
+
+  const int nvt = (V + bi::kFwdBN - 1) / bi::kFwdBN;
+  if (T > 0) {
+    bi_status st = launch_fwd(hc, T, d_rows, w_lm, H, V, I(L.y_c), L, w8, dev_status, di, s, 0);
+    if (st != BI_OK) return st;
+  }
+  RedPart* parts = reinterpret_cast<RedPart*>(w8 + L.red);
+  {
+  ProfScope ps(kKCombineIs, s);
+  bi::k_combine_is<<<L.nred, bi::kRedBlock, 0, s>>>(F(L.part_m), F(L.part_s), F(L.part_zy), T > 0 ? T : 1,
+                                                    nchunks_for(nvt), nvt, V, ctrl, I(L.y_c), F(L.logmu_c),
+                                                    I(L.respof), I(L.rowmap), reinterpret_cast<double*>(w8 + L.coef),
+                                                    logprob, is_weight, token_loss, F(L.lse_c), F(L.g_c), parts,
+                                                    dev_status);
+  }
+  {
+  ProfScope ps(kKReduce, s);
+  bi::k_reduce_parts<<<1, 1024, 0, s>>>(parts, L.nred, loss, reinterpret_cast<bi::D3Out*>(d3), dev_status);
+  }
+  if (cudaGetLastError() != cudaSuccess) return BI_ERR_CUDA;
+
+  // backward: dH (row tiles) and dW (vocabulary tiles)
+  CUtensorMap tm_h, tm_w, tm_dz;
+  const int64_t trows = T > 0 ? T : 1;
+  if (!make_map(&tm_h, hc ? hc : reinterpret_cast<const uint16_t*>(w8 + L.hc), trows, H, 128) ||
+      !make_map(&tm_w, w_lm, V, H, 128) ||
+      !make_map(&tm_dz, w8 + L.dz, static_cast<int64_t>(kDzSlotsMax) * 128, 128, 128))
+    return BI_ERR_CUDA;
+  bi::BwdArgs a{};
+  a.H = H;
+  a.V = V;
+  a.C = C;
+  a.Hs = H / C;
+  const int su = a.Hs / 64;
+  a.nchunk = su > 4 ? 2 : 1;
+  a.chunk_units[0] = a.nchunk == 2 ? (su + 1) / 2 : su;
+  a.chunk_units[1] = a.nchunk == 2 ? su / 2 : 0;
+  a.T = trows;
+  a.d_rows = d_rows;
+  a.nvt128 = (V + 127) / 128;
+  a.lse = F(L.lse_c);
+  a.g = F(L.g_c);
+  a.y = I(L.y_c);
+  a.rowmap = I(L.rowmap);
+  a.grad_hidden = grad_hidden;
+  a.grad_w = grad_w;
+  a.dz_scratch = reinterpret_cast<uint16_t*>(w8 + L.dz);
+  a.status = dev_status;
+  a.limit_ns = kWaitLimitNs;
+  bi_status st = BI_OK;
+  if (T > 0) st = launch_bwd<bi::kModeDH>(tm_h, tm_w, tm_dz, a, (T + 127) / 128, di, s);
+  if (st != BI_OK) return st;
+  return launch_bwd<bi::kModeDW>(tm_w, tm_h, tm_dz, a, a.nvt128, di, s);
+}
+
+bi_status bi_d3_stats(const float* learner_logprob, const float* rollout_logprob, const uint8_t* mask, int64_t T,
+                      bi_d3* out, int32_t* dev_status, void* ws, size_t ws_bytes, void* stream) {
+  if (T < 0 || !out || !dev_status || (T > 0 && (!learner_logprob || !rollout_logprob))) return BI_ERR_INVALID_ARG;
+  const size_t nred = static_cast<size_t>((T > 0 ? T : 1) + bi::kRedBlock - 1) / bi::kRedBlock;
+  if (!ws || ws_bytes < nred * sizeof(RedPart) || (reinterpret_cast<uintptr_t>(ws) & 255u)) return BI_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s) != cudaSuccess) return BI_ERR_CUDA;
+  RedPart* parts = static_cast<RedPart*>(ws);
+  {
+  ProfScope ps(kKD3Partial, s);
+  bi::k_d3_partial<<<static_cast<unsigned>(nred), bi::kRedBlock, 0, s>>>(learner_logprob, rollout_logprob, mask, T,
+                                                                         parts);
+  }
+  ProfScope ps(kKReduce, s);
+  bi::k_reduce_parts<<<1, 1024, 0, s>>>(parts, static_cast<int>(nred), nullptr, reinterpret_cast<bi::D3Out*>(out),
+                                        dev_status);
+  return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+}
+
+}  // extern "C"

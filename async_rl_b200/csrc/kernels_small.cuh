@@ -1,0 +1,288 @@
+// kernels_small.cuh -- the light, memory-bound steps around the two tensor-core kernels:
+// offsets validation and per-response coefficients, the scored-row map, the gather of scored
+// rows, the per-row combine (lse, log pi, IS weight, D3 term, token loss) and the fixed-order
+// reductions of the loss and the D3 statistics.  No atomics take part in any sum: every
+// reduction has a fixed tree shape that depends only on the number of rows.
+//
+// Definitions: "Zero Mismatch, Simple Async RL", sections "Only one probability gap comes from
+// old weights" (w = pi / mu, D3 = mean of w - 1 - log w) and "Alignment permits a simpler
+// learning path" (advantage = reward - group mean, tokens averaged within each response,
+// no clipping, no gate).
+#pragma once
+
+#include "kernels_fwd.cuh"
+
+namespace bi {
+
+constexpr int kRedBlock = 256;
+
+struct RedPart {
+  double loss;
+  double d3sum;
+  float d3max;
+  int32_t pad;
+  int64_t count;
+  int64_t nonfinite;
+};
+
+struct Ctrl {          // small device-side control block at the start of the workspace
+  int64_t n_scored;    // number of scored (compact) rows
+  int32_t valid;       // offsets passed validation
+  int32_t pad;
+};
+
+// Largest i in [0, R) with off[i] <= r (off[R] > r is guaranteed by validation).
+__device__ __forceinline__ int find_response(const int64_t* __restrict__ off, int R, int64_t r) {
+  int lo = 0, hi = R - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (off[mid] <= r) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// One block.  Validates the offsets, then A_i = r_i - mean_group(r), n_i, c_i = A_i / (R* n_i)
+// in float64, the exclusive prefix of n_i and the number of scored rows.
+__global__ void k_prep(const float* __restrict__ rewards, const int64_t* __restrict__ off,
+                       const int32_t* __restrict__ goff, const int32_t* __restrict__ plen, int R, int G,
+                       double rstar, int64_t T, double* __restrict__ coef, int64_t* __restrict__ cprefix,
+                       Ctrl* ctrl, int32_t* status) {
+  __shared__ int bad;
+  if (threadIdx.x == 0) {
+    bad = 0;
+    if (off[0] != 0 || off[R] != T || goff[0] != 0 || goff[G] != R) bad = 1;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < R; i += blockDim.x) {
+    const int64_t len = off[i + 1] - off[i];
+    const int64_t pl = plen ? plen[i] : 0;
+    if (len < 0 || pl < 0 || pl > len) bad = 1;
+  }
+  for (int k = threadIdx.x; k < G; k += blockDim.x)
+    if (goff[k + 1] < goff[k]) bad = 1;
+  __syncthreads();
+  if (bad) {
+    if (threadIdx.x == 0) {
+      raise_status(status, 8 /* BI_ERR_BAD_OFFSETS */);
+      ctrl->n_scored = 0;
+      ctrl->valid = 0;
+    }
+    return;
+  }
+  for (int k = threadIdx.x; k < G; k += blockDim.x) {
+    const int a = goff[k], b = goff[k + 1];
+    double sum = 0.0;
+    for (int i = a; i < b; ++i) sum += static_cast<double>(rewards[i]);
+    const double mean = (b > a) ? sum / static_cast<double>(b - a) : 0.0;
+    for (int i = a; i < b; ++i) {
+      const double A = static_cast<double>(rewards[i]) - mean;
+      const int64_t n = (off[i + 1] - off[i]) - (plen ? plen[i] : 0);
+      coef[i] = (n > 0) ? A / (rstar * static_cast<double>(n)) : 0.0;
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int64_t acc = 0;
+    for (int i = 0; i < R; ++i) {
+      cprefix[i] = acc;
+      acc += (off[i + 1] - off[i]) - (plen ? plen[i] : 0);
+    }
+    cprefix[R] = acc;
+    ctrl->n_scored = acc;
+    ctrl->valid = 1;
+  }
+}
+
+// One thread per packed row: compact index of scored rows, and zeros in the per-row outputs of
+// prompt rows.
+__global__ void k_rowmap(const int64_t* __restrict__ off, const int32_t* __restrict__ plen, int R, int64_t T,
+                         const int64_t* __restrict__ cprefix, const Ctrl* ctrl, const int32_t* __restrict__ targets,
+                         const float* __restrict__ logmu, int32_t* __restrict__ rowmap, int32_t* __restrict__ respof,
+                         int32_t* __restrict__ y_c, float* __restrict__ logmu_c, float* __restrict__ logprob,
+                         float* __restrict__ is_weight, float* __restrict__ token_loss) {
+  const int64_t r = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (r >= T || !ctrl->valid) return;
+  const int i = find_response(off, R, r);
+  const int64_t p = r - off[i];
+  const int64_t pl = plen ? plen[i] : 0;
+  if (p < pl) {
+    logprob[r] = 0.f;
+    if (is_weight) is_weight[r] = 0.f;
+    if (token_loss) token_loss[r] = 0.f;
+    return;
+  }
+  const int64_t k = cprefix[i] + (p - pl);
+  rowmap[k] = static_cast<int32_t>(r);
+  respof[k] = i;
+  y_c[k] = targets[r];
+  logmu_c[k] = logmu[r];
+}
+
+// One warp per packed row: zero the gradient row of prompt rows.
+__global__ void k_zero_prompt_rows(const int64_t* __restrict__ off, const int32_t* __restrict__ plen, int R,
+                                   int64_t T, int H, const Ctrl* ctrl, uint16_t* __restrict__ grad_hidden) {
+  const int64_t r = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (r >= T || !ctrl->valid) return;
+  const int i = find_response(off, R, r);
+  if (r - off[i] >= plen[i]) return;
+  uint4* row = reinterpret_cast<uint4*>(grad_hidden + r * H);
+  for (int q = lane; q < H / 8; q += 32) row[q] = make_uint4(0u, 0u, 0u, 0u);
+}
+
+// One warp per compact row: copy the scored hidden rows into the compact buffer and zero the rows
+// that pad the last 128-row tile.
+__global__ void k_gather_rows(const uint16_t* __restrict__ hidden, int64_t T, int H, const Ctrl* ctrl,
+                              const int32_t* __restrict__ rowmap, uint16_t* __restrict__ hc) {
+  const int64_t k = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t ns = ctrl->n_scored;
+  const int64_t lim = ((ns + 127) / 128) * 128;
+  if (k >= T || k >= lim) return;
+  uint4* dst = reinterpret_cast<uint4*>(hc + k * H);
+  if (k < ns) {
+    const uint4* src = reinterpret_cast<const uint4*>(hidden + static_cast<int64_t>(rowmap[k]) * H);
+    for (int q = lane; q < H / 8; q += 32) dst[q] = src[q];
+  } else {
+    for (int q = lane; q < H / 8; q += 32) dst[q] = make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+__global__ void k_combine_logprob(const float* __restrict__ pm, const float* __restrict__ ps,
+                                  const float* __restrict__ pzy, int64_t T, int nchunks, int nvt, int V,
+                                  const int32_t* __restrict__ targets, float* __restrict__ logprob,
+                                  float* __restrict__ lse_out, int32_t* status) {
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (t >= T) return;
+  const int32_t y = targets[t];
+  float lse, zy;
+  combine_row(pm, ps, pzy, T, t, nchunks, nvt, y, lse, zy);
+  if (y < 0 || y >= V) {
+    raise_status(status, 6 /* BI_ERR_BAD_TARGET */);
+    logprob[t] = __int_as_float(0x7fc00000);
+  } else {
+    logprob[t] = zy - lse;
+  }
+  if (lse_out) lse_out[t] = lse;
+}
+
+// Fixed-shape block reduction of a RedPart (warp butterflies, then warps in order).
+__device__ __forceinline__ RedPart block_reduce(RedPart v) {
+  for (int o = 16; o > 0; o >>= 1) {
+    v.loss += __shfl_xor_sync(0xffffffffu, v.loss, o);
+    v.d3sum += __shfl_xor_sync(0xffffffffu, v.d3sum, o);
+    v.d3max = fmaxf(v.d3max, __shfl_xor_sync(0xffffffffu, v.d3max, o));
+    v.count += __shfl_xor_sync(0xffffffffu, v.count, o);
+    v.nonfinite += __shfl_xor_sync(0xffffffffu, v.nonfinite, o);
+  }
+  __shared__ RedPart wp[32];
+  const int w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  if ((threadIdx.x & 31) == 0) wp[w] = v;
+  __syncthreads();
+  RedPart out = wp[0];
+  if (threadIdx.x == 0) {
+    for (int i = 1; i < nw; ++i) {
+      out.loss += wp[i].loss;
+      out.d3sum += wp[i].d3sum;
+      out.d3max = fmaxf(out.d3max, wp[i].d3max);
+      out.count += wp[i].count;
+      out.nonfinite += wp[i].nonfinite;
+    }
+  }
+  return out;
+}
+
+// One thread per compact row: lse and log pi (same code as the logprob-only path), then
+// delta = log pi - log mu, w = exp(delta) (unclipped), d3 = expm1(delta) - delta,
+// token loss = -c_i w, and the per-row gradient coefficient g = token loss.
+__global__ void k_combine_is(const float* __restrict__ pm, const float* __restrict__ ps,
+                             const float* __restrict__ pzy, int64_t T, int nchunks, int nvt, int V,
+                             const Ctrl* ctrl, const int32_t* __restrict__ y_c, const float* __restrict__ logmu_c,
+                             const int32_t* __restrict__ respof, const int32_t* __restrict__ rowmap,
+                             const double* __restrict__ coef, float* __restrict__ logprob,
+                             float* __restrict__ is_weight, float* __restrict__ token_loss,
+                             float* __restrict__ lse_c, float* __restrict__ g_c, RedPart* parts, int32_t* status) {
+  const int64_t k = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t ns = ctrl->n_scored;
+  RedPart v{0.0, 0.0, -INFINITY, 0, 0, 0};
+  if (k < ns) {
+    const int32_t y = y_c[k];
+    float lse, zy;
+    combine_row(pm, ps, pzy, T, k, nchunks, nvt, y, lse, zy);
+    float lp = zy - lse;
+    if (y < 0 || y >= V) {
+      raise_status(status, 6 /* BI_ERR_BAD_TARGET */);
+      lp = __int_as_float(0x7fc00000);
+    }
+    const float delta = lp - logmu_c[k];
+    const float w = expf(delta);
+    const float d3 = expm1f(delta) - delta;
+    const float tl = static_cast<float>(-coef[respof[k]] * static_cast<double>(w));
+    const int64_t r = rowmap[k];
+    logprob[r] = lp;
+    if (is_weight) is_weight[r] = w;
+    if (token_loss) token_loss[r] = tl;
+    lse_c[k] = lse;
+    g_c[k] = tl;
+    v.loss = static_cast<double>(tl);
+    v.d3sum = static_cast<double>(d3);
+    v.d3max = d3;
+    v.count = 1;
+    v.nonfinite = isfinite(d3) ? 0 : 1;
+  }
+  const RedPart b = block_reduce(v);
+  if (threadIdx.x == 0) parts[blockIdx.x] = b;
+}
+
+// One thread per row of bi_d3_stats.
+__global__ void k_d3_partial(const float* __restrict__ lp, const float* __restrict__ mu,
+                             const uint8_t* __restrict__ mask, int64_t T, RedPart* parts) {
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  RedPart v{0.0, 0.0, -INFINITY, 0, 0, 0};
+  if (t < T && (mask == nullptr || mask[t] != 0)) {
+    const float delta = lp[t] - mu[t];
+    const float d3 = expm1f(delta) - delta;
+    v.d3sum = static_cast<double>(d3);
+    v.d3max = d3;
+    v.count = 1;
+    v.nonfinite = isfinite(d3) ? 0 : 1;
+  }
+  const RedPart b = block_reduce(v);
+  if (threadIdx.x == 0) parts[blockIdx.x] = b;
+}
+
+// One block: sum the block partials in a fixed order; write loss and D3 statistics.
+struct D3Out {
+  float mean;
+  float max;
+  int64_t count;
+  int64_t n_nonfinite;
+};
+
+__global__ void k_reduce_parts(const RedPart* __restrict__ parts, int nparts, float* loss, D3Out* d3,
+                               int32_t* status) {
+  RedPart v{0.0, 0.0, -INFINITY, 0, 0, 0};
+  for (int i = threadIdx.x; i < nparts; i += blockDim.x) {
+    const RedPart p = parts[i];
+    v.loss += p.loss;
+    v.d3sum += p.d3sum;
+    v.d3max = fmaxf(v.d3max, p.d3max);
+    v.count += p.count;
+    v.nonfinite += p.nonfinite;
+  }
+  const RedPart b = block_reduce(v);
+  if (threadIdx.x == 0) {
+    if (loss) *loss = static_cast<float>(b.loss);
+    if (d3) {
+      D3Out o;
+      o.mean = (b.count > 0) ? static_cast<float>(b.d3sum / static_cast<double>(b.count)) : 0.f;
+      o.max = (b.count > 0) ? b.d3max : 0.f;
+      o.count = b.count;
+      o.n_nonfinite = b.nonfinite;
+      *d3 = o;
+    }
+    if (b.nonfinite > 0 || (loss && !isfinite(b.loss))) raise_status(status, 7 /* BI_ERR_NONFINITE */);
+  }
+}
+
+}  // namespace bi

@@ -1,0 +1,342 @@
+#!/usr/bin/env python
+"""Throughput of the fused token-logprob + unclipped IS-loss forward+backward on B200.
+
+One step = one call of bi_is_loss_fwd_bwd over one synthetic batch with the shapes of the
+1.5B-parameter workload (H = 1536, V = 151936, 8 groups x 8 responses of U[256, 2048] tokens):
+forward logits + log-softmax + target gather, IS weight, D3, advantages, loss, dH and dW.
+Inputs (hidden 0.2 GB, W 0.47 GB) are larger than the 126 MB L2, so no flush is needed between
+steps.  Prints one JSON line (rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs one process per GPU (torchrun): each rank scores its own batch (weak scaling) and the
+ranks sum dW and the three loss/D3 scalars with NCCL, the one exchange step of data parallelism.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "fused logprob+IS-loss fwd+bwd tokens/s at H1536 V151936; % bf16 tensor peak"
+UNIT = "tokens/s"
+CONFIG = "qwen1.5b"
+CPU_SAMPLE_ROWS = 1024
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def sub_batch(b, nrows):
+    """The first `nrows` packed rows with the responses and groups that cover them (host tensors)."""
+    off = b.resp_offsets.cpu().numpy()
+    goff = b.group_offsets.cpu().numpy()
+    keep = int(np.searchsorted(off, nrows, side="left"))  # responses starting before nrows
+    new_off = np.minimum(off[:keep + 1], nrows)
+    if new_off[-1] < nrows:
+        new_off = np.append(new_off, nrows)
+    R = len(new_off) - 1
+    new_goff = [0]
+    for g in range(len(goff) - 1):
+        hi = min(goff[g + 1], R)
+        if hi > new_goff[-1]:
+            new_goff.append(hi)
+        if hi >= R:
+            break
+    return new_off, np.array(new_goff), b.rewards.cpu().numpy()[:R]
+
+
+def cpu_oracle_sample(b, logmu_host, nrows):
+    """Time the fp64 oracle (test infrastructure) on a bounded slice of the same workload."""
+    from oracle import isloss_oracle as orc
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max((d.get("num_threads", 1) for d in threadpool_info()), default=os.cpu_count())
+    except Exception:  # pragma: no cover
+        cores = os.cpu_count()
+    off, goff, rew = sub_batch(b, nrows)
+    h = b.hidden[:nrows].cpu()
+    w = b.w.cpu()
+    y = b.targets[:nrows].cpu()
+    t0 = time.perf_counter()
+    orc.is_loss_fwd_bwd(h, w, y, logmu_host[:nrows].astype(np.float64), rew, off, goff)
+    dt = time.perf_counter() - t0
+    return {"value": nrows / dt, "unit": UNIT, "cores": int(cores), "kind": "oracle",
+            "sample": f"first {nrows} rows of the {CONFIG} batch (fwd + loss + dH + dW in fp64 NumPy), {dt:.1f} s"}
+
+
+def run_reference(args):
+    """--impl reference: the fp64 CPU oracle on the machine's host cores, a bounded slice per step."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    from workloads import make_batch, spec_for
+    from oracle import isloss_oracle as orc
+    b = make_batch(spec_for(CONFIG))
+    nrows = 256
+    lp_roll, _ = orc.token_logprob(b.hidden[:nrows], b.w_roll, b.targets[:nrows])
+    logmu = lp_roll + b.logmu_noise[:nrows].double().numpy()
+    times = []
+    for i in range(args.warmup + args.steps):
+        r = cpu_oracle_sample(b, logmu, nrows)
+        if i >= args.warmup:
+            times.append(nrows / r["value"])
+    ms = 1e3 * statistics.mean(times)
+    val = nrows / (ms * 1e-3)
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"{CONFIG}: H=1536 V=151936, {nrows}-row slice per step on host cores"},
+            "cpu_baseline": {"value": val, "unit": UNIT, "cores": r["cores"], "kind": "oracle",
+                             "sample": f"first {nrows} rows of the {CONFIG} batch per step"},
+            "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args):
+    rank, world, local = dist_env()
+    import async_rl_b200 as bi
+    from async_rl_b200.build import build
+    from workloads import make_batch, spec_for
+
+    if rank == 0:
+        build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        dist.barrier()
+        pg = dist
+    spec = spec_for(CONFIG)
+    b = make_batch(spec, seed=1234 + spec.index + 1000 * rank, device=dev)
+    T, H, V, R = b.n_rows, spec.H, spec.V, b.R
+    # rollout log-probabilities from the lagged head (the rollout engine's role), plus noise rows
+    logmu, _, st = bi.logprob_fwd(b.hidden, b.w_roll, b.targets)
+    logmu += b.logmu_noise
+    bi.check_status(st)
+    b.w_roll = None
+    ws = bi.make_workspace(T, H, V, R, dev)
+    out = bi.LossOutputs.allocate(T, H, V, dev)
+    rnorm = float(R * world)
+
+    def step():
+        bi.is_loss_fwd_bwd(b.hidden, b.w, b.targets, logmu, b.rewards, b.resp_offsets, b.group_offsets,
+                           None, rnorm, ws=ws, out=out)
+        if pg is not None:
+            pg.all_reduce(out.grad_w)
+            pg.all_reduce(out.loss)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    bi.check_status(out.status)
+
+    clocks = ClockSampler(local)
+    if pg is not None:
+        pg.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    bi.profile_reset()
+    bi.profile_enable(True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    bi.profile_enable(False)
+    if pg is not None:
+        pg.barrier()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    prof = bi.profile_read()
+    bi.check_status(out.status)
+
+    tok = torch.tensor([float(T), ms], dtype=torch.float64, device=dev)
+    if pg is not None:
+        tot = tok[:1].clone()
+        pg.all_reduce(tot)
+        mx = tok[1:].clone()
+        pg.all_reduce(mx, op=pg.ReduceOp.MAX)
+        total_tokens, ms_max = float(tot.item()), float(mx.item())
+    else:
+        total_tokens, ms_max = float(T), ms
+    value = total_tokens / (ms_max * 1e-3)
+
+    # end to end through the public API with host buffers (pinned), per-step H2D + D2H
+    e2e = None
+    if not args.no_e2e:
+        host = {k: getattr(b, k).cpu().pin_memory() for k in ("hidden", "targets", "rewards", "resp_offsets",
+                                                              "group_offsets")}
+        host["logmu"] = logmu.cpu().pin_memory()
+        dbuf = {k: torch.empty_like(v, device=dev) for k, v in host.items()}
+        loss_h = torch.empty(1, dtype=torch.float32).pin_memory()
+        d3_h = torch.empty(24, dtype=torch.uint8).pin_memory()
+        h2d = sum(v.numel() * v.element_size() for v in host.values())
+        d2h = loss_h.numel() * 4 + d3_h.numel()
+
+        def e2e_step():
+            for k in host:
+                dbuf[k].copy_(host[k], non_blocking=True)
+            bi.is_loss_fwd_bwd(dbuf["hidden"], b.w, dbuf["targets"], dbuf["logmu"], dbuf["rewards"],
+                               dbuf["resp_offsets"], dbuf["group_offsets"], None, rnorm, ws=ws, out=out)
+            if pg is not None:
+                pg.all_reduce(out.grad_w)
+                pg.all_reduce(out.loss)
+            loss_h.copy_(out.loss, non_blocking=True)
+            d3_h.copy_(out.d3_raw, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record()
+        for _ in range(args.steps):
+            e2e_step()
+        f1.record()
+        torch.cuda.synchronize()
+        ems = torch.tensor([f0.elapsed_time(f1) / args.steps], dtype=torch.float64, device=dev)
+        if pg is not None:
+            pg.all_reduce(ems, op=pg.ReduceOp.MAX)
+        e2e = {"value": total_tokens / (float(ems.item()) * 1e-3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(d2h)}
+
+    peaks, peak_src = measured_peaks()
+    peak_tf = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    flops_tvh = 2.0 * T * V * H  # one LM-head contraction over the batch
+    alg = {"k_fwd_logits": flops_tvh, "k_bwd_dh": flops_tvh, "k_bwd_dw": flops_tvh}
+    executed = {"k_fwd_logits": flops_tvh, "k_bwd_dh": 2 * flops_tvh, "k_bwd_dw": 2 * flops_tvh}
+    dom = max(alg, key=lambda k: prof.get(k, (0.0, 1))[0])
+    dms, dn = prof.get(dom, (float("nan"), 1))
+    davg = dms / max(dn, 1)
+    achieved = alg[dom] / (davg * 1e-3) / 1e12
+    step_tflops = 6.0 * T * V * H / (ms * 1e-3) / 1e12
+    kernels = {k: {"ms_per_launch": v[0] / max(v[1], 1), "launches": v[1]} for k, v in prof.items()}
+    launches = int(sum(v[1] for v in prof.values()))
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"{CONFIG}: H={H} V={V}, {spec.groups}x{spec.per_group} responses "
+                                   f"U[{spec.len_lo},{spec.len_hi}] rows, T={T} scored rows per rank",
+                       "global_batch_tokens": int(total_tokens), "parallelism": f"dp{world}",
+                       "l2": "inputs larger than L2 (hidden 0.23 GB, W 0.47 GB); no flush"},
+            "pct_bf16_peak": 100.0 * step_tflops / peak_tf,
+            "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak_tf,
+                         "unit": "TFLOP/s", "frac": achieved / peak_tf, "traffic": None,
+                         "peak_source": f"{peak_src} bf16_tflops_sustained",
+                         "algorithmic_flops_per_launch": alg[dom],
+                         "executed_frac": executed[dom] / (davg * 1e-3) / 1e12 / peak_tf},
+            "step_roofline": {"achieved": step_tflops, "frac": step_tflops / peak_tf,
+                              "algorithmic_flops": 6.0 * T * V * H, "unit": "TFLOP/s"},
+            "kernels": kernels, "gpu_launches": launches, "clocks": clk, "e2e": e2e}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_oracle_sample(b, logmu.cpu().double().numpy(), CPU_SAMPLE_ROWS)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.barrier()
+        pg.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

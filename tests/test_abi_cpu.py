@@ -1,0 +1,105 @@
+"""The C-ABI library loads and exports every symbol the header declares; host-side argument
+checks return their error codes before any CUDA call.  No GPU needed."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from async_rl_b200 import _lib
+from async_rl_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "bi_isloss.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return _lib.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(bi_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for must in ("bi_logprob_fwd", "bi_is_loss_fwd_bwd", "bi_d3_stats", "bi_workspace_bytes", "bi_status_string"):
+        assert must in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert set(_lib.EXPORTED) <= set(declared_functions())
+
+
+def test_status_strings(lib):
+    for code, name in _lib.STATUS_NAMES.items():
+        assert lib.bi_status_string(code).decode() == name
+    assert lib.bi_status_string(99).decode() == "BI_UNKNOWN"
+    assert lib.bi_version() >= 100
+
+
+def test_workspace_bytes_monotone(lib):
+    a = lib.bi_workspace_bytes(1000, 1536, 151936, 0)
+    b = lib.bi_workspace_bytes(2000, 1536, 151936, 0)
+    c = lib.bi_workspace_bytes(2000, 1536, 151936, 64)
+    assert 0 < a < b < c
+    assert lib.bi_workspace_bytes(-1, 128, 512, 0) == 0
+    # the compact copy of the hidden states is part of the loss workspace
+    assert c - b >= 2000 * 1536 * 2
+
+
+FAKE = 1 << 20  # aligned non-null address; never dereferenced on the paths below
+
+
+def test_logprob_argument_checks(lib):
+    st = FAKE
+    ws_bytes = lib.bi_workspace_bytes(10, 128, 512, 0)
+    # NULL hidden
+    assert lib.bi_logprob_fwd(None, FAKE, FAKE, 10, 128, 512, FAKE, None, st, FAKE, ws_bytes, None) == 1
+    # misaligned hidden
+    assert lib.bi_logprob_fwd(FAKE + 2, FAKE, FAKE, 10, 128, 512, FAKE, None, st, FAKE, ws_bytes, None) == 1
+    # unsupported H
+    assert lib.bi_logprob_fwd(FAKE, FAKE, FAKE, 10, 100, 512, FAKE, None, st, FAKE, ws_bytes, None) == 2
+    assert lib.bi_logprob_fwd(FAKE, FAKE, FAKE, 10, 448, 512, FAKE, None, st, FAKE, ws_bytes, None) == 2
+    # workspace too small / missing / misaligned
+    assert lib.bi_logprob_fwd(FAKE, FAKE, FAKE, 10, 128, 512, FAKE, None, st, FAKE, ws_bytes - 1, None) == 3
+    assert lib.bi_logprob_fwd(FAKE, FAKE, FAKE, 10, 128, 512, FAKE, None, st, None, ws_bytes, None) == 3
+    assert lib.bi_logprob_fwd(FAKE, FAKE, FAKE, 10, 128, 512, FAKE, None, st, FAKE + 16, ws_bytes, None) == 3
+    # negative sizes
+    assert lib.bi_logprob_fwd(FAKE, FAKE, FAKE, -1, 128, 512, FAKE, None, st, FAKE, ws_bytes, None) == 1
+    assert lib.bi_logprob_fwd(FAKE, FAKE, FAKE, 10, 128, 0, FAKE, None, st, FAKE, ws_bytes, None) == 1
+
+
+def test_is_loss_argument_checks(lib):
+    T, H, V, R = 40, 128, 512, 4
+    ws_bytes = lib.bi_workspace_bytes(T, H, V, R)
+    args = [FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, R, 2, 0.0, T, H, V,
+            FAKE, FAKE, None, None, None, FAKE, FAKE, FAKE, FAKE, ws_bytes, None]
+
+    def call(**kw):
+        a = list(args)
+        idx = {"hidden": 0, "R": 8, "G": 9, "rnorm": 10, "H": 12, "grad_w": 20, "ws_bytes": 23, "loss": 14}
+        for k, v in kw.items():
+            a[idx[k]] = v
+        return lib.bi_is_loss_fwd_bwd(*a)
+
+    assert call(hidden=None) == 1
+    assert call(R=0) == 1
+    assert call(G=5) == 1          # more groups than responses
+    assert call(rnorm=-1.0) == 1
+    assert call(loss=None) == 1
+    assert call(grad_w=FAKE + 4) == 1  # misaligned
+    assert call(H=448) == 2            # 7 * 64: no split into <= 384-column multiples of 64
+    assert call(ws_bytes=ws_bytes - 1) == 3
+
+
+def test_d3_argument_checks(lib):
+    assert lib.bi_d3_stats(None, FAKE, None, 10, FAKE, FAKE, FAKE, 256, None) == 1
+    assert lib.bi_d3_stats(FAKE, FAKE, None, 10, None, FAKE, FAKE, 256, None) == 1
+    assert lib.bi_d3_stats(FAKE, FAKE, None, 1000, FAKE, FAKE, FAKE, 16, None) == 3

@@ -1,0 +1,142 @@
+"""Parity of the CUDA path against the fp64 oracle on the same seeded inputs.
+
+Sizes span several tiles and ragged tails (rows not a multiple of 128, vocabularies not a
+multiple of 256 or 32) and include the full H = 1536, V = 151936 head."""
+import numpy as np
+import pytest
+import torch
+
+import async_rl_b200 as bi
+from oracle import isloss_oracle as orc
+from workloads import make_batch, spec_for
+from workloads.synth import random_inputs
+
+from .util import GRAD_TOL, LOGPROB_TOL, LOSS_TOL, assert_close, assert_grad_close, f64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from async_rl_b200.build import build
+    build()
+
+
+def _logprob_case(T, H, V, seed, cuda_device, w_std=0.02):
+    h, w, y = random_inputs(T, H, V, seed, w_std=w_std)
+    lp_ref, lse_ref = orc.token_logprob(h, w, y)
+    lp, lse, st = bi.logprob_fwd(h.to(cuda_device), w.to(cuda_device), y.to(cuda_device), want_lse=True)
+    torch.cuda.synchronize()
+    bi.check_status(st)
+    assert_close("logprob", f64(lp), lp_ref, LOGPROB_TOL, LOGPROB_TOL)
+    assert_close("lse", f64(lse), lse_ref, LOGPROB_TOL, LOGPROB_TOL)
+    return lp
+
+
+@pytest.mark.parametrize("T,H,V", [(1, 128, 512), (7, 128, 549), (160, 128, 512), (300, 256, 1000),
+                                   (129, 192, 4133), (257, 1536, 151936)])
+def test_logprob_matches_oracle(T, H, V, cuda_device):
+    _logprob_case(T, H, V, seed=T * 7 + H + V, cuda_device=cuda_device)
+
+
+def test_logprob_peaky_logits(cuda_device):
+    """Large logits (W ~ N(0, 0.5)): the running max moves across chunks; no overflow."""
+    _logprob_case(200, 256, 3001, seed=5, cuda_device=cuda_device, w_std=0.5)
+
+
+def test_logprob_empty_batch(cuda_device):
+    h = torch.empty(0, 128, dtype=torch.bfloat16, device=cuda_device)
+    w = torch.zeros(512, 128, dtype=torch.bfloat16, device=cuda_device)
+    y = torch.empty(0, dtype=torch.int32, device=cuda_device)
+    lp, _, st = bi.logprob_fwd(h, w, y)
+    torch.cuda.synchronize()
+    bi.check_status(st)
+    assert lp.numel() == 0
+
+
+def test_logprob_uniform_closed_form(cuda_device):
+    """W = 0: every logit is 0 and log pi = -log V for every row."""
+    T, H, V = 130, 128, 1000
+    h = torch.randn(T, H).to(torch.bfloat16).to(cuda_device)
+    w = torch.zeros(V, H, dtype=torch.bfloat16, device=cuda_device)
+    y = torch.randint(0, V, (T,), dtype=torch.int32).to(cuda_device)
+    lp, _, st = bi.logprob_fwd(h, w, y)
+    torch.cuda.synchronize()
+    bi.check_status(st)
+    assert np.allclose(f64(lp), -np.log(V), rtol=0, atol=2e-6)
+
+
+def test_bad_target_sets_status(cuda_device):
+    h, w, y = random_inputs(10, 128, 512, seed=1)
+    y[3] = 512
+    lp, _, st = bi.logprob_fwd(h.to(cuda_device), w.to(cuda_device), y.to(cuda_device))
+    torch.cuda.synchronize()
+    assert int(st.item()) == 6
+    assert np.isnan(f64(lp)[3]) and np.isfinite(np.delete(f64(lp), 3)).all()
+
+
+def _loss_case(batch, cuda_device, rollout_lp=None, resp_normalizer=0.0, check_dw=True):
+    b = batch
+    if rollout_lp is None:
+        rollout_lp, _ = orc.token_logprob(b.hidden, b.w_roll, b.targets)
+        rollout_lp = rollout_lp + b.logmu_noise.double().numpy()
+    mu = torch.tensor(rollout_lp, dtype=torch.float32)
+    mu64 = mu.double().numpy()   # the oracle sees exactly the fp32 values the GPU sees
+    ref = orc.is_loss_fwd_bwd(b.hidden, b.w, b.targets, mu64, b.rewards, b.resp_offsets, b.group_offsets,
+                              b.prompt_lens, resp_normalizer, want_grad_w=check_dw)
+    d = b.to(cuda_device)
+    out = bi.is_loss_fwd_bwd(d.hidden, d.w, d.targets, mu.to(cuda_device), d.rewards, d.resp_offsets,
+                             d.group_offsets, d.prompt_lens, resp_normalizer)
+    torch.cuda.synchronize()
+    bi.check_status(out.status)
+    assert_close("loss", f64(out.loss), [ref["loss"]], LOSS_TOL, LOSS_TOL)
+    # tighter: the loss error is small against the sum of |token losses|
+    scale = float(np.sum(np.abs(ref["token_loss"])))
+    assert abs(float(out.loss.item()) - ref["loss"]) <= 1e-4 * scale + 1e-9
+    assert_close("logprob", f64(out.logprob), ref["logprob"], LOGPROB_TOL, LOGPROB_TOL)
+    assert_close("is_weight", f64(out.is_weight), ref["is_weight"], LOGPROB_TOL, LOGPROB_TOL)
+    assert_close("token_loss", f64(out.token_loss), ref["token_loss"], LOSS_TOL * np.max(np.abs(ref["token_loss"])),
+                 LOSS_TOL)
+    d3 = out.d3()
+    assert d3["count"] == ref["d3"]["count"] and d3["n_nonfinite"] == 0
+    assert_close("d3.mean", [d3["mean"]], [ref["d3"]["mean"]], 1e-7, 5e-2)
+    assert_grad_close("grad_hidden", f64(out.grad_hidden), ref["grad_hidden"])
+    if check_dw:
+        assert_grad_close("grad_w", f64(out.grad_w), ref["grad_w"])
+    return out, ref
+
+
+def test_loss_tiny(cuda_device):
+    _loss_case(make_batch(spec_for("tiny")), cuda_device)
+
+
+def test_loss_tiny_prompt_masked_and_normaliser(cuda_device):
+    spec = spec_for("tiny", prompt_len=5)
+    _loss_case(make_batch(spec), cuda_device, resp_normalizer=13.0)
+
+
+def test_loss_odd_shapes(cuda_device):
+    """V not a multiple of 32, rows not a multiple of 128, groups of unequal size, an empty response."""
+    spec = spec_for("tiny", V=549, H=192, groups=3, per_group=3, len_lo=1, len_hi=70)
+    b = make_batch(spec, lengths=[37, 0, 64, 129, 5, 1, 70, 33, 2])
+    b.group_offsets = torch.tensor([0, 2, 3, 9], dtype=torch.int32)
+    _loss_case(b, cuda_device)
+
+
+def test_loss_cluster_split_h2048(cuda_device):
+    """H = 2048: eight CTAs share each tile (256 columns each)."""
+    spec = spec_for("tiny", H=2048, V=3000, groups=2, per_group=2, len_lo=40, len_hi=150)
+    _loss_case(make_batch(spec), cuda_device)
+
+
+def test_loss_cluster_split_h2560(cuda_device):
+    """H = 2560: 320 columns per CTA, two MMA column chunks of 192 and 128."""
+    spec = spec_for("tiny", H=2560, V=2000, groups=2, per_group=2, len_lo=40, len_hi=150, prompt_len=16)
+    _loss_case(make_batch(spec), cuda_device)
+
+
+@pytest.mark.slow
+def test_loss_full_head_1536(cuda_device):
+    """Full H = 1536, V = 151936 LM head with a few hundred rows over several tiles."""
+    spec = spec_for("qwen1.5b", groups=2, per_group=2, len_lo=60, len_hi=130)
+    _loss_case(make_batch(spec), cuda_device)
