@@ -4,4 +4,5 @@ The compute path is the CUDA library ``libbi_isloss.so`` behind the C ABI in
 ``include/bi_isloss.h``; this package only loads it and marshals tensors.
 """
 from .api import (BiError, LossOutputs, check_status, d3_stats, decode_d3, debug_force_timeout_once,  # noqa: F401
-                  is_loss_fwd_bwd, logprob_fwd, make_workspace, workspace_bytes)
+                  is_loss_fwd_bwd, logprob_fwd, make_workspace, profile_enable, profile_read, profile_reset,
+                  workspace_bytes)
