@@ -9,7 +9,7 @@
 #include <mutex>
 #include <vector>
 
-#include "../../include/bi_isloss.h"
+#include "bi_isloss.h"
 #include "kernels_bwd.cuh"
 #include "kernels_fwd.cuh"
 #include "kernels_small.cuh"
@@ -441,10 +441,9 @@ bi_status bi_is_loss_fwd_bwd(const uint16_t* hidden, const uint16_t* w_lm, const
   a.V = V;
   a.C = C;
   a.Hs = H / C;
-  const int su = a.Hs / 64;
-  a.nchunk = su > 4 ? 2 : 1;
-  a.chunk_units[0] = a.nchunk == 2 ? (su + 1) / 2 : su;
-  a.chunk_units[1] = a.nchunk == 2 ? su / 2 : 0;
+  const int su = a.Hs / 64;  // 64-column units of the slice: chunks of two units, a last one of one
+  a.nchunk = (su + 1) / 2;
+  for (int c = 0; c < bi::kMaxChunks; ++c) a.chunk_units[c] = c < a.nchunk ? ((2 * c + 1 < su) ? 2 : 1) : 0;
   a.T = trows;
   a.d_rows = d_rows;
   a.nvt128 = (V + 127) / 128;

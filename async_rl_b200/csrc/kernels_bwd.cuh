@@ -15,64 +15,98 @@
 // Tile shape, K order and the order of the reduction are fixed and independent of T, so each
 // row of dH has the same bits in any batch (the "Zero Mismatch" post, "Alignment permits a
 // simpler learning path": bit-identical rows for the same weights and tokens).
+//
+// Issue-loop design: the single issuing lane is the critical resource (a tcgen05.mma takes 64-96
+// tensor cycles here), so the MMA and TMA warps run converged loops with position counters (no
+// integer division), precomputed descriptors, and one commit per 32 KB shared-memory slot.
 #pragma once
 
 #include "sm100.cuh"
 
 namespace bi {
 
-constexpr int kUnitBytes = 16384;  // one [128 rows][64 bf16] 128B-swizzled tile
-constexpr int kRing = 13;          // shared-memory ring of units
-constexpr int kBwdSmemBytes = kRing * kUnitBytes + 1024;
+constexpr int kUnitBytes = 16384;             // one [128 rows][64 bf16] 128B-swizzled tile
+constexpr int kSlotBytes = 2 * kUnitBytes;    // ring slot: two units, one barrier pair
+constexpr int kSlots = 7;
 constexpr int kBwdThreads = 192;
-constexpr int kZCol = 384;          // TMEM column of the 128-column logit accumulator
-constexpr int kSlotsPerCta = 2;     // dZ scratch slots per producer CTA
+constexpr int kZCol = 384;                    // TMEM column of the 128-column logit accumulator
+constexpr int kSlotsPerCta = 2;               // dZ scratch slots per producer CTA
 constexpr int kMaxCluster = 8;
 constexpr int kMaxSlots = kMaxCluster * kSlotsPerCta;
+constexpr int kMaxChunks = 3;                 // slice update chunks of <= 128 columns (H / C <= 384)
 
 enum BwdMode : int { kModeDH = 0, kModeDW = 1 };
 
 struct BwdArgs {
   int32_t H, V;
-  int32_t C;              // CTAs per cluster
-  int32_t Hs;             // H / C: columns owned by each CTA
-  int32_t nchunk;         // MMA column chunks of the slice update (1 or 2)
-  int32_t chunk_units[2]; // 64-column units per chunk
-  int64_t T;              // rows of the compact hidden-state tensor map (upper bound)
-  const int64_t* d_rows;  // number of valid compact rows (device)
-  int32_t nvt128;         // ceil(V / 128)
-  const float* lse;       // [rows] compact
-  const float* g;         // [rows] compact: -c_i w_t (0 for rows without gradient)
-  const int32_t* y;       // [rows] compact targets
-  const int32_t* rowmap;  // [rows] compact row -> output row of grad_hidden
-  uint16_t* grad_hidden;  // [*, H] bf16 (kModeDH)
-  float* grad_w;          // [V, H] fp32 (kModeDW)
-  uint16_t* dz_scratch;   // [clusters * C * kSlotsPerCta * 128][128] bf16
+  int32_t C;                      // CTAs per cluster
+  int32_t Hs;                     // H / C: columns owned by each CTA
+  int32_t nchunk;                 // slice-update chunks (<= 3)
+  int32_t chunk_units[kMaxChunks];// 64-column units per chunk (1 or 2)
+  int64_t T;                      // rows of the compact hidden-state tensor map (upper bound)
+  const int64_t* d_rows;          // number of valid compact rows (device)
+  int32_t nvt128;                 // ceil(V / 128)
+  const float* lse;               // [rows] compact
+  const float* g;                 // [rows] compact: -c_i w_t (0 for rows without gradient)
+  const int32_t* y;               // [rows] compact targets
+  const int32_t* rowmap;          // [rows] compact row -> output row of grad_hidden
+  uint16_t* grad_hidden;          // [*, H] bf16 (kModeDH)
+  float* grad_w;                  // [V, H] fp32 (kModeDW)
+  uint16_t* dz_scratch;           // [clusters * C * kSlotsPerCta * 128][128] bf16
   int32_t* status;
   uint64_t limit_ns;
 };
 
 struct BwdShared {
-  uint64_t full[kRing];
-  uint64_t empty[kRing];
+  uint64_t full[kSlots];
+  uint64_t empty[kSlots];
   uint64_t z_full, z_empty, o_full, o_empty, mma_done;
-  uint64_t ep_bar;       // rendezvous of the 128 epilogue threads (bounded, unlike bar.sync)
+  uint64_t ep_bar;                // rendezvous of the 128 epilogue threads (bounded, unlike bar.sync)
   uint64_t dz_ready[kMaxSlots];
   uint64_t dz_free[kMaxSlots];
-  float col_lse2[128];   // kModeDW: per-column lse * log2(e)
-  float col_g[128];      // kModeDW: per-column g
-  int32_t col_y[128];    // kModeDW: per-column target (INT32_MIN: column not valid)
+  float col_lse2[128];            // kModeDW: per-column lse * log2(e)
+  float col_g[128];               // kModeDW: per-column g
+  int32_t col_y[128];             // kModeDW: per-column target (INT32_MIN: column not valid)
   uint32_t tmem_base;
   volatile uint32_t abort_flag;
+};
+
+constexpr int kBwdSmemBytes = kSlots * kSlotBytes + static_cast<int>((sizeof(BwdShared) + 127) / 128 * 128);
+
+__device__ __forceinline__ bool elect_one() {
+  uint32_t p;
+  asm volatile(
+      "{\n\t.reg .pred q;\n\t.reg .b32 r;\n\t"
+      "elect.sync r|q, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(p));
+  return p != 0;
+}
+
+// Position in a cluster's step stream, advanced without division.
+struct StreamPos {
+  int64_t s;        // stream index
+  int u_idx;        // index of the unit among this cluster's units
+  int j;            // step inside the unit
+  uint32_t modc;    // s mod C  (the producer CTA of step s)
+  uint32_t slot;    // s mod (C * kSlotsPerCta)  (dZ scratch slot)
+  uint32_t round;   // s div (C * kSlotsPerCta)
+  __device__ __forceinline__ void zero() { s = 0; u_idx = 0; j = 0; modc = 0; slot = 0; round = 0; }
+  __device__ __forceinline__ void next(int steps, uint32_t C, uint32_t nslot) {
+    ++s;
+    if (++j == steps) { j = 0; ++u_idx; }
+    if (++modc == C) modc = 0;
+    if (++slot == nslot) { slot = 0; ++round; }
+  }
 };
 
 template <int kMode>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     k_bwd_cluster(const __grid_constant__ CUtensorMap tm_stat, const __grid_constant__ CUtensorMap tm_stream,
                   const __grid_constant__ CUtensorMap tm_dz, BwdArgs a) {
-  extern __shared__ uint8_t dsmem_raw[];
-  uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ BwdShared sh;
+  extern __shared__ __align__(1024) uint8_t dsmem[];
+  uint8_t* ring = dsmem;
+  BwdShared& sh = *reinterpret_cast<BwdShared*>(dsmem + kSlots * kSlotBytes);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -83,7 +117,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t nslot = C * kSlotsPerCta;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kRing; ++i) {
+    for (int i = 0; i < kSlots; ++i) {
       mbar_init(&sh.full[i], 1);
       mbar_init(&sh.empty[i], 1);
     }
@@ -110,7 +144,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   tc_fence_after();
   const uint32_t tmem = sh.tmem_base;
 
-  // On a timeout, stop this CTA and its peers (their own waits would run out later anyway).
+  // Bounded wait with a warp-uniform outcome.  On a timeout, stop this CTA and its peers.
   auto wait = [&](uint64_t* bar, uint32_t parity, bool cluster_acq) -> bool {
     const WaitCtl wc{&sh.abort_flag, a.status, a.limit_ns};
     const bool ok = cluster_acq ? mbar_wait<true>(bar, parity, wc) : mbar_wait<false>(bar, parity, wc);
@@ -118,170 +152,195 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const uint32_t la = smem_u32(const_cast<uint32_t*>(&sh.abort_flag));
       for (uint32_t q = 0; q < C; ++q) st_cluster_u32(mapa_shared(la, q), 1u);
     }
-    return ok;
+    return __all_sync(0xffffffffu, ok) != 0;
   };
 
-  const int64_t rows = *a.d_rows;
+  const uint32_t ring_base = smem_u32(ring);
+  // the 128B-swizzled tiles need 1024-byte aligned slots; refuse to run otherwise
+  const bool misaligned = (ring_base & 1023u) != 0;
+  if (misaligned && threadIdx.x == 0) raise_status(a.status, 4 /* BI_ERR_CUDA */);
+  const int64_t rows = misaligned ? 0 : *a.d_rows;
   const int mtiles = static_cast<int>((rows + 127) / 128);
-  const int nunits = (kMode == kModeDH) ? mtiles : a.nvt128;
+  const int nunits = misaligned ? 0 : ((kMode == kModeDH) ? mtiles : a.nvt128);
   const int steps = (kMode == kModeDH) ? a.nvt128 : mtiles;
-  const int my_units = (static_cast<int>(cl) < nunits) ? (nunits - static_cast<int>(cl) + static_cast<int>(ncl) - 1) / static_cast<int>(ncl) : 0;
+  const int my_units =
+      (static_cast<int>(cl) < nunits) ? (nunits - static_cast<int>(cl) + static_cast<int>(ncl) - 1) / static_cast<int>(ncl) : 0;
   const int64_t total = static_cast<int64_t>(my_units) * steps;
   const int KB = a.H / 64;
   const int slice0 = static_cast<int>(rank) * a.Hs;
-  auto own = [&](int64_t s) { return static_cast<uint32_t>(s % C) == rank; };
-  auto unit_of = [&](int64_t s) { return static_cast<int>(cl) + static_cast<int>(s / steps) * static_cast<int>(ncl); };
 
   if (warp == 0) {
-    if (lane == 0) {
-      // ---------------- TMA producer ----------------
+    // ---------------- TMA producer (whole warp; one elected lane issues) ----------------
+    if (elect_one()) {
       tma_prefetch_desc(&tm_stat);
       tma_prefetch_desc(&tm_stream);
       tma_prefetch_desc(&tm_dz);
-      uint32_t pos = 0;
-      bool ok = true;
-      auto load_unit = [&](const CUtensorMap* m, int x, int y) {
-        const uint32_t st = pos % kRing, ph = (pos / kRing) & 1u;
-        if (!wait(&sh.empty[st], ph ^ 1u, false)) return false;
-        mbar_arrive_expect_tx(&sh.full[st], kUnitBytes);
-        tma_load_2d(smem_u32(ring + st * kUnitBytes), m, &sh.full[st], x, y);
-        ++pos;
-        return true;
-      };
-      auto pad_unit = [&]() {
-        const uint32_t st = pos % kRing, ph = (pos / kRing) & 1u;
-        if (!wait(&sh.empty[st], ph ^ 1u, false)) return false;
-        mbar_arrive(&sh.full[st]);
-        ++pos;
-        return true;
-      };
-      auto ztile = [&](int64_t s) {
-        const int u = unit_of(s), j = static_cast<int>(s % steps);
-        for (int kb = 0; kb < KB; ++kb) {
-          if (!load_unit(&tm_stat, kb * 64, u * 128)) return false;
-          if (!load_unit(&tm_stream, kb * 64, j * 128)) return false;
+    }
+    uint32_t slot = 0, phase = 0;
+    auto acquire = [&](uint32_t bytes) -> bool {
+      if (!wait(&sh.empty[slot], phase ^ 1u, false)) return false;
+      if (elect_one()) mbar_arrive_expect_tx(&sh.full[slot], bytes);
+      return true;
+    };
+    auto advance = [&]() {
+      if (++slot == kSlots) { slot = 0; phase ^= 1u; }
+    };
+    auto ztile = [&](const StreamPos& p) -> bool {
+      const int ustat = (static_cast<int>(cl) + p.u_idx * static_cast<int>(ncl)) * 128;
+      const int ystr = p.j * 128;
+      for (int kb = 0; kb < KB; ++kb) {
+        if (!acquire(kSlotBytes)) return false;
+        if (elect_one()) {
+          const uint32_t dst = ring_base + slot * kSlotBytes;
+          tma_load_2d(dst, &tm_stat, &sh.full[slot], kb * 64, ustat);
+          tma_load_2d(dst + kUnitBytes, &tm_stream, &sh.full[slot], kb * 64, ystr);
         }
-        return true;
-      };
-      auto ostep = [&](int64_t s) {
-        const int j = static_cast<int>(s % steps);
-        const uint32_t slot = static_cast<uint32_t>(s % nslot);
-        if (!wait(&sh.dz_ready[slot], static_cast<uint32_t>((s / nslot) & 1), true)) return false;
-        fence_proxy_async_global();
-        const int dz_row = static_cast<int>((cl * nslot + slot) * 128);
-        if (!load_unit(&tm_dz, 0, dz_row)) return false;
-        if (!load_unit(&tm_dz, 64, dz_row)) return false;
-        int su = 0;
-        for (int ch = 0; ch < a.nchunk; ++ch) {
-          const int g = a.chunk_units[ch];
-          while ((pos % kRing) + g > kRing)
-            if (!pad_unit()) return false;
-          for (int i = 0; i < g; ++i)
-            if (!load_unit(&tm_stream, slice0 + (su + i) * 64, j * 128)) return false;
-          su += g;
-        }
-        return true;
-      };
-      for (int64_t s = 0; ok && s < total && s < C; ++s)
-        if (own(s)) ok = ztile(s);
-      for (int64_t s = 0; ok && s < total; ++s) {
-        if (own(s) && s + C < total) ok = ztile(s + C);
-        if (ok) ok = ostep(s);
+        advance();
       }
-      for (uint32_t i = (pos > kRing ? pos - kRing : 0u); i < pos; ++i) {
+      return true;
+    };
+    auto ostep = [&](const StreamPos& p) -> bool {
+      if (!wait(&sh.dz_ready[p.slot], p.round & 1u, true)) return false;
+      if (!acquire(kSlotBytes)) return false;
+      if (elect_one()) {
+        const int dz_row = static_cast<int>((cl * nslot + p.slot) * 128);
+        const uint32_t dst = ring_base + slot * kSlotBytes;
+        tma_load_2d(dst, &tm_dz, &sh.full[slot], 0, dz_row);
+        tma_load_2d(dst + kUnitBytes, &tm_dz, &sh.full[slot], 64, dz_row);
+      }
+      advance();
+      int col = slice0;
+      for (int ch = 0; ch < a.nchunk; ++ch) {
+        const int nu = a.chunk_units[ch];
+        if (!acquire(nu * kUnitBytes)) return false;
+        if (elect_one()) {
+          const uint32_t dst = ring_base + slot * kSlotBytes;
+          tma_load_2d(dst, &tm_stream, &sh.full[slot], col, p.j * 128);
+          if (nu == 2) tma_load_2d(dst + kUnitBytes, &tm_stream, &sh.full[slot], col + 64, p.j * 128);
+        }
+        advance();
+        col += 64 * nu;
+      }
+      return true;
+    };
+    StreamPos p, pz;  // p: step whose slice update is loaded; pz: step whose logit tile is loaded (p + C)
+    p.zero();
+    pz.zero();
+    bool ok = true;
+    for (uint32_t i = 0; ok && i < C && pz.s < total; ++i) {
+      if (pz.modc == rank) ok = ztile(pz);
+      pz.next(steps, C, nslot);
+    }
+    for (; ok && p.s < total; p.next(steps, C, nslot)) {
+      if (pz.s < total) {
+        if (pz.modc == rank) ok = ztile(pz);
+        pz.next(steps, C, nslot);
+      }
+      if (ok) ok = ostep(p);
+    }
+    // loads still in flight must land before the CTA may exit: the last fill of each slot
+    if (elect_one()) {
+      for (uint32_t i = 0; i < static_cast<uint32_t>(kSlots); ++i) {
+        const uint32_t ph = (i < slot) ? phase : (phase ^ 1u);
         const uint64_t t0 = globaltimer_ns();
-        while (!mbar_test(&sh.full[i % kRing], (i / kRing) & 1u))
+        while (!mbar_test(&sh.full[i], ph))
           if (globaltimer_ns() - t0 > a.limit_ns) break;
       }
     }
+    __syncwarp();
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------- MMA issuer ----------------
-      constexpr uint32_t idesc_z = idesc_bf16(128, 128, false, false);
-      uint32_t pos = 0, zc = 0, oc = 0;
-      bool ok = true;
-      auto take = [&](uint32_t& st) {
-        st = pos % kRing;
-        const uint32_t ph = (pos / kRing) & 1u;
-        ++pos;
-        return wait(&sh.full[st], ph, false);
-      };
-      auto ztile = [&]() {
-        if (!wait(&sh.z_empty, (zc & 1u) ^ 1u, false)) return false;
-        tc_fence_after();
-        for (int kb = 0; kb < KB; ++kb) {
-          uint32_t sa, sb;
-          if (!take(sa) || !take(sb)) return false;
-          tc_fence_after();
-          const uint32_t aa = smem_u32(ring + sa * kUnitBytes), ab = smem_u32(ring + sb * kUnitBytes);
+    // ---------------- MMA issuer (whole warp; one elected lane issues) ----------------
+    constexpr uint32_t idesc_z = idesc_bf16(128, 128, false, false);
+    constexpr uint32_t idesc_o2 = idesc_bf16(128, 128, false, true);
+    constexpr uint32_t idesc_o1 = idesc_bf16(128, 64, false, true);
+    // descriptors of slot 0 (K-major and MN-major forms); slot i adds i * kSlotBytes >> 4
+    const uint64_t dk0 = sdesc_k_sw128(ring_base);
+    const uint64_t dm0 = sdesc_mn_sw128(ring_base, kUnitBytes);
+    uint32_t slot = 0, phase = 0, zc = 0, oc = 0;
+    auto take = [&]() -> bool {
+      if (!wait(&sh.full[slot], phase, false)) return false;
+      tc_fence_after();
+      return true;
+    };
+    auto advance = [&]() {
+      if (++slot == kSlots) { slot = 0; phase ^= 1u; }
+    };
+    auto ztile = [&]() -> bool {
+      if (!wait(&sh.z_empty, (zc & 1u) ^ 1u, false)) return false;
+      tc_fence_after();
+      for (int kb = 0; kb < KB; ++kb) {
+        if (!take()) return false;
+        if (elect_one()) {
+          const uint64_t da = dk0 + static_cast<uint64_t>(slot * (kSlotBytes >> 4));
+          const uint64_t db = da + (kUnitBytes >> 4);
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            umma_bf16(tmem + kZCol, sdesc_k_sw128(aa + k * 32), sdesc_k_sw128(ab + k * 32), idesc_z, (kb | k) != 0);
-          umma_commit(&sh.empty[sa]);
-          umma_commit(&sh.empty[sb]);
+          for (int k = 0; k < 4; ++k) umma_bf16(tmem + kZCol, da + 2 * k, db + 2 * k, idesc_z, (kb | k) != 0);
+          umma_commit(&sh.empty[slot]);
         }
-        umma_commit(&sh.z_full);
-        ++zc;
-        return true;
-      };
-      auto ostep = [&](int64_t s) {
-        const int j = static_cast<int>(s % steps);
-        if (j == 0) {
-          if (!wait(&sh.o_empty, (oc & 1u) ^ 1u, false)) return false;
-          tc_fence_after();
-        }
-        uint32_t d0, d1;
-        if (!take(d0) || !take(d1)) return false;
+        advance();
+      }
+      if (elect_one()) umma_commit(&sh.z_full);
+      ++zc;
+      return true;
+    };
+    auto ostep = [&](const StreamPos& p) -> bool {
+      if (p.j == 0) {
+        if (!wait(&sh.o_empty, (oc & 1u) ^ 1u, false)) return false;
         tc_fence_after();
-        // the tile is in shared memory now: its scratch slot may be refilled by the producer
-        const uint32_t slot = static_cast<uint32_t>(s % nslot);
-        mbar_arrive_cluster(mapa_shared(smem_u32(&sh.dz_free[slot]), static_cast<uint32_t>(s % C)));
-        const uint32_t a0 = smem_u32(ring + d0 * kUnitBytes), a1 = smem_u32(ring + d1 * kUnitBytes);
-        uint32_t col = 0;
-        for (int ch = 0; ch < a.nchunk; ++ch) {
-          const int g = a.chunk_units[ch];
-          while ((pos % kRing) + g > kRing) {
-            uint32_t sp;
-            if (!take(sp)) return false;
-            mbar_arrive(&sh.empty[sp]);
-          }
-          uint32_t first = 0;
-          for (int i = 0; i < g; ++i) {
-            uint32_t st;
-            if (!take(st)) return false;
-            if (i == 0) first = st;
-          }
-          tc_fence_after();
-          const uint32_t bb = smem_u32(ring + first * kUnitBytes);
-          const uint32_t idesc_o = idesc_bf16(128, 64 * g, false, true);
+      }
+      if (!take()) return false;
+      const uint32_t dslot = slot;
+      if (elect_one())  // the tile is in shared memory now: its scratch slot may be refilled
+        mbar_arrive_cluster(mapa_shared(smem_u32(&sh.dz_free[p.slot]), p.modc));
+      advance();
+      const uint64_t da = dk0 + static_cast<uint64_t>(dslot * (kSlotBytes >> 4));
+      uint32_t col = 0;
+      for (int ch = 0; ch < a.nchunk; ++ch) {
+        const int nu = a.chunk_units[ch];
+        if (!take()) return false;
+        if (elect_one()) {
+          const uint64_t db = dm0 + static_cast<uint64_t>(slot * (kSlotBytes >> 4));
+          const uint32_t idesc = (nu == 2) ? idesc_o2 : idesc_o1;
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t aa = ((kk < 4) ? a0 : a1) + (kk & 3) * 32;
-            umma_bf16(tmem + col, sdesc_k_sw128(aa), sdesc_mn_sw128(bb + kk * 2048, kUnitBytes), idesc_o,
-                      (j > 0 || kk > 0) ? 1u : 0u);
+            // A: dZ tile, K = 128 in two 64-wide units; B: slice tile, MN-major, 16 K-rows = 2 KB per step
+            const uint64_t ak = da + ((kk < 4) ? 0 : (kUnitBytes >> 4)) + 2 * (kk & 3);
+            umma_bf16(tmem + col, ak, db + (2048 >> 4) * kk, idesc, (p.j > 0 || kk > 0) ? 1u : 0u);
           }
-          for (int i = 0; i < g; ++i) umma_commit(&sh.empty[first + i]);
-          col += 64 * g;
+          umma_commit(&sh.empty[slot]);
         }
-        umma_commit(&sh.empty[d0]);
-        umma_commit(&sh.empty[d1]);
-        if (j == steps - 1) {
-          umma_commit(&sh.o_full);
-          ++oc;
-        }
-        return true;
-      };
-      for (int64_t s = 0; ok && s < total && s < C; ++s)
-        if (own(s)) ok = ztile();
-      for (int64_t s = 0; ok && s < total; ++s) {
-        if (own(s) && s + C < total) ok = ztile();
-        if (ok) ok = ostep(s);
+        advance();
+        col += 64 * nu;
       }
+      if (elect_one()) {
+        umma_commit(&sh.empty[dslot]);
+        if (p.j == steps - 1) umma_commit(&sh.o_full);
+      }
+      if (p.j == steps - 1) ++oc;
+      return true;
+    };
+    StreamPos p, pz;
+    p.zero();
+    pz.zero();
+    bool ok = true;
+    for (uint32_t i = 0; ok && i < C && pz.s < total; ++i) {
+      if (pz.modc == rank) ok = ztile();
+      pz.next(steps, C, nslot);
+    }
+    for (; ok && p.s < total; p.next(steps, C, nslot)) {
+      if (pz.s < total) {
+        if (pz.modc == rank) ok = ztile();
+        pz.next(steps, C, nslot);
+      }
+      if (ok) ok = ostep(p);
+    }
+    if (elect_one()) {
       umma_commit(&sh.mma_done);
       const uint64_t t0 = globaltimer_ns();
       while (!mbar_test(&sh.mma_done, 0))
         if (globaltimer_ns() - t0 > a.limit_ns) break;
     }
+    __syncwarp();
   } else {
     // ---------------- epilogue: 4 warps, one accumulator lane (row) per thread ----------------
     const int quarter = warp & 3;
@@ -290,22 +349,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t tl = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     uint32_t zc = 0, oc = 0, epc = 0;
     bool ok = true;
-    // warp-uniform outcome of a wait: the tcgen05.ld that follows is .sync.aligned
-    auto ewait = [&](uint64_t* bar, uint32_t parity, bool cluster_acq) {
-      return __all_sync(0xffffffffu, wait(bar, parity, cluster_acq)) != 0;
-    };
     auto ep_sync = [&]() {
       mbar_arrive(&sh.ep_bar);
-      return ewait(&sh.ep_bar, (epc++) & 1u, false);
+      return wait(&sh.ep_bar, (epc++) & 1u, false);
     };
     float r_lse2 = 0.f, r_g = 0.f;
     int32_t r_y = -1;
     bool r_valid = false;
-    int64_t r_out = 0;
 
     auto drain = [&](int u, bool have_acc) {
       if (have_acc) {
-        if (!ewait(&sh.o_full, oc & 1u, false)) return false;
+        if (!wait(&sh.o_full, oc & 1u, false)) return false;
         tc_fence_after();
       }
       if (kMode == kModeDH) {
@@ -361,34 +415,33 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       // no rows: every owned vocabulary tile gets a zero gradient
       for (int u = static_cast<int>(cl); u < nunits; u += static_cast<int>(ncl)) drain(u, false);
     }
-    for (int64_t s = 0; ok && s < total; ++s) {
-      const int u = unit_of(s);
-      const int j = static_cast<int>(s % steps);
-      if (kMode == kModeDH && j == 0) {
+    StreamPos p;
+    p.zero();
+    for (; ok && p.s < total; p.next(steps, C, nslot)) {
+      const int u = static_cast<int>(cl) + p.u_idx * static_cast<int>(ncl);
+      if (kMode == kModeDH && p.j == 0) {
         const int64_t t = static_cast<int64_t>(u) * 128 + row;
         r_valid = t < rows;
         r_lse2 = r_valid ? a.lse[t] * kLog2e : 0.f;
         r_g = r_valid ? a.g[t] : 0.f;
         r_y = r_valid ? a.y[t] : -1;
-        r_out = t;
       }
-      if (own(s)) {
-        const uint32_t slot = static_cast<uint32_t>(s % nslot);
+      if (p.modc == rank) {
         if (kMode == kModeDW) {
           if (!ep_sync()) { ok = false; break; }  // previous step's column parameters are no longer read
-          const int64_t t = static_cast<int64_t>(j) * 128 + et;
+          const int64_t t = static_cast<int64_t>(p.j) * 128 + et;
           const bool tv = t < rows;
           sh.col_lse2[et] = tv ? a.lse[t] * kLog2e : 0.f;
           sh.col_g[et] = tv ? a.g[t] : 0.f;
           sh.col_y[et] = tv ? a.y[t] : INT32_MIN;
           if (!ep_sync()) { ok = false; break; }
         }
-        if (!ewait(&sh.z_full, zc & 1u, false)) { ok = false; break; }
+        if (!wait(&sh.z_full, zc & 1u, false)) { ok = false; break; }
         tc_fence_after();
-        if (s >= nslot) {
-          if (!ewait(&sh.dz_free[slot], static_cast<uint32_t>(((s / nslot) - 1) & 1), true)) { ok = false; break; }
+        if (p.round > 0) {
+          if (!wait(&sh.dz_free[p.slot], (p.round - 1) & 1u, true)) { ok = false; break; }
         }
-        uint16_t* dzrow = a.dz_scratch + (static_cast<int64_t>(cl * nslot + slot) * 128 + row) * 128;
+        uint16_t* dzrow = a.dz_scratch + (static_cast<int64_t>(cl * nslot + p.slot) * 128 + row) * 128;
         const int64_t vrow = static_cast<int64_t>(u) * 128 + row;  // kModeDW: this lane's vocabulary row
         for (int c = 0; c < 4; ++c) {
           uint32_t v[32];
@@ -396,22 +449,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tmem_ld_wait();
           float d[32];
           if (kMode == kModeDH) {
-            const int vbase = j * 128 + c * 32;
+            const int vbase = p.j * 128 + c * 32;
 #pragma unroll
             for (int q = 0; q < 32; ++q) {
-              const float p = ex2_approx(fmaf(__uint_as_float(v[q]), kLog2e, -r_lse2));
+              const float pr = ex2_approx(fmaf(__uint_as_float(v[q]), kLog2e, -r_lse2));
               const float oh = (vbase + q == r_y) ? 1.f : 0.f;
-              d[q] = (r_valid && vbase + q < a.V) ? r_g * (oh - p) : 0.f;
+              d[q] = (r_valid && vbase + q < a.V) ? r_g * (oh - pr) : 0.f;
             }
           } else {
             const bool v_ok = vrow < a.V;
 #pragma unroll
             for (int q = 0; q < 32; ++q) {
               const int tc = c * 32 + q;
-              const float p = ex2_approx(fmaf(__uint_as_float(v[q]), kLog2e, -sh.col_lse2[tc]));
+              const float pr = ex2_approx(fmaf(__uint_as_float(v[q]), kLog2e, -sh.col_lse2[tc]));
               const int32_t yc = sh.col_y[tc];
               const float oh = (static_cast<int64_t>(yc) == vrow) ? 1.f : 0.f;
-              d[q] = (v_ok && yc != INT32_MIN) ? sh.col_g[tc] * (oh - p) : 0.f;
+              d[q] = (v_ok && yc != INT32_MIN) ? sh.col_g[tc] * (oh - pr) : 0.f;
             }
           }
           uint4* d4 = reinterpret_cast<uint4*>(dzrow + c * 32);
@@ -427,15 +480,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         fence_proxy_async_global();
         if (!ep_sync()) { ok = false; break; }
         if (et == 0) {
-          const uint32_t la = smem_u32(&sh.dz_ready[slot]);
+          const uint32_t la = smem_u32(&sh.dz_ready[p.slot]);
           for (uint32_t q = 0; q < C; ++q) mbar_arrive_cluster(mapa_shared(la, q));
         }
       }
-      if (j == steps - 1) {
+      if (p.j == steps - 1) {
         if (!drain(u, true)) { ok = false; break; }
       }
     }
-    (void)r_out;
   }
 
   tc_fence_before();

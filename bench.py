@@ -43,6 +43,8 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--small", action="store_true",
+                    help="profiling case: same head, 4 responses of 1024 rows (T=4096); not a bench line")
     return ap.parse_args()
 
 
@@ -198,6 +200,8 @@ def run_ours(args):
         dist.barrier()
         pg = dist
     spec = spec_for(CONFIG)
+    if args.small:
+        spec = spec_for(CONFIG, groups=1, per_group=4, len_lo=1024, len_hi=1024)
     b = make_batch(spec, seed=1234 + spec.index + 1000 * rank, device=dev)
     T, H, V, R = b.n_rows, spec.H, spec.V, b.R
     # rollout log-probabilities from the lagged head (the rollout engine's role), plus noise rows
