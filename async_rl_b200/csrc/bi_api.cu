@@ -109,15 +109,19 @@ WsLayout ws_layout(int64_t T, int32_t H, int32_t R) {
   L.nred = static_cast<int>((t + bi::kRedBlock - 1) / bi::kRedBlock);
   L.red = take(static_cast<size_t>(L.nred) * sizeof(RedPart));
   L.hc = take(R > 0 ? t * static_cast<size_t>(H) * 2 : 0);
-  L.dz = take(static_cast<size_t>(kDzSlotsMax) * 128 * 128 * 2);
+  L.dz = take(static_cast<size_t>(kDzSlotsMax) * 128 * bi::kMaxNZ * 2);
   L.total = o;
   return L;
 }
 
-// Split of H over a cluster: smallest C in {1, 2, 4, 8} with H / C <= 384 and a multiple of 64.
+// Column split of H over a cluster of C CTAs: Hs = H / C must be a multiple of 64 and at most
+// 384 (its fp32 accumulator plus a logit tile of NZ >= 128 columns fill the 512 TMEM columns).
+bool split_ok(int32_t H, int c) { return H % c == 0 && (H / c) % 64 == 0 && H / c <= 384; }
+int logit_cols(int Hs) { return ((512 - Hs) < 256 ? (512 - Hs) : 256) / 64 * 64; }
+// Any valid split exists (shape check that needs no device).
 int cluster_split(int32_t H) {
-  for (int c : {1, 2, 4, 8})
-    if (H % c == 0 && (H / c) % 64 == 0 && H / c <= 384) return c;
+  for (int c = 1; c <= bi::kMaxCluster; ++c)
+    if (split_ok(H, c)) return c;
   return 0;
 }
 
@@ -163,7 +167,7 @@ struct DevInfo {
   bool ready = false;
   bool ok = false;
   int sms = 0;
-  int max_clusters[2][9] = {};  // [mode][C]
+  int max_clusters[2][bi::kMaxCluster + 1] = {};  // [mode][C]
 };
 std::mutex g_dev_mu;
 std::array<DevInfo, 64> g_dev;
@@ -173,7 +177,7 @@ int query_clusters(int C) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(C, 1, 1);
   cfg.blockDim = dim3(bi::kBwdThreads, 1, 1);
-  cfg.dynamicSmemBytes = bi::kBwdSmemBytes;
+  cfg.dynamicSmemBytes = bi::kBwdSmemLimit;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = C;
@@ -182,8 +186,21 @@ int query_clusters(int C) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, bi::k_bwd_cluster<kMode>, &cfg) != cudaSuccess) return 0;
+  // every compiled tiling needs one CTA per SM; the occupancy of one of them stands for all
+  if (cudaOccupancyMaxActiveClusters(&n, bi::k_bwd_cluster<kMode, 256, 256>, &cfg) != cudaSuccess) return 0;
   return n;
+}
+
+bool set_bwd_attributes() {
+  bool ok = true;
+#define BI_SET_ATTR(NZ_, HS_)                                                                                   \
+  ok = ok && cudaFuncSetAttribute(bi::k_bwd_cluster<bi::kModeDH, NZ_, HS_>,                                    \
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, bi::kBwdSmemLimit) == cudaSuccess; \
+  ok = ok && cudaFuncSetAttribute(bi::k_bwd_cluster<bi::kModeDW, NZ_, HS_>,                                    \
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, bi::kBwdSmemLimit) == cudaSuccess;
+  BI_BWD_CONFIGS(BI_SET_ATTR)
+#undef BI_SET_ATTR
+  return ok;
 }
 
 const DevInfo* device_info() {
@@ -196,12 +213,9 @@ const DevInfo* device_info() {
   if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return nullptr;
   if (cudaFuncSetAttribute(bi::k_fwd_logits, cudaFuncAttributeMaxDynamicSharedMemorySize, bi::kFwdSmemBytes) !=
           cudaSuccess ||
-      cudaFuncSetAttribute(bi::k_bwd_cluster<bi::kModeDH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           bi::kBwdSmemBytes) != cudaSuccess ||
-      cudaFuncSetAttribute(bi::k_bwd_cluster<bi::kModeDW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           bi::kBwdSmemBytes) != cudaSuccess)
+      !set_bwd_attributes())
     return nullptr;
-  for (int c : {1, 2, 4, 8}) {
+  for (int c = 1; c <= bi::kMaxCluster; ++c) {
     d.max_clusters[0][c] = query_clusters<bi::kModeDH>(c);
     d.max_clusters[1][c] = query_clusters<bi::kModeDW>(c);
   }
@@ -238,9 +252,33 @@ bi_status launch_fwd(const uint16_t* hidden, int64_t T, const int64_t* d_rows, c
   return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
 }
 
-template <int kMode>
-bi_status launch_bwd(const CUtensorMap& tm_stat, const CUtensorMap& tm_stream, const CUtensorMap& tm_dz,
-                     const bi::BwdArgs& a, int64_t units_upper, const DevInfo* di, cudaStream_t s) {
+// Backward tiling for H: the split with the widest logit tile (NZ), then the most SMs in use.
+struct BwdPlan {
+  int C = 0, Hs = 0, NZ = 0;
+};
+BwdPlan plan_bwd(int32_t H, const DevInfo* di) {
+  BwdPlan best;
+  int best_sms = -1;
+  for (int c = 1; c <= bi::kMaxCluster; ++c) {
+    if (!split_ok(H, c)) continue;
+    const int hs = H / c, nz = logit_cols(hs);
+    const int sms = di->max_clusters[0][c] * c;
+    if (di->max_clusters[0][c] <= 0 || di->max_clusters[1][c] <= 0) continue;
+    if (nz > best.NZ || (nz == best.NZ && sms > best_sms)) {
+      best.C = c;
+      best.Hs = hs;
+      best.NZ = nz;
+      best_sms = sms;
+    }
+  }
+  return best;
+}
+
+template <int kMode, int kNZ, int kHS>
+bi_status launch_bwd(const CUtensorMap& tm_stat, const CUtensorMap& tm_zb, const CUtensorMap& tm_sl,
+                     const CUtensorMap& tm_dz, const bi::BwdArgs& a, int64_t units_upper, const DevInfo* di,
+                     cudaStream_t s) {
+  const int smem = bi::BwdTile<kNZ, kHS>::smem;
   const int maxc = di->max_clusters[kMode][a.C];
   if (maxc <= 0) return BI_ERR_CUDA;
   int64_t ncl = units_upper < maxc ? units_upper : maxc;
@@ -249,7 +287,7 @@ bi_status launch_bwd(const CUtensorMap& tm_stat, const CUtensorMap& tm_stream, c
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(ncl * a.C), 1, 1);
   cfg.blockDim = dim3(bi::kBwdThreads, 1, 1);
-  cfg.dynamicSmemBytes = bi::kBwdSmemBytes;
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -259,7 +297,7 @@ bi_status launch_bwd(const CUtensorMap& tm_stat, const CUtensorMap& tm_stream, c
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   ProfScope ps(kMode == bi::kModeDH ? kKBwdDH : kKBwdDW, s);
-  return cudaLaunchKernelEx(&cfg, bi::k_bwd_cluster<kMode>, tm_stat, tm_stream, tm_dz, a) == cudaSuccess
+  return cudaLaunchKernelEx(&cfg, bi::k_bwd_cluster<kMode, kNZ, kHS>, tm_stat, tm_zb, tm_sl, tm_dz, a) == cudaSuccess
              ? BI_OK
              : BI_ERR_CUDA;
 }
@@ -430,23 +468,26 @@ bi_status bi_is_loss_fwd_bwd(const uint16_t* hidden, const uint16_t* w_lm, const
   if (cudaGetLastError() != cudaSuccess) return BI_ERR_CUDA;
 
   // backward: dH (row tiles) and dW (vocabulary tiles)
-  CUtensorMap tm_h, tm_w, tm_dz;
+  const BwdPlan pl = plan_bwd(H, di);
+  if (pl.C == 0) return BI_ERR_UNSUPPORTED_SHAPE;
+  CUtensorMap tm_h128, tm_hz, tm_h64, tm_w128, tm_wz, tm_w64, tm_dz;
   const int64_t trows = T > 0 ? T : 1;
-  if (!make_map(&tm_h, hc ? hc : reinterpret_cast<const uint16_t*>(w8 + L.hc), trows, H, 128) ||
-      !make_map(&tm_w, w_lm, V, H, 128) ||
-      !make_map(&tm_dz, w8 + L.dz, static_cast<int64_t>(kDzSlotsMax) * 128, 128, 128))
+  const void* hsrc = hc ? static_cast<const void*>(hc) : static_cast<const void*>(w8 + L.hc);
+  if (!make_map(&tm_h128, hsrc, trows, H, 128) || !make_map(&tm_hz, hsrc, trows, H, pl.NZ) ||
+      !make_map(&tm_h64, hsrc, trows, H, 64) || !make_map(&tm_w128, w_lm, V, H, 128) ||
+      !make_map(&tm_wz, w_lm, V, H, pl.NZ) || !make_map(&tm_w64, w_lm, V, H, 64) ||
+      !make_map(&tm_dz, w8 + L.dz, static_cast<int64_t>(kDzSlotsMax) * 128, pl.NZ, 128))
     return BI_ERR_CUDA;
   bi::BwdArgs a{};
   a.H = H;
   a.V = V;
-  a.C = C;
-  a.Hs = H / C;
-  const int su = a.Hs / 64;  // 64-column units of the slice: chunks of two units, a last one of one
-  a.nchunk = (su + 1) / 2;
-  for (int c = 0; c < bi::kMaxChunks; ++c) a.chunk_units[c] = c < a.nchunk ? ((2 * c + 1 < su) ? 2 : 1) : 0;
+  a.C = pl.C;
+  a.Hs = pl.Hs;
+  a.NZ = pl.NZ;
   a.T = trows;
   a.d_rows = d_rows;
-  a.nvt128 = (V + 127) / 128;
+  a.nvz = (V + pl.NZ - 1) / pl.NZ;
+  a.nv128 = (V + 127) / 128;
   a.lse = F(L.lse_c);
   a.g = F(L.g_c);
   a.y = I(L.y_c);
@@ -456,10 +497,16 @@ bi_status bi_is_loss_fwd_bwd(const uint16_t* hidden, const uint16_t* w_lm, const
   a.dz_scratch = reinterpret_cast<uint16_t*>(w8 + L.dz);
   a.status = dev_status;
   a.limit_ns = kWaitLimitNs;
-  bi_status st = BI_OK;
-  if (T > 0) st = launch_bwd<bi::kModeDH>(tm_h, tm_w, tm_dz, a, (T + 127) / 128, di, s);
-  if (st != BI_OK) return st;
-  return launch_bwd<bi::kModeDW>(tm_w, tm_h, tm_dz, a, a.nvt128, di, s);
+  bi_status st = BI_ERR_UNSUPPORTED_SHAPE;
+#define BI_LAUNCH(NZ_, HS_)                                                                                  \
+  if (pl.NZ == NZ_ && pl.Hs == HS_) {                                                                        \
+    st = BI_OK;                                                                                            \
+    if (T > 0) st = launch_bwd<bi::kModeDH, NZ_, HS_>(tm_h128, tm_wz, tm_w64, tm_dz, a, (T + 127) / 128, di, s); \
+    if (st == BI_OK) st = launch_bwd<bi::kModeDW, NZ_, HS_>(tm_w128, tm_hz, tm_h64, tm_dz, a, a.nv128, di, s); \
+  }
+  BI_BWD_CONFIGS(BI_LAUNCH)
+#undef BI_LAUNCH
+  return st;
 }
 
 bi_status bi_d3_stats(const float* learner_logprob, const float* rollout_logprob, const uint8_t* mask, int64_t T,

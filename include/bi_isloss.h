@@ -43,8 +43,8 @@
  *     weight, D3 term or loss) or BI_ERR_TIMEOUT (a bounded wait inside a kernel ran out; the
  *     kernel returned early and its outputs are undefined).  Read it after synchronising.
  *     Kernels never trap.
- *   - Supported shapes: H a multiple of 64 with H / C <= 384 and a multiple of 64 for some
- *     C in {1, 2, 4, 8} (e.g. 128, 1536, 2048, 2560, 3072); 1 <= V < 2^31; 0 <= T < 2^31.
+ *   - Supported shapes: H a multiple of 64 such that H / C is a multiple of 64 and at most 384
+ *     for some C in 1..8 (e.g. 128, 1536, 2048, 2560, 3072); 1 <= V < 2^31; 0 <= T < 2^31.
  */
 #ifndef BI_ISLOSS_H
 #define BI_ISLOSS_H

@@ -66,7 +66,7 @@ def test_logprob_argument_checks(lib):
     assert lib.bi_logprob_fwd(FAKE + 2, FAKE, FAKE, 10, 128, 512, FAKE, None, st, FAKE, ws_bytes, None) == 1
     # unsupported H
     assert lib.bi_logprob_fwd(FAKE, FAKE, FAKE, 10, 100, 512, FAKE, None, st, FAKE, ws_bytes, None) == 2
-    assert lib.bi_logprob_fwd(FAKE, FAKE, FAKE, 10, 448, 512, FAKE, None, st, FAKE, ws_bytes, None) == 2
+    assert lib.bi_logprob_fwd(FAKE, FAKE, FAKE, 10, 704, 512, FAKE, None, st, FAKE, ws_bytes, None) == 2
     # workspace too small / missing / misaligned
     assert lib.bi_logprob_fwd(FAKE, FAKE, FAKE, 10, 128, 512, FAKE, None, st, FAKE, ws_bytes - 1, None) == 3
     assert lib.bi_logprob_fwd(FAKE, FAKE, FAKE, 10, 128, 512, FAKE, None, st, None, ws_bytes, None) == 3
@@ -95,7 +95,7 @@ def test_is_loss_argument_checks(lib):
     assert call(rnorm=-1.0) == 1
     assert call(loss=None) == 1
     assert call(grad_w=FAKE + 4) == 1  # misaligned
-    assert call(H=448) == 2            # 7 * 64: no split into <= 384-column multiples of 64
+    assert call(H=704) == 2            # 11 * 64: no split into <= 384-column multiples of 64 with C <= 8
     assert call(ws_bytes=ws_bytes - 1) == 3
 
 
