@@ -182,18 +182,24 @@ __device__ __forceinline__ void bwd_tma_role(BwdShared& sh, const BwdArgs& a, co
       pz.next(x.steps, x.C, x.nslot);
     }
     if (it < 0) continue;
-    if (!bwd_wait<true>(sh, a, x.C, &sh.dz_ready[p.slot], p.round & 1u)) break;
+    // slice tiles of this CTA do not depend on the dZ tile: they are requested first, the dZ
+    // chunks once the producer has published the tile
     const int dz_row = static_cast<int>((x.cl * x.nslot + p.slot) * 128);
+    bool dz_ok = false;
 #pragma unroll 1
     for (int kc = 0; kc < nkc; ++kc) {
       if (!bwd_wait<false>(sh, a, x.C, &sh.empty[stage], phase ^ 1u)) { ok = false; break; }
       mbar_arrive_expect_tx(&sh.full[stage], obytes);
       const uint32_t dst = x.ring_base + stage * sbytes;
-      tma_load_2d(dst, m.dz, &sh.full[stage], kc * 64, dz_row);
       const int yrow = p.j * kNZ + kc * 64;
 #pragma unroll
       for (int u = 0; u < nsl; ++u)
         tma_load_2d(dst + kAUnitBytes + u * kSlUnitBytes, m.sl, &sh.full[stage], x.slice0 + u * 64, yrow);
+      if (!dz_ok) {
+        if (!bwd_wait<true>(sh, a, x.C, &sh.dz_ready[p.slot], p.round & 1u)) { ok = false; break; }
+        dz_ok = true;
+      }
+      tma_load_2d(dst, m.dz, &sh.full[stage], kc * 64, dz_row);
       ring_advance(stage, phase, nst);
     }
     if (!ok) break;
@@ -265,8 +271,10 @@ __device__ __forceinline__ void bwd_mma_role(BwdShared& sh, const BwdArgs& a, co
     for (int kc = 0; kc < nkc; ++kc) {
       if (!bwd_wait<false>(sh, a, x.C, &sh.full[stage], phase)) { ok = false; break; }
       tc_fence_after();
-      if (kc == nkc - 1)  // every chunk of the dZ tile has landed: its scratch slot may be refilled
-        mbar_arrive_cluster(mapa_shared(smem_u32(&sh.dz_free[p.slot]), p.modc));
+      // every chunk of the dZ tile has landed in shared memory (the full barrier completed): the
+      // producer may refill its scratch slot.  Nothing this thread wrote needs ordering, so the
+      // signal is relaxed (a release here stalls the issuing lane for ~0.4 us).
+      if (kc == nkc - 1) mbar_arrive_cluster_relaxed(mapa_shared(smem_u32(&sh.dz_free[p.slot]), p.modc));
       const uint64_t da = dk0 + stage * sb_desc;
       const uint64_t db = dmb0 + stage * sb_desc;
       const uint32_t acc0 = (p.j > 0 || kc > 0) ? 1u : 0u;
