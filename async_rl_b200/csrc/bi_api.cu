@@ -306,6 +306,40 @@ unsigned blocks_for(int64_t n, int per) { return static_cast<unsigned>((n + per 
 
 }  // namespace
 
+namespace {
+
+// ---------------------------------------------------------------------------------------------
+// Fixed scratch for bi_logprob_fwd_noalloc.  Some callers cannot allocate device memory at all:
+// code that runs inside a host framework which owns every device allocation (a serving engine's
+// fixed memory pool, a plugin given no allocator handle) has no way to hand this library a
+// workspace.  For them, the forward's per-chunk partials live in this array instead.  It is a
+// file-scope device array, so every GPU that loads the library holds it (1.5 MB) until the
+// process exits.  All calls share it: calls whose kernels overlap on the GPU (different streams,
+// different host threads) race on it.
+// ---------------------------------------------------------------------------------------------
+constexpr int64_t kNoAllocMaxRows = 8192;  // largest T accepted by bi_logprob_fwd_noalloc
+constexpr size_t kNoAllocFloats = 3 * static_cast<size_t>(bi::kMaxVChunks) * kNoAllocMaxRows;
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocFloats];
+
+// The array's name is only a host-side stand-in; the kernel needs its device address, looked up
+// once per device with that device current (on the first call made on it).
+float* noalloc_scratch_address() {
+  static std::mutex mu;
+  static std::array<float*, 64> addr{};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= static_cast<int>(addr.size())) return nullptr;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    addr[dev] = static_cast<float*>(p);
+  }
+  return addr[dev];
+}
+
+
+}  // namespace
+
 extern "C" {
 
 int32_t bi_version(void) { return 100; }
@@ -385,6 +419,38 @@ bi_status bi_logprob_fwd(const uint16_t* hidden, const uint16_t* w_lm, const int
   if (st != BI_OK) return st;
   const int nvt = (V + bi::kFwdBN - 1) / bi::kFwdBN;
   ProfScope ps(kKCombineLp, s);
+  bi::k_combine_logprob<<<blocks_for(T, 256), 256, 0, s>>>(
+      reinterpret_cast<float*>(w8 + L.part_m), reinterpret_cast<float*>(w8 + L.part_s),
+      reinterpret_cast<float*>(w8 + L.part_zy), T, nchunks_for(nvt), nvt, V, targets, logprob, lse, dev_status);
+  return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+}
+
+// Same computation as bi_logprob_fwd, with the chunk partials in the library's fixed scratch
+// array instead of a caller workspace: no device allocation by anyone.  T <= 8192.
+bi_status bi_logprob_fwd_noalloc(const uint16_t* hidden, const uint16_t* w_lm, const int32_t* targets, int64_t T,
+                                 int32_t H, int32_t V, float* logprob, float* lse, int32_t* dev_status,
+                                 void* stream) {
+  if (T < 0 || H <= 0 || V <= 0) return BI_ERR_INVALID_ARG;
+  if (T > kNoAllocMaxRows) return BI_ERR_WORKSPACE;  // the fixed scratch holds 8192 rows
+  if (!dev_status || (T > 0 && (!hidden || !w_lm || !targets || !logprob))) return BI_ERR_INVALID_ARG;
+  if (T > 0 && (!aligned16(hidden) || !aligned16(w_lm))) return BI_ERR_INVALID_ARG;
+  if (H % 64 != 0 || cluster_split(H) == 0) return BI_ERR_UNSUPPORTED_SHAPE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const DevInfo* di = device_info();
+  if (!di) return BI_ERR_CUDA;
+  float* scratch = noalloc_scratch_address();
+  if (!scratch) return BI_ERR_CUDA;
+  if (cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s) != cudaSuccess) return BI_ERR_CUDA;
+  if (T == 0) return BI_OK;
+  // partials [3][kMaxVChunks][T] carved from the scratch; every entry read is written first
+  WsLayout L{};
+  L.part_m = 0;
+  L.part_s = static_cast<size_t>(bi::kMaxVChunks) * static_cast<size_t>(T) * sizeof(float);
+  L.part_zy = 2 * L.part_s;
+  uint8_t* w8 = reinterpret_cast<uint8_t*>(scratch);
+  bi_status st = launch_fwd(hidden, T, nullptr, w_lm, H, V, targets, L, w8, dev_status, di, s, 0);
+  if (st != BI_OK) return st;
+  const int nvt = (V + bi::kFwdBN - 1) / bi::kFwdBN;
   bi::k_combine_logprob<<<blocks_for(T, 256), 256, 0, s>>>(
       reinterpret_cast<float*>(w8 + L.part_m), reinterpret_cast<float*>(w8 + L.part_s),
       reinterpret_cast<float*>(w8 + L.part_zy), T, nchunks_for(nvt), nvt, V, targets, logprob, lse, dev_status);

@@ -103,6 +103,25 @@ BI_API bi_status bi_logprob_fwd(const uint16_t* hidden, const uint16_t* w_lm, co
                          int64_t T, int32_t H, int32_t V, float* logprob, float* lse,
                          int32_t* dev_status, void* ws, size_t ws_bytes, void* stream);
 
+/* bi_logprob_fwd for callers that cannot allocate device memory.  The source pages have no
+ * counterpart of this entry point; it exists for code that runs inside a host framework which
+ * owns every device allocation (a serving engine's fixed memory pool, a plugin given no allocator
+ * handle) and so cannot pass a workspace.  Arguments and results are those of bi_logprob_fwd
+ * without the workspace; the forward's scratch lives in a fixed device array inside the library
+ * (1.5 MB, held by every GPU that loads the library until the process exits).
+ *   - T is limited to 8192 rows; a larger T returns BI_ERR_WORKSPACE and launches nothing.
+ *   - The call allocates nothing (no cudaMalloc, no library allocator).  Its first call on a
+ *     device looks up the array's device address with that device current; make that first call
+ *     before any stream capture.
+ *   - All calls share the one array and it keeps the last call's contents (every value read is
+ *     written first by the same call).  Calls whose kernels overlap on the GPU -- different
+ *     streams or host threads without ordering between them -- race on it and must be serialised
+ *     by the caller. */
+BI_API bi_status bi_logprob_fwd_noalloc(const uint16_t* hidden, const uint16_t* w_lm,
+                                        const int32_t* targets, int64_t T, int32_t H, int32_t V,
+                                        float* logprob, float* lse, int32_t* dev_status,
+                                        void* stream);
+
 /* Fused forward + backward of the unclipped token-level IS REINFORCE loss.
  *   hidden, w_lm, targets, T, H, V   as in bi_logprob_fwd (T = all packed rows)
  *   rollout_logprob [T] float   log mu of each row's target under the rollout policy
