@@ -10,8 +10,7 @@
 #include <vector>
 
 #include "bi_isloss.h"
-#include "kernels_bwd.cuh"
-#include "kernels_fwd.cuh"
+#include "kernels_lm.cuh"
 #include "kernels_small.cuh"
 
 namespace {
@@ -28,11 +27,11 @@ thread_local uint64_t g_force_timeout_ns = 0;
 // ---------------------------------------------------------------------------------------------
 // optional per-kernel timing (events around each launch; measurement tools only)
 // ---------------------------------------------------------------------------------------------
-enum KernelKind : int { kKPrep, kKRowmap, kKZeroRows, kKGather, kKFwd, kKCombineLp, kKCombineIs, kKReduce,
-                        kKBwdDH, kKBwdDW, kKD3Partial, kNumKinds };
+enum KernelKind : int { kKPrep, kKRowmap, kKZeroRows, kKGather, kKLmFwd, kKLmFwdDH, kKLmDW, kKRowParts,
+                        kKReduce, kKD3Partial, kNumKinds };
 const char* const kKindNames[kNumKinds] = {"k_prep", "k_rowmap", "k_zero_prompt_rows", "k_gather_rows",
-                                           "k_fwd_logits", "k_combine_logprob", "k_combine_is",
-                                           "k_reduce_parts", "k_bwd_dh", "k_bwd_dw", "k_d3_partial"};
+                                           "k_lm_fwd", "k_lm_fwd_dh", "k_lm_dw", "k_row_parts",
+                                           "k_reduce_parts", "k_d3_partial"};
 struct Pending {
   int kind;
   cudaEvent_t a, b;
@@ -81,10 +80,13 @@ struct ProfScope {  // records an event pair around one launch when profiling is
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct WsLayout {
-  size_t ctrl, part_m, part_s, part_zy, lse_c, g_c, y_c, logmu_c, rowmap, respof, coef, cprefix, red, hc, dz, total;
+  size_t ctrl, lse_c, g_c, tl_c, d3_c, y_c, logmu_c, rowmap, respof, coef, cprefix, red, hc, dz, alpha, fin, total;
   int nred;
 };
 
+constexpr size_t kFinBytes = static_cast<size_t>(kMaxSms) * 2 * 384 * sizeof(float);  // [CTAs][2][3][128]
+
+// R == 0: the logprob-only layout (per-CTA partials only).  R > 0: the loss layout.
 WsLayout ws_layout(int64_t T, int32_t H, int32_t R) {
   WsLayout L{};
   const size_t t = static_cast<size_t>(T > 0 ? T : 1);
@@ -94,22 +96,27 @@ WsLayout ws_layout(int64_t T, int32_t H, int32_t R) {
     o = align_up(o + bytes, 256);
     return at;
   };
-  L.ctrl = take(256);
-  L.part_m = take(bi::kMaxVChunks * t * 4);
-  L.part_s = take(bi::kMaxVChunks * t * 4);
-  L.part_zy = take(bi::kMaxVChunks * t * 4);
-  L.lse_c = take(t * 4);
-  L.g_c = take(t * 4);
-  L.y_c = take(t * 4);
-  L.logmu_c = take(t * 4);
-  L.rowmap = take(t * 4);
-  L.respof = take(t * 4);
-  L.coef = take(static_cast<size_t>(R > 0 ? R : 1) * 8);
-  L.cprefix = take(static_cast<size_t>(R + 1) * 8);
-  L.nred = static_cast<int>((t + bi::kRedBlock - 1) / bi::kRedBlock);
-  L.red = take(static_cast<size_t>(L.nred) * sizeof(RedPart));
-  L.hc = take(R > 0 ? t * static_cast<size_t>(H) * 2 : 0);
-  L.dz = take(static_cast<size_t>(kDzSlotsMax) * 128 * bi::kMaxNZ * 2);
+  const size_t nred = (t + bi::kRedBlock - 1) / bi::kRedBlock;
+  // R == 0 also serves bi_d3_stats, whose block partials share the region
+  L.fin = take(R > 0 || kFinBytes >= nred * sizeof(RedPart) ? kFinBytes : nred * sizeof(RedPart));
+  if (R > 0) {
+    L.ctrl = take(256);
+    L.lse_c = take(t * 4);
+    L.g_c = take(t * 4);
+    L.tl_c = take(t * 4);
+    L.d3_c = take(t * 4);
+    L.y_c = take(t * 4);
+    L.logmu_c = take(t * 4);
+    L.rowmap = take(t * 4);
+    L.respof = take(t * 4);
+    L.coef = take(static_cast<size_t>(R) * 8);
+    L.cprefix = take(static_cast<size_t>(R + 1) * 8);
+    L.nred = static_cast<int>(nred);
+    L.red = take(static_cast<size_t>(L.nred) * sizeof(RedPart));
+    L.hc = take(t * static_cast<size_t>(H) * 2);
+    L.dz = take(static_cast<size_t>(kDzSlotsMax) * 128 * bi::kMaxNZ * 2);
+    L.alpha = take(static_cast<size_t>(kDzSlotsMax) * 128 * 4);
+  }
   L.total = o;
   return L;
 }
@@ -167,7 +174,7 @@ struct DevInfo {
   bool ready = false;
   bool ok = false;
   int sms = 0;
-  int max_clusters[2][bi::kMaxCluster + 1] = {};  // [mode][C]
+  int max_clusters[3][bi::kMaxCluster + 1] = {};  // [mode][C]
 };
 std::mutex g_dev_mu;
 std::array<DevInfo, 64> g_dev;
@@ -176,8 +183,8 @@ template <int kMode>
 int query_clusters(int C) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(C, 1, 1);
-  cfg.blockDim = dim3(bi::kBwdThreads, 1, 1);
-  cfg.dynamicSmemBytes = bi::kBwdSmemLimit;
+  cfg.blockDim = dim3(bi::LmThreads<kMode>::value, 1, 1);
+  cfg.dynamicSmemBytes = bi::LmTile<256, 256>::smem;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = C;
@@ -187,18 +194,23 @@ int query_clusters(int C) {
   cfg.numAttrs = 1;
   int n = 0;
   // every compiled tiling needs one CTA per SM; the occupancy of one of them stands for all
-  if (cudaOccupancyMaxActiveClusters(&n, bi::k_bwd_cluster<kMode, 256, 256>, &cfg) != cudaSuccess) return 0;
+  if (cudaOccupancyMaxActiveClusters(&n, bi::k_lm_cluster<kMode, 256, 256>, &cfg) != cudaSuccess) return 0;
   return n;
 }
 
-bool set_bwd_attributes() {
+bool set_lm_attributes() {
   bool ok = true;
-#define BI_SET_ATTR(NZ_, HS_)                                                                                   \
-  ok = ok && cudaFuncSetAttribute(bi::k_bwd_cluster<bi::kModeDH, NZ_, HS_>,                                    \
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize, bi::kBwdSmemLimit) == cudaSuccess; \
-  ok = ok && cudaFuncSetAttribute(bi::k_bwd_cluster<bi::kModeDW, NZ_, HS_>,                                    \
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize, bi::kBwdSmemLimit) == cudaSuccess;
-  BI_BWD_CONFIGS(BI_SET_ATTR)
+#define BI_SET_ATTR(NZ_, HS_)                                                                                  \
+  ok = ok && cudaFuncSetAttribute(bi::k_lm_cluster<bi::kModeFwd, NZ_, HS_>,                                   \
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize,                                \
+                                  bi::LmTile<NZ_, HS_>::smem) == cudaSuccess;                                 \
+  ok = ok && cudaFuncSetAttribute(bi::k_lm_cluster<bi::kModeFwdDH, NZ_, HS_>,                                 \
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize,                                \
+                                  bi::LmTile<NZ_, HS_>::smem) == cudaSuccess;                                 \
+  ok = ok && cudaFuncSetAttribute(bi::k_lm_cluster<bi::kModeDW, NZ_, HS_>,                                    \
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize,                                \
+                                  bi::LmTile<NZ_, HS_>::smem) == cudaSuccess;
+  BI_LM_CONFIGS(BI_SET_ATTR)
 #undef BI_SET_ATTR
   return ok;
 }
@@ -211,59 +223,32 @@ const DevInfo* device_info() {
   if (d.ready) return d.ok ? &d : nullptr;
   d.ready = true;
   if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return nullptr;
-  if (cudaFuncSetAttribute(bi::k_fwd_logits, cudaFuncAttributeMaxDynamicSharedMemorySize, bi::kFwdSmemBytes) !=
-          cudaSuccess ||
-      !set_bwd_attributes())
-    return nullptr;
+  if (!set_lm_attributes()) return nullptr;
   for (int c = 1; c <= bi::kMaxCluster; ++c) {
-    d.max_clusters[0][c] = query_clusters<bi::kModeDH>(c);
-    d.max_clusters[1][c] = query_clusters<bi::kModeDW>(c);
+    d.max_clusters[bi::kModeFwd][c] = query_clusters<bi::kModeFwd>(c);
+    d.max_clusters[bi::kModeFwdDH][c] = query_clusters<bi::kModeFwdDH>(c);
+    d.max_clusters[bi::kModeDW][c] = query_clusters<bi::kModeDW>(c);
   }
   cudaGetLastError();
   d.ok = d.sms > 0 && d.sms <= kMaxSms;
   return d.ok ? &d : nullptr;
 }
 
-int nchunks_for(int nvt) { return nvt < bi::kMaxVChunks ? nvt : bi::kMaxVChunks; }
-
-bi_status launch_fwd(const uint16_t* hidden, int64_t T, const int64_t* d_rows, const uint16_t* w, int32_t H,
-                     int32_t V, const int32_t* targets, const WsLayout& L, uint8_t* ws, int32_t* dev_status,
-                     const DevInfo* di, cudaStream_t s, uint64_t force_timeout_ns) {
-  CUtensorMap tm_h, tm_w;
-  if (!make_map(&tm_h, hidden, T, H, bi::kFwdBM) || !make_map(&tm_w, w, V, H, bi::kFwdBN)) return BI_ERR_CUDA;
-  bi::FwdArgs a{};
-  a.T = T;
-  a.d_rows = d_rows;
-  a.H = H;
-  a.V = V;
-  a.nvt = (V + bi::kFwdBN - 1) / bi::kFwdBN;
-  a.nchunks = nchunks_for(a.nvt);
-  a.targets = targets;
-  a.part_m = reinterpret_cast<float*>(ws + L.part_m);
-  a.part_s = reinterpret_cast<float*>(ws + L.part_s);
-  a.part_zy = reinterpret_cast<float*>(ws + L.part_zy);
-  a.status = dev_status;
-  a.limit_ns = kWaitLimitNs;
-  a.force_timeout_ns = force_timeout_ns;
-  const int64_t units = ((T + bi::kFwdBM - 1) / bi::kFwdBM) * a.nchunks;
-  const int grid = static_cast<int>(units < di->sms ? units : di->sms);
-  ProfScope ps(kKFwd, s);
-  bi::k_fwd_logits<<<grid, bi::kFwdThreads, bi::kFwdSmemBytes, s>>>(tm_h, tm_w, a);
-  return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
-}
-
-// Backward tiling for H: the split with the widest logit tile (NZ), then the most SMs in use.
-struct BwdPlan {
+// Tiling for H: the split with the widest logit tile (NZ), then the most SMs in use.  It depends
+// on H and the device only, so every call on a device (any T, any entry point) sees the same
+// vocabulary tiles and the same C partial-sum classes: the bits of a row's logprob are a
+// function of the row alone.
+struct LmPlan {
   int C = 0, Hs = 0, NZ = 0;
 };
-BwdPlan plan_bwd(int32_t H, const DevInfo* di) {
-  BwdPlan best;
+LmPlan plan_lm(int32_t H, const DevInfo* di) {
+  LmPlan best;
   int best_sms = -1;
   for (int c = 1; c <= bi::kMaxCluster; ++c) {
     if (!split_ok(H, c)) continue;
     const int hs = H / c, nz = logit_cols(hs);
-    const int sms = di->max_clusters[0][c] * c;
-    if (di->max_clusters[0][c] <= 0 || di->max_clusters[1][c] <= 0) continue;
+    if (di->max_clusters[0][c] <= 0 || di->max_clusters[1][c] <= 0 || di->max_clusters[2][c] <= 0) continue;
+    const int sms = di->max_clusters[1][c] * c;
     if (nz > best.NZ || (nz == best.NZ && sms > best_sms)) {
       best.C = c;
       best.Hs = hs;
@@ -275,18 +260,18 @@ BwdPlan plan_bwd(int32_t H, const DevInfo* di) {
 }
 
 template <int kMode, int kNZ, int kHS>
-bi_status launch_bwd(const CUtensorMap& tm_stat, const CUtensorMap& tm_zb, const CUtensorMap& tm_sl,
-                     const CUtensorMap& tm_dz, const bi::BwdArgs& a, int64_t units_upper, const DevInfo* di,
-                     cudaStream_t s) {
-  const int smem = bi::BwdTile<kNZ, kHS>::smem;
+bi_status launch_lm(const CUtensorMap& tm_stat, const CUtensorMap& tm_zb, const CUtensorMap& tm_sl,
+                    const CUtensorMap& tm_dz, const bi::LmArgs& a, int64_t units_upper, const DevInfo* di,
+                    cudaStream_t s) {
+  const int smem = bi::LmTile<kNZ, kHS>::smem;
   const int maxc = di->max_clusters[kMode][a.C];
   if (maxc <= 0) return BI_ERR_CUDA;
   int64_t ncl = units_upper < maxc ? units_upper : maxc;
   if (ncl < 1) ncl = 1;
-  if (ncl * a.C * bi::kSlotsPerCta > kDzSlotsMax) return BI_ERR_CUDA;
+  if (ncl * a.C * bi::kSlotsPerCta > kDzSlotsMax || ncl * a.C > kMaxSms) return BI_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(ncl * a.C), 1, 1);
-  cfg.blockDim = dim3(bi::kBwdThreads, 1, 1);
+  cfg.blockDim = dim3(bi::LmThreads<kMode>::value, 1, 1);
   cfg.dynamicSmemBytes = static_cast<size_t>(smem);
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -296,13 +281,52 @@ bi_status launch_bwd(const CUtensorMap& tm_stat, const CUtensorMap& tm_zb, const
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  ProfScope ps(kMode == bi::kModeDH ? kKBwdDH : kKBwdDW, s);
-  return cudaLaunchKernelEx(&cfg, bi::k_bwd_cluster<kMode, kNZ, kHS>, tm_stat, tm_zb, tm_sl, tm_dz, a) == cudaSuccess
+  ProfScope ps(kMode == bi::kModeFwd ? kKLmFwd : (kMode == bi::kModeFwdDH ? kKLmFwdDH : kKLmDW), s);
+  return cudaLaunchKernelEx(&cfg, bi::k_lm_cluster<kMode, kNZ, kHS>, tm_stat, tm_zb, tm_sl, tm_dz, a) == cudaSuccess
              ? BI_OK
              : BI_ERR_CUDA;
 }
 
 unsigned blocks_for(int64_t n, int per) { return static_cast<unsigned>((n + per - 1) / per); }
+
+// The logprob-only forward (kModeFwd), shared by the two logprob entry points.
+bi_status logprob_forward(const uint16_t* hidden, const uint16_t* w_lm, const int32_t* targets, int64_t T, int32_t H,
+                          int32_t V, float* logprob, float* lse, int32_t* dev_status, float* fin,
+                          uint64_t force_timeout_ns, const DevInfo* di, cudaStream_t s) {
+  const LmPlan pl = plan_lm(H, di);
+  if (pl.C == 0) return BI_ERR_UNSUPPORTED_SHAPE;
+  CUtensorMap tm_h, tm_wz, tm_w64;
+  if (!make_map(&tm_h, hidden, T, H, 128) || !make_map(&tm_wz, w_lm, V, H, pl.NZ) ||
+      !make_map(&tm_w64, w_lm, V, H, 64))
+    return BI_ERR_CUDA;
+  bi::LmArgs a{};
+  a.H = H;
+  a.V = V;
+  a.C = pl.C;
+  a.Hs = pl.Hs;
+  a.NZ = pl.NZ;
+  a.T = T;
+  a.d_rows = nullptr;
+  a.nvz = (V + pl.NZ - 1) / pl.NZ;
+  a.nv128 = (V + 127) / 128;
+  a.w_lm = w_lm;
+  a.y = targets;
+  a.logprob = logprob;
+  a.lse_out = lse;
+  a.fin = fin;
+  a.status = dev_status;
+  a.limit_ns = kWaitLimitNs;
+  a.force_timeout_ns = force_timeout_ns;
+  const int64_t units = (T + 127) / 128;
+  bi_status st = BI_ERR_UNSUPPORTED_SHAPE;
+  // the slice and scratch maps are not read in this mode; any valid map fills their places
+#define BI_LAUNCH_FWD(NZ_, HS_)                                                                    \
+  if (pl.NZ == NZ_ && pl.Hs == HS_)                                                              \
+    st = launch_lm<bi::kModeFwd, NZ_, HS_>(tm_h, tm_wz, tm_w64, tm_w64, a, units, di, s);
+  BI_LM_CONFIGS(BI_LAUNCH_FWD)
+#undef BI_LAUNCH_FWD
+  return st;
+}
 
 }  // namespace
 
@@ -312,13 +336,13 @@ namespace {
 // Fixed scratch for bi_logprob_fwd_noalloc.  Some callers cannot allocate device memory at all:
 // code that runs inside a host framework which owns every device allocation (a serving engine's
 // fixed memory pool, a plugin given no allocator handle) has no way to hand this library a
-// workspace.  For them, the forward's per-chunk partials live in this array instead.  It is a
-// file-scope device array, so every GPU that loads the library holds it (1.5 MB) until the
-// process exits.  All calls share it: calls whose kernels overlap on the GPU (different streams,
+// workspace.  For them, the forward's per-CTA partials live in this array instead.  It is a
+// file-scope device array, so every GPU that loads the library holds it (480 KB) until the
+// process exits.  Its size depends on the SM count only (one [2][3][128] block per CTA), so any
+// T fits.  All calls share it: calls whose kernels overlap on the GPU (different streams,
 // different host threads) race on it.
 // ---------------------------------------------------------------------------------------------
-constexpr int64_t kNoAllocMaxRows = 8192;  // largest T accepted by bi_logprob_fwd_noalloc
-constexpr size_t kNoAllocFloats = 3 * static_cast<size_t>(bi::kMaxVChunks) * kNoAllocMaxRows;
+constexpr size_t kNoAllocFloats = kFinBytes / sizeof(float);
 static __device__ __align__(256) float g_noalloc_scratch[kNoAllocFloats];
 
 // The array's name is only a host-side stand-in; the kernel needs its device address, looked up
@@ -336,7 +360,6 @@ float* noalloc_scratch_address() {
   }
   return addr[dev];
 }
-
 
 }  // namespace
 
@@ -414,24 +437,17 @@ bi_status bi_logprob_fwd(const uint16_t* hidden, const uint16_t* w_lm, const int
   if (!di) return BI_ERR_CUDA;
   if (cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s) != cudaSuccess) return BI_ERR_CUDA;
   if (T == 0) return BI_OK;
-  uint8_t* w8 = static_cast<uint8_t*>(ws);
-  bi_status st = launch_fwd(hidden, T, nullptr, w_lm, H, V, targets, L, w8, dev_status, di, s, force);
-  if (st != BI_OK) return st;
-  const int nvt = (V + bi::kFwdBN - 1) / bi::kFwdBN;
-  ProfScope ps(kKCombineLp, s);
-  bi::k_combine_logprob<<<blocks_for(T, 256), 256, 0, s>>>(
-      reinterpret_cast<float*>(w8 + L.part_m), reinterpret_cast<float*>(w8 + L.part_s),
-      reinterpret_cast<float*>(w8 + L.part_zy), T, nchunks_for(nvt), nvt, V, targets, logprob, lse, dev_status);
-  return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+  float* fin = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + L.fin);
+  return logprob_forward(hidden, w_lm, targets, T, H, V, logprob, lse, dev_status, fin, force, di, s);
 }
 
-// Same computation as bi_logprob_fwd, with the chunk partials in the library's fixed scratch
-// array instead of a caller workspace: no device allocation by anyone.  T <= 8192.
+// Same computation as bi_logprob_fwd (same kernel, same tiles, same bits), with the per-CTA
+// partials in the library's fixed scratch array instead of a caller workspace: no device
+// allocation by anyone.
 bi_status bi_logprob_fwd_noalloc(const uint16_t* hidden, const uint16_t* w_lm, const int32_t* targets, int64_t T,
                                  int32_t H, int32_t V, float* logprob, float* lse, int32_t* dev_status,
                                  void* stream) {
-  if (T < 0 || H <= 0 || V <= 0) return BI_ERR_INVALID_ARG;
-  if (T > kNoAllocMaxRows) return BI_ERR_WORKSPACE;  // the fixed scratch holds 8192 rows
+  if (T < 0 || T >= (int64_t(1) << 31) || H <= 0 || V <= 0) return BI_ERR_INVALID_ARG;
   if (!dev_status || (T > 0 && (!hidden || !w_lm || !targets || !logprob))) return BI_ERR_INVALID_ARG;
   if (T > 0 && (!aligned16(hidden) || !aligned16(w_lm))) return BI_ERR_INVALID_ARG;
   if (H % 64 != 0 || cluster_split(H) == 0) return BI_ERR_UNSUPPORTED_SHAPE;
@@ -442,19 +458,7 @@ bi_status bi_logprob_fwd_noalloc(const uint16_t* hidden, const uint16_t* w_lm, c
   if (!scratch) return BI_ERR_CUDA;
   if (cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s) != cudaSuccess) return BI_ERR_CUDA;
   if (T == 0) return BI_OK;
-  // partials [3][kMaxVChunks][T] carved from the scratch; every entry read is written first
-  WsLayout L{};
-  L.part_m = 0;
-  L.part_s = static_cast<size_t>(bi::kMaxVChunks) * static_cast<size_t>(T) * sizeof(float);
-  L.part_zy = 2 * L.part_s;
-  uint8_t* w8 = reinterpret_cast<uint8_t*>(scratch);
-  bi_status st = launch_fwd(hidden, T, nullptr, w_lm, H, V, targets, L, w8, dev_status, di, s, 0);
-  if (st != BI_OK) return st;
-  const int nvt = (V + bi::kFwdBN - 1) / bi::kFwdBN;
-  bi::k_combine_logprob<<<blocks_for(T, 256), 256, 0, s>>>(
-      reinterpret_cast<float*>(w8 + L.part_m), reinterpret_cast<float*>(w8 + L.part_s),
-      reinterpret_cast<float*>(w8 + L.part_zy), T, nchunks_for(nvt), nvt, V, targets, logprob, lse, dev_status);
-  return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+  return logprob_forward(hidden, w_lm, targets, T, H, V, logprob, lse, dev_status, scratch, 0, di, s);
 }
 
 bi_status bi_is_loss_fwd_bwd(const uint16_t* hidden, const uint16_t* w_lm, const int32_t* targets,
@@ -470,14 +474,14 @@ bi_status bi_is_loss_fwd_bwd(const uint16_t* hidden, const uint16_t* w_lm, const
   if (T > 0 && (!hidden || !targets || !rollout_logprob || !logprob || !grad_hidden)) return BI_ERR_INVALID_ARG;
   if (!aligned16(w_lm) || !aligned16(grad_w) || (T > 0 && (!aligned16(hidden) || !aligned16(grad_hidden))))
     return BI_ERR_INVALID_ARG;
-  if (H % 64 != 0) return BI_ERR_UNSUPPORTED_SHAPE;
-  const int C = cluster_split(H);
-  if (C == 0) return BI_ERR_UNSUPPORTED_SHAPE;
+  if (H % 64 != 0 || cluster_split(H) == 0) return BI_ERR_UNSUPPORTED_SHAPE;
   const WsLayout L = ws_layout(T, H, R);
   if (!ws || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) return BI_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const DevInfo* di = device_info();
   if (!di) return BI_ERR_CUDA;
+  const LmPlan pl = plan_lm(H, di);
+  if (pl.C == 0) return BI_ERR_UNSUPPORTED_SHAPE;
   if (cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s) != cudaSuccess) return BI_ERR_CUDA;
 
   uint8_t* w8 = static_cast<uint8_t*>(ws);
@@ -487,10 +491,11 @@ bi_status bi_is_loss_fwd_bwd(const uint16_t* hidden, const uint16_t* w_lm, const
   auto I = [&](size_t o) { return reinterpret_cast<int32_t*>(w8 + o); };
   const double rstar = resp_normalizer > 0.0 ? resp_normalizer : static_cast<double>(R);
 
-  { ProfScope ps(kKPrep, s);
-  bi::k_prep<<<1, 1024, 0, s>>>(rewards, resp_offsets, group_offsets, prompt_lens, R, G, rstar, T,
-                                reinterpret_cast<double*>(w8 + L.coef), reinterpret_cast<int64_t*>(w8 + L.cprefix),
-                                ctrl, dev_status);
+  {
+    ProfScope ps(kKPrep, s);
+    bi::k_prep<<<1, 1024, 0, s>>>(rewards, resp_offsets, group_offsets, prompt_lens, R, G, rstar, T,
+                                  reinterpret_cast<double*>(w8 + L.coef), reinterpret_cast<int64_t*>(w8 + L.cprefix),
+                                  ctrl, dev_status);
   }
   if (T > 0) {
     ProfScope ps(kKRowmap, s);
@@ -513,29 +518,6 @@ bi_status bi_is_loss_fwd_bwd(const uint16_t* hidden, const uint16_t* w_lm, const
   }
   if (cudaGetLastError() != cudaSuccess) return BI_ERR_CUDA;
 
-  const int nvt = (V + bi::kFwdBN - 1) / bi::kFwdBN;
-  if (T > 0) {
-    bi_status st = launch_fwd(hc, T, d_rows, w_lm, H, V, I(L.y_c), L, w8, dev_status, di, s, 0);
-    if (st != BI_OK) return st;
-  }
-  RedPart* parts = reinterpret_cast<RedPart*>(w8 + L.red);
-  {
-  ProfScope ps(kKCombineIs, s);
-  bi::k_combine_is<<<L.nred, bi::kRedBlock, 0, s>>>(F(L.part_m), F(L.part_s), F(L.part_zy), T > 0 ? T : 1,
-                                                    nchunks_for(nvt), nvt, V, ctrl, I(L.y_c), F(L.logmu_c),
-                                                    I(L.respof), I(L.rowmap), reinterpret_cast<double*>(w8 + L.coef),
-                                                    logprob, is_weight, token_loss, F(L.lse_c), F(L.g_c), parts,
-                                                    dev_status);
-  }
-  {
-  ProfScope ps(kKReduce, s);
-  bi::k_reduce_parts<<<1, 1024, 0, s>>>(parts, L.nred, loss, reinterpret_cast<bi::D3Out*>(d3), dev_status);
-  }
-  if (cudaGetLastError() != cudaSuccess) return BI_ERR_CUDA;
-
-  // backward: dH (row tiles) and dW (vocabulary tiles)
-  const BwdPlan pl = plan_bwd(H, di);
-  if (pl.C == 0) return BI_ERR_UNSUPPORTED_SHAPE;
   CUtensorMap tm_h128, tm_hz, tm_h64, tm_w128, tm_wz, tm_w64, tm_dz;
   const int64_t trows = T > 0 ? T : 1;
   const void* hsrc = hc ? static_cast<const void*>(hc) : static_cast<const void*>(w8 + L.hc);
@@ -544,7 +526,7 @@ bi_status bi_is_loss_fwd_bwd(const uint16_t* hidden, const uint16_t* w_lm, const
       !make_map(&tm_wz, w_lm, V, H, pl.NZ) || !make_map(&tm_w64, w_lm, V, H, 64) ||
       !make_map(&tm_dz, w8 + L.dz, static_cast<int64_t>(kDzSlotsMax) * 128, pl.NZ, 128))
     return BI_ERR_CUDA;
-  bi::BwdArgs a{};
+  bi::LmArgs a{};
   a.H = H;
   a.V = V;
   a.C = pl.C;
@@ -554,23 +536,47 @@ bi_status bi_is_loss_fwd_bwd(const uint16_t* hidden, const uint16_t* w_lm, const
   a.d_rows = d_rows;
   a.nvz = (V + pl.NZ - 1) / pl.NZ;
   a.nv128 = (V + 127) / 128;
-  a.lse = F(L.lse_c);
-  a.g = F(L.g_c);
+  a.w_lm = w_lm;
   a.y = I(L.y_c);
+  a.logmu = F(L.logmu_c);
+  a.respof = I(L.respof);
+  a.coef = reinterpret_cast<const double*>(w8 + L.coef);
   a.rowmap = I(L.rowmap);
+  a.lse_c = F(L.lse_c);
+  a.g_c = F(L.g_c);
+  a.tl_c = F(L.tl_c);
+  a.d3_c = F(L.d3_c);
+  a.logprob = logprob;
+  a.is_weight = is_weight;
+  a.token_loss = token_loss;
   a.grad_hidden = grad_hidden;
   a.grad_w = grad_w;
   a.dz_scratch = reinterpret_cast<uint16_t*>(w8 + L.dz);
+  a.alpha = F(L.alpha);
+  a.fin = F(L.fin);
   a.status = dev_status;
   a.limit_ns = kWaitLimitNs;
+  RedPart* parts = reinterpret_cast<RedPart*>(w8 + L.red);
   bi_status st = BI_ERR_UNSUPPORTED_SHAPE;
+  // forward + dH over row tiles, the loss and D3 reductions, then dW over vocabulary tiles
 #define BI_LAUNCH(NZ_, HS_)                                                                                  \
   if (pl.NZ == NZ_ && pl.Hs == HS_) {                                                                        \
     st = BI_OK;                                                                                            \
-    if (T > 0) st = launch_bwd<bi::kModeDH, NZ_, HS_>(tm_h128, tm_wz, tm_w64, tm_dz, a, (T + 127) / 128, di, s); \
-    if (st == BI_OK) st = launch_bwd<bi::kModeDW, NZ_, HS_>(tm_w128, tm_hz, tm_h64, tm_dz, a, a.nv128, di, s); \
+    if (T > 0) st = launch_lm<bi::kModeFwdDH, NZ_, HS_>(tm_h128, tm_wz, tm_w64, tm_dz, a, (T + 127) / 128, di, s); \
+    if (st == BI_OK) {                                                                                     \
+      {                                                                                                    \
+        ProfScope ps(kKRowParts, s);                                                                       \
+        bi::k_row_parts<<<L.nred, bi::kRedBlock, 0, s>>>(F(L.tl_c), F(L.d3_c), ctrl, parts);              \
+      }                                                                                                    \
+      {                                                                                                    \
+        ProfScope ps(kKReduce, s);                                                                         \
+        bi::k_reduce_parts<<<1, 1024, 0, s>>>(parts, L.nred, loss, reinterpret_cast<bi::D3Out*>(d3), dev_status); \
+      }                                                                                                    \
+      if (cudaGetLastError() != cudaSuccess) st = BI_ERR_CUDA;                                             \
+    }                                                                                                      \
+    if (st == BI_OK) st = launch_lm<bi::kModeDW, NZ_, HS_>(tm_w128, tm_hz, tm_h64, tm_dz, a, a.nv128, di, s); \
   }
-  BI_BWD_CONFIGS(BI_LAUNCH)
+  BI_LM_CONFIGS(BI_LAUNCH)
 #undef BI_LAUNCH
   return st;
 }
@@ -584,9 +590,9 @@ bi_status bi_d3_stats(const float* learner_logprob, const float* rollout_logprob
   if (cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s) != cudaSuccess) return BI_ERR_CUDA;
   RedPart* parts = static_cast<RedPart*>(ws);
   {
-  ProfScope ps(kKD3Partial, s);
-  bi::k_d3_partial<<<static_cast<unsigned>(nred), bi::kRedBlock, 0, s>>>(learner_logprob, rollout_logprob, mask, T,
-                                                                         parts);
+    ProfScope ps(kKD3Partial, s);
+    bi::k_d3_partial<<<static_cast<unsigned>(nred), bi::kRedBlock, 0, s>>>(learner_logprob, rollout_logprob, mask, T,
+                                                                           parts);
   }
   ProfScope ps(kKReduce, s);
   bi::k_reduce_parts<<<1, 1024, 0, s>>>(parts, static_cast<int>(nred), nullptr, reinterpret_cast<bi::D3Out*>(out),

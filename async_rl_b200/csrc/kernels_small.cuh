@@ -1,8 +1,7 @@
-// kernels_small.cuh -- the light, memory-bound steps around the two tensor-core kernels:
-// offsets validation and per-response coefficients, the scored-row map, the gather of scored
-// rows, the per-row combine (lse, log pi, IS weight, D3 term, token loss) and the fixed-order
-// reductions of the loss and the D3 statistics.  No atomics take part in any sum: every
-// reduction has a fixed tree shape that depends only on the number of rows.
+// kernels_small.cuh -- the light, memory-bound steps around the tensor-core kernels: offsets
+// validation and per-response coefficients, the scored-row map, the gather of scored rows and
+// the fixed-order reductions of the loss and the D3 statistics.  No atomics take part in any
+// sum: every reduction has a fixed tree shape that depends only on the number of rows.
 //
 // Definitions: "Zero Mismatch, Simple Async RL", sections "Only one probability gap comes from
 // old weights" (w = pi / mu, D3 = mean of w - 1 - log w) and "Alignment permits a simpler
@@ -10,7 +9,7 @@
 // no clipping, no gate).
 #pragma once
 
-#include "kernels_fwd.cuh"
+#include "sm100.cuh"
 
 namespace bi {
 
@@ -148,24 +147,6 @@ __global__ void k_gather_rows(const uint16_t* __restrict__ hidden, int64_t T, in
   }
 }
 
-__global__ void k_combine_logprob(const float* __restrict__ pm, const float* __restrict__ ps,
-                                  const float* __restrict__ pzy, int64_t T, int nchunks, int nvt, int V,
-                                  const int32_t* __restrict__ targets, float* __restrict__ logprob,
-                                  float* __restrict__ lse_out, int32_t* status) {
-  const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (t >= T) return;
-  const int32_t y = targets[t];
-  float lse, zy;
-  combine_row(pm, ps, pzy, T, t, nchunks, nvt, y, lse, zy);
-  if (y < 0 || y >= V) {
-    raise_status(status, 6 /* BI_ERR_BAD_TARGET */);
-    logprob[t] = __int_as_float(0x7fc00000);
-  } else {
-    logprob[t] = zy - lse;
-  }
-  if (lse_out) lse_out[t] = lse;
-}
-
 // Fixed-shape block reduction of a RedPart (warp butterflies, then warps in order).
 __device__ __forceinline__ RedPart block_reduce(RedPart v) {
   for (int o = 16; o > 0; o >>= 1) {
@@ -192,39 +173,16 @@ __device__ __forceinline__ RedPart block_reduce(RedPart v) {
   return out;
 }
 
-// One thread per compact row: lse and log pi (same code as the logprob-only path), then
-// delta = log pi - log mu, w = exp(delta) (unclipped), d3 = expm1(delta) - delta,
-// token loss = -c_i w, and the per-row gradient coefficient g = token loss.
-__global__ void k_combine_is(const float* __restrict__ pm, const float* __restrict__ ps,
-                             const float* __restrict__ pzy, int64_t T, int nchunks, int nvt, int V,
-                             const Ctrl* ctrl, const int32_t* __restrict__ y_c, const float* __restrict__ logmu_c,
-                             const int32_t* __restrict__ respof, const int32_t* __restrict__ rowmap,
-                             const double* __restrict__ coef, float* __restrict__ logprob,
-                             float* __restrict__ is_weight, float* __restrict__ token_loss,
-                             float* __restrict__ lse_c, float* __restrict__ g_c, RedPart* parts, int32_t* status) {
+// One thread per compact row: the block partial of the token losses and D3 terms that the
+// forward kernel left per row (loss = sum of token losses; D3 mean, max and non-finite count).
+__global__ void k_row_parts(const float* __restrict__ tl_c, const float* __restrict__ d3_c, const Ctrl* ctrl,
+                            RedPart* parts) {
   const int64_t k = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t ns = ctrl->n_scored;
   RedPart v{0.0, 0.0, -INFINITY, 0, 0, 0};
   if (k < ns) {
-    const int32_t y = y_c[k];
-    float lse, zy;
-    combine_row(pm, ps, pzy, T, k, nchunks, nvt, y, lse, zy);
-    float lp = zy - lse;
-    if (y < 0 || y >= V) {
-      raise_status(status, 6 /* BI_ERR_BAD_TARGET */);
-      lp = __int_as_float(0x7fc00000);
-    }
-    const float delta = lp - logmu_c[k];
-    const float w = expf(delta);
-    const float d3 = expm1f(delta) - delta;
-    const float tl = static_cast<float>(-coef[respof[k]] * static_cast<double>(w));
-    const int64_t r = rowmap[k];
-    logprob[r] = lp;
-    if (is_weight) is_weight[r] = w;
-    if (token_loss) token_loss[r] = tl;
-    lse_c[k] = lse;
-    g_c[k] = tl;
-    v.loss = static_cast<double>(tl);
+    const float d3 = d3_c[k];
+    v.loss = static_cast<double>(tl_c[k]);
     v.d3sum = static_cast<double>(d3);
     v.d3max = d3;
     v.count = 1;

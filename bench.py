@@ -299,8 +299,10 @@ def run_ours(args):
     peaks, peak_src = measured_peaks()
     peak_tf = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
     flops_tvh = 2.0 * T * V * H  # one LM-head contraction over the batch
-    alg = {"k_fwd_logits": flops_tvh, "k_bwd_dh": flops_tvh, "k_bwd_dw": flops_tvh}
-    executed = {"k_fwd_logits": flops_tvh, "k_bwd_dh": 2 * flops_tvh, "k_bwd_dw": 2 * flops_tvh}
+    # algorithmic: logits + dH in the fused forward, dW in the second kernel; executed adds the
+    # logit recompute of the dW kernel
+    alg = {"k_lm_fwd": flops_tvh, "k_lm_fwd_dh": 2 * flops_tvh, "k_lm_dw": flops_tvh}
+    executed = {"k_lm_fwd": flops_tvh, "k_lm_fwd_dh": 2 * flops_tvh, "k_lm_dw": 2 * flops_tvh}
     dom = max(alg, key=lambda k: prof.get(k, (0.0, 1))[0])
     dms, dn = prof.get(dom, (float("nan"), 1))
     davg = dms / max(dn, 1)

@@ -107,9 +107,11 @@ BI_API bi_status bi_logprob_fwd(const uint16_t* hidden, const uint16_t* w_lm, co
  * counterpart of this entry point; it exists for code that runs inside a host framework which
  * owns every device allocation (a serving engine's fixed memory pool, a plugin given no allocator
  * handle) and so cannot pass a workspace.  Arguments and results are those of bi_logprob_fwd
- * without the workspace; the forward's scratch lives in a fixed device array inside the library
- * (1.5 MB, held by every GPU that loads the library until the process exits).
- *   - T is limited to 8192 rows; a larger T returns BI_ERR_WORKSPACE and launches nothing.
+ * without the workspace; the forward's per-CTA partials live in a fixed device array inside the
+ * library (480 KB, one [2][3][128] float block per CTA of a full-device grid, held by every GPU
+ * that loads the library until the process exits).  Its size does not depend on T: any T that
+ * bi_logprob_fwd accepts is accepted, and the results are bit-identical to bi_logprob_fwd's
+ * (same kernel, same tiles).
  *   - The call allocates nothing (no cudaMalloc, no library allocator).  Its first call on a
  *     device looks up the array's device address with that device current; make that first call
  *     before any stream capture.

@@ -1,10 +1,7 @@
 """bi_logprob_fwd_noalloc: the entry point for callers that cannot allocate device memory (code
 inside a host framework that owns every device allocation, so it cannot pass a workspace).  It
-must give the results of bi_logprob_fwd, call after call, from its fixed scratch array, and refuse
-sizes beyond that array.  This file is collected last on purpose."""
-import ctypes
-
-import numpy as np
+must give the bits of bi_logprob_fwd, call after call, from its fixed scratch array, whose size
+does not depend on T.  This file is collected last on purpose."""
 import pytest
 import torch
 
@@ -12,11 +9,8 @@ from async_rl_b200 import _lib
 from async_rl_b200.build import build
 from workloads.synth import random_inputs
 
-from .util import LOGPROB_TOL
 
 pytestmark = pytest.mark.gpu
-
-NOALLOC_MAX_ROWS = 8192
 
 
 def _call_noalloc(lib, h, w, y, want_lse=True):
@@ -44,17 +38,12 @@ def _call_with_workspace(lib, h, w, y):
     return code, lp, lse, st
 
 
-def _close(a, b):
-    a = a.double().cpu().numpy()
-    b = b.double().cpu().numpy()
-    return np.all(np.abs(a - b) <= LOGPROB_TOL + LOGPROB_TOL * np.abs(b))
-
-
 def test_noalloc_matches_workspace_entry_point_on_consecutive_calls(cuda_device):
     build()
     lib = _lib.load()
-    # two calls in a row, the second smaller, so stale scratch from the first would show up
-    for (T, H, V, seed) in [(3000, 1536, 151936, 31), (701, 1536, 151936, 32)]:
+    # calls in a row, the second smaller, so stale scratch from the first would show up; the third
+    # has more rows than any fixed per-row scratch of a few MB could hold
+    for (T, H, V, seed) in [(3000, 1536, 151936, 31), (701, 1536, 151936, 32), (20000, 1536, 151936, 33)]:
         h, w, y = random_inputs(T, H, V, seed)
         h, w, y = h.to(cuda_device), w.to(cuda_device), y.to(cuda_device)
         code, lp, lse, st = _call_noalloc(lib, h, w, y)
@@ -63,14 +52,15 @@ def test_noalloc_matches_workspace_entry_point_on_consecutive_calls(cuda_device)
         assert rcode == 0
         torch.cuda.synchronize()
         assert int(st.item()) == 0 and int(rst.item()) == 0
-        assert _close(lp, rlp) and _close(lse, rlse)
+        assert torch.equal(lp, rlp) and torch.equal(lse, rlse)
+        assert torch.isfinite(lp).all()
 
 
-def test_noalloc_refuses_more_rows_than_its_scratch(cuda_device):
+def test_noalloc_refuses_unsupported_shape_without_launching(cuda_device):
     lib = _lib.load()
-    T = NOALLOC_MAX_ROWS + 1
-    h = torch.zeros(T, 128, dtype=torch.bfloat16, device=cuda_device)
-    w = torch.zeros(512, 128, dtype=torch.bfloat16, device=cuda_device)
+    T, H = 16, 704  # no column split of H = 704 over <= 8 CTAs has 64-multiple slices
+    h = torch.zeros(T, H, dtype=torch.bfloat16, device=cuda_device)
+    w = torch.zeros(512, H, dtype=torch.bfloat16, device=cuda_device)
     y = torch.zeros(T, dtype=torch.int32, device=cuda_device)
     code, _, _, _ = _call_noalloc(lib, h, w, y, want_lse=False)
-    assert code == 3  # BI_ERR_WORKSPACE: nothing launched
+    assert code == 2  # BI_ERR_UNSUPPORTED_SHAPE: nothing launched
