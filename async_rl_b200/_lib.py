@@ -9,7 +9,7 @@ import os
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libbi_isloss.so")
 
-EXPORTED = ("bi_workspace_bytes", "bi_logprob_fwd", "bi_logprob_fwd_noalloc", "bi_is_loss_fwd_bwd", "bi_d3_stats",
+EXPORTED = ("bi_workspace_bytes", "bi_workspace_bytes_min", "bi_logprob_fwd", "bi_logprob_fwd_noalloc", "bi_is_loss_fwd_bwd", "bi_d3_stats",
             "bi_status_string", "bi_version", "bi_debug_force_timeout_once", "bi_profile_enable",
             "bi_profile_reset", "bi_profile_read")
 
@@ -37,6 +37,8 @@ def load() -> ctypes.CDLL:
     lib = ctypes.CDLL(LIB_PATH)
     lib.bi_workspace_bytes.argtypes = [_i64, _i32, _i32, _i32]
     lib.bi_workspace_bytes.restype = _sz
+    lib.bi_workspace_bytes_min.argtypes = [_i64, _i32, _i32, _i32]
+    lib.bi_workspace_bytes_min.restype = _sz
     lib.bi_logprob_fwd.argtypes = [_p, _p, _p, _i64, _i32, _i32, _p, _p, _p, _p, _sz, _p]
     lib.bi_logprob_fwd.restype = ctypes.c_int
     lib.bi_logprob_fwd_noalloc.argtypes = [_p, _p, _p, _i64, _i32, _i32, _p, _p, _p, _p]

@@ -38,12 +38,16 @@ def _check_cuda(t: torch.Tensor, name: str, dtype: torch.dtype, device: torch.de
         raise ValueError(f"{name} must be contiguous")
 
 
-def workspace_bytes(T: int, H: int, V: int, R: int = 0) -> int:
-    return int(_lib.load().bi_workspace_bytes(T, H, V, R))
+def workspace_bytes(T: int, H: int, V: int, R: int = 0, minimal: bool = False) -> int:
+    """Workspace of the fastest path, or (minimal=True) the smallest accepted one, whose dW
+    recomputes the logits instead of reading the stored probability tiles."""
+    lib = _lib.load()
+    fn = lib.bi_workspace_bytes_min if minimal else lib.bi_workspace_bytes
+    return int(fn(T, H, V, R))
 
 
-def make_workspace(T: int, H: int, V: int, R: int = 0, device="cuda") -> torch.Tensor:
-    n = workspace_bytes(T, H, V, R)
+def make_workspace(T: int, H: int, V: int, R: int = 0, device="cuda", minimal: bool = False) -> torch.Tensor:
+    n = workspace_bytes(T, H, V, R, minimal)
     return torch.empty(max(n, 256), dtype=torch.uint8, device=device)
 
 

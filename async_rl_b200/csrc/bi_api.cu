@@ -10,6 +10,7 @@
 #include <vector>
 
 #include "bi_isloss.h"
+#include "kernels_dw.cuh"
 #include "kernels_lm.cuh"
 #include "kernels_small.cuh"
 
@@ -27,11 +28,11 @@ thread_local uint64_t g_force_timeout_ns = 0;
 // ---------------------------------------------------------------------------------------------
 // optional per-kernel timing (events around each launch; measurement tools only)
 // ---------------------------------------------------------------------------------------------
-enum KernelKind : int { kKPrep, kKRowmap, kKZeroRows, kKGather, kKLmFwd, kKLmFwdDH, kKLmDW, kKRowParts,
-                        kKReduce, kKD3Partial, kNumKinds };
+enum KernelKind : int { kKPrep, kKRowmap, kKZeroRows, kKGather, kKLmFwd, kKLmFwdDH, kKLmDW, kKDwStream,
+                        kKRowParts, kKReduce, kKD3Partial, kNumKinds };
 const char* const kKindNames[kNumKinds] = {"k_prep", "k_rowmap", "k_zero_prompt_rows", "k_gather_rows",
-                                           "k_lm_fwd", "k_lm_fwd_dh", "k_lm_dw", "k_row_parts",
-                                           "k_reduce_parts", "k_d3_partial"};
+                                           "k_lm_fwd", "k_lm_fwd_dh", "k_lm_dw", "k_dw_stream",
+                                           "k_row_parts", "k_reduce_parts", "k_d3_partial"};
 struct Pending {
   int kind;
   cudaEvent_t a, b;
@@ -80,14 +81,19 @@ struct ProfScope {  // records an event pair around one launch when profiling is
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct WsLayout {
-  size_t ctrl, lse_c, g_c, tl_c, d3_c, y_c, logmu_c, rowmap, respof, coef, cprefix, red, hc, dz, alpha, fin, total;
+  size_t ctrl, lse_c, g_c, tl_c, d3_c, y_c, logmu_c, rowmap, respof, coef, cprefix, red, hc, dz, alpha, fin;
+  size_t dzy_c, mhist, pbuf;  // the P store (loss layout with the store only)
+  size_t total;
   int nred;
+  int64_t tpad, pcols;        // rows and columns the P store is sized for
 };
 
 constexpr size_t kFinBytes = static_cast<size_t>(kMaxSms) * 2 * 384 * sizeof(float);  // [CTAs][2][3][128]
 
-// R == 0: the logprob-only layout (per-CTA partials only).  R > 0: the loss layout.
-WsLayout ws_layout(int64_t T, int32_t H, int32_t R) {
+// R == 0: the logprob-only layout (per-CTA partials only).  R > 0: the loss layout; with
+// `store`, followed by the P store of the fused forward ([Tpad][V + 256] bf16, enough for any
+// logit-tile width NZ <= 256) and the per-step reference history ([ceil(V / 128)][Tpad] float).
+WsLayout ws_layout(int64_t T, int32_t H, int32_t V, int32_t R, bool store) {
   WsLayout L{};
   const size_t t = static_cast<size_t>(T > 0 ? T : 1);
   size_t o = 0;
@@ -100,12 +106,14 @@ WsLayout ws_layout(int64_t T, int32_t H, int32_t R) {
   // R == 0 also serves bi_d3_stats, whose block partials share the region
   L.fin = take(R > 0 || kFinBytes >= nred * sizeof(RedPart) ? kFinBytes : nred * sizeof(RedPart));
   if (R > 0) {
+    // per-row arrays hold whole 128-row tiles (the dW kernel copies them in 64-row chunks)
+    const size_t tp = (t + 127) / 128 * 128;
     L.ctrl = take(256);
-    L.lse_c = take(t * 4);
-    L.g_c = take(t * 4);
+    L.lse_c = take(tp * 4);
+    L.g_c = take(tp * 4);
     L.tl_c = take(t * 4);
     L.d3_c = take(t * 4);
-    L.y_c = take(t * 4);
+    L.y_c = take(tp * 4);
     L.logmu_c = take(t * 4);
     L.rowmap = take(t * 4);
     L.respof = take(t * 4);
@@ -116,6 +124,13 @@ WsLayout ws_layout(int64_t T, int32_t H, int32_t R) {
     L.hc = take(t * static_cast<size_t>(H) * 2);
     L.dz = take(static_cast<size_t>(kDzSlotsMax) * 128 * bi::kMaxNZ * 2);
     L.alpha = take(static_cast<size_t>(kDzSlotsMax) * 128 * 4);
+    if (store) {
+      L.tpad = static_cast<int64_t>((t + 127) / 128 * 128);
+      L.pcols = (static_cast<int64_t>(V) + 127) / 128 * 128 + 256;
+      L.dzy_c = take(tp * 4);
+      L.mhist = take(static_cast<size_t>((V + 127) / 128) * static_cast<size_t>(L.tpad) * 4);
+      L.pbuf = take(static_cast<size_t>(L.tpad) * static_cast<size_t>(L.pcols) * 2);
+    }
   }
   L.total = o;
   return L;
@@ -198,6 +213,19 @@ int query_clusters(int C) {
   return n;
 }
 
+// Dynamic shared memory of a dW launch: at least half the SM's, so one CTA (and its 512 TMEM
+// columns) per SM.
+template <int kHS>
+int dw_smem() {
+  return bi::DwTile<kHS>::smem > bi::kLmSmemLimit / 2 + 1024 ? bi::DwTile<kHS>::smem : bi::kLmSmemLimit / 2 + 1024;
+}
+// Columns per dW item: the largest of 256, 192, 128, 64 that divides H.
+int dw_split(int32_t H) {
+  for (int hs = 256; hs >= 64; hs -= 64)
+    if (H % hs == 0) return hs;
+  return 0;
+}
+
 bool set_lm_attributes() {
   bool ok = true;
 #define BI_SET_ATTR(NZ_, HS_)                                                                                  \
@@ -212,6 +240,11 @@ bool set_lm_attributes() {
                                   bi::LmTile<NZ_, HS_>::smem) == cudaSuccess;
   BI_LM_CONFIGS(BI_SET_ATTR)
 #undef BI_SET_ATTR
+#define BI_SET_DW_ATTR(HS_)                                                                                     \
+  ok = ok && cudaFuncSetAttribute(bi::k_dw_stream<HS_>, cudaFuncAttributeMaxDynamicSharedMemorySize,           \
+                                  dw_smem<HS_>()) == cudaSuccess;
+  BI_DW_CONFIGS(BI_SET_DW_ATTR)
+#undef BI_SET_DW_ATTR
   return ok;
 }
 
@@ -288,6 +321,15 @@ bi_status launch_lm(const CUtensorMap& tm_stat, const CUtensorMap& tm_zb, const 
 }
 
 unsigned blocks_for(int64_t n, int per) { return static_cast<unsigned>((n + per - 1) / per); }
+
+template <int kHS>
+bi_status launch_dw(const CUtensorMap& tm_p, const CUtensorMap& tm_h, const bi::DwArgs& a, const DevInfo* di,
+                    cudaStream_t s) {
+  const int grid = a.nitems < di->sms ? a.nitems : di->sms;
+  ProfScope ps(kKDwStream, s);
+  bi::k_dw_stream<kHS><<<grid > 0 ? grid : 1, bi::kDwThreads, dw_smem<kHS>(), s>>>(tm_p, tm_h, a);
+  return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+}
 
 // The logprob-only forward (kModeFwd), shared by the two logprob entry points.
 bi_status logprob_forward(const uint16_t* hidden, const uint16_t* w_lm, const int32_t* targets, int64_t T, int32_t H,
@@ -416,9 +458,13 @@ int32_t bi_profile_read(const char** names_out, double* ms_out, int64_t* launche
 }
 
 size_t bi_workspace_bytes(int64_t T, int32_t H, int32_t V, int32_t R) {
-  (void)V;
-  if (T < 0 || H <= 0 || R < 0) return 0;
-  return ws_layout(T, H, R).total;
+  if (T < 0 || H <= 0 || V <= 0 || R < 0) return 0;
+  return ws_layout(T, H, V, R, R > 0).total;
+}
+
+size_t bi_workspace_bytes_min(int64_t T, int32_t H, int32_t V, int32_t R) {
+  if (T < 0 || H <= 0 || V <= 0 || R < 0) return 0;
+  return ws_layout(T, H, V, R, false).total;
 }
 
 bi_status bi_logprob_fwd(const uint16_t* hidden, const uint16_t* w_lm, const int32_t* targets, int64_t T, int32_t H,
@@ -430,7 +476,7 @@ bi_status bi_logprob_fwd(const uint16_t* hidden, const uint16_t* w_lm, const int
   if (!dev_status || (T > 0 && (!hidden || !w_lm || !targets || !logprob))) return BI_ERR_INVALID_ARG;
   if (T > 0 && (!aligned16(hidden) || !aligned16(w_lm))) return BI_ERR_INVALID_ARG;
   if (H % 64 != 0 || cluster_split(H) == 0) return BI_ERR_UNSUPPORTED_SHAPE;
-  const WsLayout L = ws_layout(T, H, 0);
+  const WsLayout L = ws_layout(T, H, V, 0, false);
   if (!ws || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) return BI_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const DevInfo* di = device_info();
@@ -475,7 +521,10 @@ bi_status bi_is_loss_fwd_bwd(const uint16_t* hidden, const uint16_t* w_lm, const
   if (!aligned16(w_lm) || !aligned16(grad_w) || (T > 0 && (!aligned16(hidden) || !aligned16(grad_hidden))))
     return BI_ERR_INVALID_ARG;
   if (H % 64 != 0 || cluster_split(H) == 0) return BI_ERR_UNSUPPORTED_SHAPE;
-  const WsLayout L = ws_layout(T, H, R);
+  // the full workspace keeps the P tiles for dW; the minimum one makes dW recompute the logits
+  const WsLayout Lfull = ws_layout(T, H, V, R, true);
+  const bool store = ws_bytes >= Lfull.total && dw_split(H) != 0;
+  const WsLayout L = store ? Lfull : ws_layout(T, H, V, R, false);
   if (!ws || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) return BI_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const DevInfo* di = device_info();
@@ -518,13 +567,17 @@ bi_status bi_is_loss_fwd_bwd(const uint16_t* hidden, const uint16_t* w_lm, const
   }
   if (cudaGetLastError() != cudaSuccess) return BI_ERR_CUDA;
 
-  CUtensorMap tm_h128, tm_hz, tm_h64, tm_w128, tm_wz, tm_w64, tm_dz;
+  CUtensorMap tm_h128, tm_hz, tm_h64, tm_w128, tm_wz, tm_w64, tm_dz, tm_p64;
   const int64_t trows = T > 0 ? T : 1;
+  const int nvz = (V + pl.NZ - 1) / pl.NZ;
+  const int64_t p_ld = static_cast<int64_t>(nvz) * pl.NZ;  // <= L.pcols
   const void* hsrc = hc ? static_cast<const void*>(hc) : static_cast<const void*>(w8 + L.hc);
   if (!make_map(&tm_h128, hsrc, trows, H, 128) || !make_map(&tm_hz, hsrc, trows, H, pl.NZ) ||
       !make_map(&tm_h64, hsrc, trows, H, 64) || !make_map(&tm_w128, w_lm, V, H, 128) ||
-      !make_map(&tm_wz, w_lm, V, H, pl.NZ) || !make_map(&tm_w64, w_lm, V, H, 64) ||
-      !make_map(&tm_dz, w8 + L.dz, static_cast<int64_t>(kDzSlotsMax) * 128, pl.NZ, 128))
+      !make_map(&tm_wz, w_lm, V, H, pl.NZ) || !make_map(&tm_w64, w_lm, V, H, 64))
+    return BI_ERR_CUDA;
+  if (store ? !(make_map(&tm_dz, w8 + L.pbuf, L.tpad, p_ld, 128) && make_map(&tm_p64, w8 + L.pbuf, L.tpad, p_ld, 64))
+            : !make_map(&tm_dz, w8 + L.dz, static_cast<int64_t>(kDzSlotsMax) * 128, pl.NZ, 128))
     return BI_ERR_CUDA;
   bi::LmArgs a{};
   a.H = H;
@@ -556,6 +609,32 @@ bi_status bi_is_loss_fwd_bwd(const uint16_t* hidden, const uint16_t* w_lm, const
   a.fin = F(L.fin);
   a.status = dev_status;
   a.limit_ns = kWaitLimitNs;
+  bi::DwArgs da{};
+  if (store) {
+    a.pbuf = reinterpret_cast<uint16_t*>(w8 + L.pbuf);
+    a.p_ld = p_ld;
+    a.mhist = F(L.mhist);
+    a.Tpad = L.tpad;
+    a.dzy_c = F(L.dzy_c);
+    da.H = H;
+    da.V = V;
+    da.Hs = dw_split(H);
+    da.nsl = H / da.Hs;
+    da.NZf = pl.NZ;
+    da.nvz = nvz;
+    da.Tpad = L.tpad;
+    da.d_rows = d_rows;
+    da.nv128 = a.nv128;
+    da.nitems = a.nv128 * da.nsl;
+    da.lse_c = F(L.lse_c);
+    da.g_c = F(L.g_c);
+    da.y_c = I(L.y_c);
+    da.dzy_c = F(L.dzy_c);
+    da.mhist = F(L.mhist);
+    da.grad_w = grad_w;
+    da.status = dev_status;
+    da.limit_ns = kWaitLimitNs;
+  }
   RedPart* parts = reinterpret_cast<RedPart*>(w8 + L.red);
   bi_status st = BI_ERR_UNSUPPORTED_SHAPE;
   // forward + dH over row tiles, the loss and D3 reductions, then dW over vocabulary tiles
@@ -574,10 +653,17 @@ bi_status bi_is_loss_fwd_bwd(const uint16_t* hidden, const uint16_t* w_lm, const
       }                                                                                                    \
       if (cudaGetLastError() != cudaSuccess) st = BI_ERR_CUDA;                                             \
     }                                                                                                      \
-    if (st == BI_OK) st = launch_lm<bi::kModeDW, NZ_, HS_>(tm_w128, tm_hz, tm_h64, tm_dz, a, a.nv128, di, s); \
+    if (st == BI_OK && !store) st = launch_lm<bi::kModeDW, NZ_, HS_>(tm_w128, tm_hz, tm_h64, tm_dz, a, a.nv128, di, s); \
   }
   BI_LM_CONFIGS(BI_LAUNCH)
 #undef BI_LAUNCH
+  if (st == BI_OK && store) {
+    st = BI_ERR_UNSUPPORTED_SHAPE;
+#define BI_LAUNCH_DW(HS_) \
+    if (da.Hs == HS_) st = launch_dw<HS_>(tm_p64, tm_h64, da, di, s);
+    BI_DW_CONFIGS(BI_LAUNCH_DW)
+#undef BI_LAUNCH_DW
+  }
   return st;
 }
 

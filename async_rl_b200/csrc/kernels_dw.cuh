@@ -1,0 +1,305 @@
+// kernels_dw.cuh -- dW from the stored probability tiles: a persistent GEMM dW = dZ^T H whose
+// A operand is transformed in shared memory on its way to the tensor cores.
+//
+// The fused forward (kernels_lm.cuh, kModeFwdDH with a P store) leaves, for every scored row t
+// and vocabulary column v, P[t][v] = bf16(e^{z_tv - m_tj}) (0 at the target column), the
+// reference m_tj of the vocabulary step j that holds v, lse_t, g_t = -c_i w_t and the target
+// entry dZ_{t,y_t} = g_t (1 - p_{t,y_t}) = g_t s'_t / s_t.  Then
+//     dZ_tv = -g_t e^{m_tj - lse_t} P[t][v]     (v != y_t),      dZ_{t,y_t} as stored,
+//     dW_v  = sum_t dZ_tv h_t.
+// ("Zero Mismatch, Simple Async RL", section "Alignment permits a simpler learning path": the
+// gradient of the unclipped token-level IS loss through the LM head.)
+//
+// Work item = (128-row vocabulary tile u, Hs-column slice q of H); a CTA owns one item at a time
+// (grid = one CTA per SM, items strided by the grid) and sweeps the tokens in chunks of 64:
+//   TMA warp     P^T chunk [128 v x 64 t] (two MN-major boxes) + H chunk [64 t x Hs] -> stage
+//   transform    8 warps rewrite the P chunk in place into bf16 dZ^T (per-token scale, target)
+//   MMA lane     O[128 x Hs] += dZ^T chunk * H chunk (A and B MN-major), O double-buffered in TMEM
+//   drain        4 warps write the finished O of an item to dW while the next item accumulates
+// The six slices of one vocabulary tile run on neighbouring CTAs at the same time, so a P chunk
+// is read from HBM once and from L2 by the other five.
+#pragma once
+
+#include "kernels_lm.cuh"
+
+namespace bi {
+
+constexpr int kDwThreads = 448;  // TMA warp, MMA warp, 8 transform warps, 4 drain warps
+constexpr int kDwXfThreads = 256;
+constexpr int kDwAUnit = 8192;   // [64 tokens][64 vocabulary] bf16, 128B-swizzled
+constexpr int kDwABytes = 2 * kDwAUnit;
+constexpr int kDwTokBytes = 6 * 256;  // per chunk: lse, g, y, dZ_y, m (first half), m (second half) x 64 tokens
+
+#define BI_DW_CONFIGS(X) X(64) X(128) X(192) X(256)
+
+struct DwArgs {
+  int32_t H, V;
+  int32_t Hs;               // columns per item (multiple of 64, <= 256)
+  int32_t nsl;              // H / Hs
+  int32_t NZf;              // vocabulary step width of the forward (granularity of the references)
+  int32_t nvz;              // steps of the forward (rows of the reference history)
+  int64_t Tpad;             // leading dimension of the reference history (rows of the P store);
+                            // every per-row array below holds Tpad entries
+  const int64_t* d_rows;    // number of scored rows on the device
+  int32_t nv128;            // ceil(V / 128)
+  int32_t nitems;           // nv128 * nsl
+  const float* lse_c;       // [rows]
+  const float* g_c;         // [rows]
+  const int32_t* y_c;       // [rows]
+  const float* dzy_c;       // [rows] dZ at the target column
+  const float* mhist;       // [nvz][Tpad] reference of each row at each vocabulary step
+  float* grad_w;            // [V, H] fp32
+  int32_t* status;
+  uint64_t limit_ns;
+};
+
+struct DwShared {
+  uint64_t full[kMaxStages];    // TMA -> transform (transaction bytes)
+  uint64_t tready[kMaxStages];  // transform (256 threads) -> MMA
+  uint64_t empty[kMaxStages];   // MMA commit -> TMA
+  uint64_t o_full[2], o_empty[2];
+  uint64_t mma_done;
+  uint32_t tmem_base;
+  volatile uint32_t abort_flag;
+};
+
+constexpr int kDwSharedBytes = static_cast<int>((sizeof(DwShared) + 127) / 128 * 128);
+
+template <int kHS>
+struct DwTile {
+  static constexpr int tok_off = kDwABytes + kHS * 128;  // per-token values after the two tiles
+  static constexpr int stage_bytes = (tok_off + kDwTokBytes + 1023) / 1024 * 1024;
+  static constexpr int fit = (kLmSmemLimit - kDwSharedBytes) / stage_bytes;
+  static constexpr int nstages = fit < kMaxStages ? fit : kMaxStages;
+  static constexpr int smem = nstages * stage_bytes + kDwSharedBytes;
+  static_assert(kHS % 64 == 0 && kHS <= 256, "two accumulators of Hs columns fill at most 512 TMEM columns");
+  static_assert(nstages >= 2, "pipeline needs at least two stages");
+};
+
+__device__ __forceinline__ bool dw_wait(DwShared& sh, const DwArgs& a, uint64_t* bar, uint32_t parity) {
+  const WaitCtl wc{&sh.abort_flag, a.status, a.limit_ns};
+  return mbar_wait<false>(bar, parity, wc);
+}
+
+// generic-proxy writes to shared memory -> visible to the tensor cores' (async proxy) reads
+__device__ __forceinline__ void fence_proxy_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+template <int kHS>
+__global__ void __launch_bounds__(kDwThreads, 1)
+    k_dw_stream(const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_h, DwArgs a) {
+  extern __shared__ __align__(1024) uint8_t dsmem[];
+  constexpr int nst = DwTile<kHS>::nstages;
+  constexpr uint32_t sbytes = DwTile<kHS>::stage_bytes;
+  DwShared& sh = *reinterpret_cast<DwShared*>(dsmem + nst * sbytes);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kMaxStages; ++i) {
+      mbar_init(&sh.full[i], 1);
+      mbar_init(&sh.tready[i], kDwXfThreads);
+      mbar_init(&sh.empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sh.o_full[i], 1);
+      mbar_init(&sh.o_empty[i], 128);
+    }
+    mbar_init(&sh.mma_done, 1);
+    sh.abort_flag = 0u;
+    fence_mbar_init_cluster();
+  }
+  if (warp == 1) {
+    tmem_alloc(&sh.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sh.tmem_base;
+  const uint32_t ring = smem_u32(dsmem);
+  const bool misaligned = (ring & 1023u) != 0;
+  if (misaligned && threadIdx.x == 0) raise_status(a.status, 4 /* BI_ERR_CUDA */);
+  const int64_t rows = misaligned ? 0 : *a.d_rows;
+  const int nk = static_cast<int>((rows + 63) / 64);  // token chunks per item
+  const int nitems = misaligned ? 0 : a.nitems;
+
+  if (warp == 0) {
+    // ---------------- TMA ----------------
+    if (lane == 0 && nk > 0) {
+      tma_prefetch_desc(&tm_p);
+      tma_prefetch_desc(&tm_h);
+      uint32_t stage = 0, phase = 0;
+      bool ok = true;
+      for (int it = blockIdx.x; ok && it < nitems; it += gridDim.x) {
+        const int u = it / a.nsl, q = it - (it / a.nsl) * a.nsl;
+        // forward steps of the two 64-column halves (a half past V reads a valid, unused row)
+        const int jm0 = min((u * 128) / a.NZf, a.nvz - 1);
+        const int jm1 = min((u * 128 + 64) / a.NZf, a.nvz - 1);
+#pragma unroll 1
+        for (int k = 0; k < nk; ++k) {
+          if (!dw_wait(sh, a, &sh.empty[stage], phase ^ 1u)) { ok = false; break; }
+          mbar_arrive_expect_tx(&sh.full[stage], DwTile<kHS>::tok_off + kDwTokBytes);
+          const uint32_t dst = ring + stage * sbytes;
+          tma_load_2d(dst, &tm_p, &sh.full[stage], u * 128, k * 64);
+          tma_load_2d(dst + kDwAUnit, &tm_p, &sh.full[stage], u * 128 + 64, k * 64);
+#pragma unroll
+          for (int m = 0; m < kHS / 64; ++m)
+            tma_load_2d(dst + kDwABytes + m * kDwAUnit, &tm_h, &sh.full[stage], q * kHS + m * 64, k * 64);
+          // the chunk's per-token values (64 x 4 bytes each; the arrays hold Tpad >= 64 nk entries)
+          const uint32_t tok = dst + DwTile<kHS>::tok_off;
+          const int64_t t0 = static_cast<int64_t>(k) * 64;
+          bulk_load(tok, a.lse_c + t0, 256, &sh.full[stage]);
+          bulk_load(tok + 256, a.g_c + t0, 256, &sh.full[stage]);
+          bulk_load(tok + 512, a.y_c + t0, 256, &sh.full[stage]);
+          bulk_load(tok + 768, a.dzy_c + t0, 256, &sh.full[stage]);
+          bulk_load(tok + 1024, a.mhist + static_cast<int64_t>(jm0) * a.Tpad + t0, 256, &sh.full[stage]);
+          bulk_load(tok + 1280, a.mhist + static_cast<int64_t>(jm1) * a.Tpad + t0, 256, &sh.full[stage]);
+          ring_advance(stage, phase, nst);
+        }
+      }
+      for (uint32_t i = 0; i < static_cast<uint32_t>(nst); ++i) {
+        const uint32_t ph = (i < stage) ? phase : (phase ^ 1u);
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_test(&sh.full[i], ph))
+          if (globaltimer_ns() - t0 > a.limit_ns) break;
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------- MMA ----------------
+    if (lane == 0 && nk > 0) {
+      constexpr uint32_t idesc = idesc_bf16(128, kHS, true, true);
+      const uint64_t da0 = sdesc_mn_sw128(ring, kDwAUnit);
+      const uint64_t db0 = sdesc_mn_sw128(ring + kDwABytes, kDwAUnit);
+      constexpr uint64_t sb = sbytes >> 4;
+      uint32_t stage = 0, phase = 0, n_it = 0;
+      bool ok = true;
+      for (int it = blockIdx.x; ok && it < nitems; it += gridDim.x, ++n_it) {
+        const uint32_t b = n_it & 1u;
+        if (!dw_wait(sh, a, &sh.o_empty[b], ((n_it >> 1) & 1u) ^ 1u)) break;
+        tc_fence_after();
+        const uint32_t acc = tmem + b * kHS;
+#pragma unroll 1
+        for (int k = 0; k < nk; ++k) {
+          if (!dw_wait(sh, a, &sh.tready[stage], phase)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)  // 16 tokens = 16 MN-major rows of 128 B = 2 KB
+            umma_bf16(acc, da0 + stage * sb + kk * (2048 >> 4), db0 + stage * sb + kk * (2048 >> 4), idesc,
+                      (k > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(&sh.empty[stage]);
+          ring_advance(stage, phase, nst);
+        }
+        if (!ok) break;
+        umma_commit(&sh.o_full[b]);
+      }
+      umma_commit(&sh.mma_done);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_test(&sh.mma_done, 0))
+        if (globaltimer_ns() - t0 > a.limit_ns) break;
+    }
+    __syncwarp();
+  } else if (warp < 10) {
+    // ---------------- transform: P chunk -> dZ^T chunk, in place ----------------
+    // Two warps per SM sub-partition: the rewrite is a short dependent chain per 16-byte chunk,
+    // and a second warp hides its latency.
+    const int tt = threadIdx.x - 64;  // 0..255
+    uint32_t stage = 0, phase = 0;
+    bool ok = true;
+    for (int it = blockIdx.x; ok && nk > 0 && it < nitems; it += gridDim.x) {
+      const int u = it / a.nsl;
+#pragma unroll 1
+      for (int k = 0; k < nk; ++k) {
+        if (!dw_wait(sh, a, &sh.full[stage], phase)) { ok = false; break; }
+        const uint32_t base = ring + stage * sbytes;
+        const float* tok = reinterpret_cast<const float*>(dsmem + stage * sbytes + DwTile<kHS>::tok_off);
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          // 16-byte chunk c = tt + 256 i of each 8 KB half: token row tl, logical chunk cq
+          const int c = tt + 256 * i;
+          const int tl = c >> 3, cq = c & 7;
+          const int64_t t = static_cast<int64_t>(k) * 64 + tl;
+          const bool tv = t < rows;
+          const float lse = tok[tl], g = tok[64 + tl], dzy = tok[192 + tl];
+          const int32_t yy = tv ? reinterpret_cast<const int32_t*>(tok)[128 + tl] : -1;
+          const uint32_t off = static_cast<uint32_t>(tl * 128 + ((cq ^ (tl & 7)) << 4));
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            // a half at or past V has no forward step (and P there is zero-filled); the two halves
+            // each lie inside one forward step (NZf is a multiple of 64)
+            const bool hv = tv && (u * 128 + h * 64 < a.V);
+            const float sig = hv ? -g * ex2_approx((tok[256 + 64 * h + tl] - lse) * kLog2e) : 0.f;
+            const uint32_t sig2 = pack_bf16x2(sig, sig);
+            const uint32_t addr = base + h * kDwAUnit + off;
+            uint32_t w[4];
+            asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
+                         : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                         : "r"(addr));
+#pragma unroll
+            for (int e = 0; e < 4; ++e) asm("mul.rn.bf16x2 %0, %0, %1;" : "+r"(w[e]) : "r"(sig2));
+            // the target column (stored as 0) takes g (1 - p_y); rare, so a branch
+            const uint32_t dv = static_cast<uint32_t>(yy - (u * 128 + h * 64 + cq * 8));
+            if (dv < 8u) {
+              const uint32_t bz = pack_bf16x2(dzy, dzy);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const uint32_t m = ((dv == 2u * e) ? 0x0000ffffu : 0u) | ((dv == 2u * e + 1u) ? 0xffff0000u : 0u);
+                w[e] = (w[e] & ~m) | (bz & m);
+              }
+            }
+            asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(w[0]), "r"(w[1]), "r"(w[2]),
+                         "r"(w[3])
+                         : "memory");
+          }
+        }
+        fence_proxy_async_shared();
+        mbar_arrive(&sh.tready[stage]);
+        ring_advance(stage, phase, nst);
+      }
+    }
+  } else {
+    // ---------------- drain: O -> dW rows ----------------
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t tl = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    uint32_t n_it = 0;
+    for (int it = blockIdx.x; it < nitems; it += gridDim.x, ++n_it) {
+      const int u = it / a.nsl, q = it - (it / a.nsl) * a.nsl;
+      const int64_t v = static_cast<int64_t>(u) * 128 + row;
+      float* dst = (v < a.V) ? a.grad_w + v * a.H + q * kHS : nullptr;
+      const uint32_t b = n_it & 1u;
+      if (nk == 0) {  // no scored rows: the gradient is zero
+        if (dst)
+          for (int c = 0; c < kHS / 4; ++c) reinterpret_cast<float4*>(dst)[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+        continue;
+      }
+      const WaitCtl wc{&sh.abort_flag, a.status, a.limit_ns};
+      if (!__all_sync(0xffffffffu, mbar_wait<false>(&sh.o_full[b], (n_it >> 1) & 1u, wc))) break;
+      tc_fence_after();
+#pragma unroll 1
+      for (int c = 0; c < kHS / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tl + b * kHS + c * 32, r);
+        tmem_ld_wait();
+        if (dst) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) d4[e] = make_uint4(r[4 * e], r[4 * e + 1], r[4 * e + 2], r[4 * e + 3]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&sh.o_empty[b]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace bi

@@ -95,6 +95,12 @@ struct LmArgs {
   float* token_loss;       // nullable
   uint16_t* grad_hidden;   // [*, H] bf16 (kModeFwdDH)
   float* grad_w;           // [V, H] fp32 (kModeDW)
+  // P store (kModeFwdDH, optional): every P tile stays in HBM for the dW kernel
+  uint16_t* pbuf;          // [Tpad][p_ld] bf16, row = compact row, column = vocabulary id (nullptr: off)
+  int64_t p_ld;            // nvz * NZ
+  float* mhist;            // [nvz][Tpad] reference of each row at each step
+  int64_t Tpad;            // ceil(T / 128) * 128
+  float* dzy_c;            // [rows] dZ at the target column, g (1 - p_y)
   // scratch
   uint16_t* dz_scratch;    // [clusters * C * kSlotsPerCta * 128][NZ] bf16 (P or dZ tiles)
   float* alpha;            // [clusters * C * kSlotsPerCta][128] per-row O rescale factors (kModeFwdDH)
@@ -262,7 +268,11 @@ __device__ __forceinline__ void lm_tma_role(LmShared& sh, const LmArgs& a, const
     if (kMode != kModeFwd) {
       // slice tiles of this CTA do not depend on the published tile: they are requested first,
       // the tile's chunks once the producer has published it
-      const int dz_row = static_cast<int>((x.cl * x.nslot + p.slot) * 128);
+      // the published tile: a scratch slot, or its place in the P store
+      const bool stored = (kMode == kModeFwdDH) && a.pbuf != nullptr;
+      const int dz_x0 = stored ? p.j * kNZ : 0;
+      const int dz_row = stored ? (static_cast<int>(x.cl) + p.u_idx * static_cast<int>(x.ncl)) * 128
+                                : static_cast<int>((x.cl * x.nslot + p.slot) * 128);
       bool dz_ok = false;
 #pragma unroll 1
       for (int kc = 0; kc < nkc; ++kc) {
@@ -277,7 +287,7 @@ __device__ __forceinline__ void lm_tma_role(LmShared& sh, const LmArgs& a, const
           if (!lm_wait<true>(sh, a, x.C, &sh.dz_ready[p.slot], p.round & 1u)) { ok = false; break; }
           dz_ok = true;
         }
-        tma_load_2d(dst, m.dz, &sh.full[stage], kc * 64, dz_row);
+        tma_load_2d(dst, m.dz, &sh.full[stage], dz_x0 + kc * 64, dz_row);
         ring_advance(stage, phase, nst);
       }
       if (!ok) break;
@@ -551,7 +561,13 @@ __device__ __forceinline__ void lm_fwd_epilogue_role(LmShared& sh, const LmArgs&
         if (p.round > 0) {
           if (!ep_wait<true>(sh, a, x.C, &sh.dz_free[p.slot], (p.round - 1) & 1u)) break;
         }
-        dzrow = a.dz_scratch + (static_cast<int64_t>(x.cl * x.nslot + p.slot) * 128 + row) * kNZ;
+        const int64_t urow = static_cast<int64_t>(static_cast<int>(x.cl) + p.u_idx * static_cast<int>(x.ncl)) * 128 + row;
+        if (a.pbuf != nullptr) {
+          dzrow = a.pbuf + urow * a.p_ld + p.j * kNZ;
+          a.mhist[static_cast<int64_t>(p.j) * a.Tpad + urow] = mnew;
+        } else {
+          dzrow = a.dz_scratch + (static_cast<int64_t>(x.cl * x.nslot + p.slot) * 128 + row) * kNZ;
+        }
       }
       // pass 2: P = e^{z - m} without the target column, the partial sum, the target logit
 #pragma unroll 1
@@ -643,6 +659,7 @@ __device__ __forceinline__ void lm_fwd_epilogue_role(LmShared& sh, const LmArgs&
             a.g_c[t] = tlv;
             a.tl_c[t] = tlv;
             a.d3_c[t] = d3;
+            if (a.dzy_c) a.dzy_c[t] = tlv * (s_ex / s);
           }
         }
         // dH_t = (g / s) (s' W_y - O') on this CTA's columns; O', s' and s share the reference m*

@@ -66,7 +66,7 @@ typedef enum {
   BI_OK = 0,
   BI_ERR_INVALID_ARG = 1,       /* NULL pointer, negative size, misaligned pointer */
   BI_ERR_UNSUPPORTED_SHAPE = 2, /* H not supported (see above) */
-  BI_ERR_WORKSPACE = 3,         /* ws == NULL or ws_bytes < bi_workspace_bytes(...) */
+  BI_ERR_WORKSPACE = 3,         /* ws == NULL or ws_bytes < bi_workspace_bytes_min(...) */
   BI_ERR_CUDA = 4,              /* a CUDA runtime call or launch failed */
   BI_ERR_TIMEOUT = 5,           /* device: a bounded wait ran out */
   BI_ERR_BAD_TARGET = 6,        /* device: a target id outside [0, V) */
@@ -85,11 +85,21 @@ typedef struct {
   int64_t n_nonfinite;
 } bi_d3;
 
-/* Size in bytes of the scratch workspace that every entry point needs for these sizes
- * (R = number of responses; pass 0 for bi_logprob_fwd / bi_d3_stats).  Deterministic and
- * free of side effects; the caller allocates the workspace (256-byte aligned) and may reuse it
- * across calls on the same stream. */
+/* Size in bytes of the scratch workspace for these sizes (R = number of responses; pass 0 for
+ * bi_logprob_fwd / bi_d3_stats).  Deterministic and free of side effects; the caller allocates
+ * the workspace (256-byte aligned) and may reuse it across calls on the same stream.
+ * For bi_is_loss_fwd_bwd this is the workspace of the fastest path: besides O(T) per-row arrays
+ * it holds every bf16 probability tile of the forward (about 2 T (V + 384) bytes, 23 GB for
+ * T = 76,000 rows of a 151,936-token vocabulary), so that dW is one GEMM over stored tiles instead
+ * of a second pass over the logits. */
 BI_API size_t bi_workspace_bytes(int64_t T, int32_t H, int32_t V, int32_t R);
+
+/* Smallest workspace bi_is_loss_fwd_bwd accepts (O(T H) bytes).  Any ws_bytes from this size up
+ * to just below bi_workspace_bytes(...) selects the low-memory path, whose dW kernel recomputes
+ * the logits (about a third more tensor work per step).  Both paths produce the same bits for
+ * every output except grad_w, where they differ by rounding only.  For R = 0 it equals
+ * bi_workspace_bytes. */
+BI_API size_t bi_workspace_bytes_min(int64_t T, int32_t H, int32_t V, int32_t R);
 
 /* Token log-probabilities log pi(y_t | h_t) under the LM head W (definition above).
  *   hidden   [T, H] bf16      rows to score (row-major, 16-byte aligned)

@@ -58,6 +58,11 @@ def test_workspace_bytes(lib):
     assert lib.bi_workspace_bytes(-1, 128, 512, 0) == 0
     # the compact copy of the hidden states is part of the loss workspace
     assert d - c >= 1000 * 1536 * 2
+    # the full loss workspace stores the bf16 probability tiles (T x (V + 256) rounded to 128 rows);
+    # the minimum one does not, and the logprob-only one is its own minimum
+    lo = lib.bi_workspace_bytes_min(2000, 1536, 151936, 64)
+    assert d - lo >= 2048 * 151936 * 2 and lo < 2000 * 1536 * 2 * 4 + (64 << 20)
+    assert lib.bi_workspace_bytes_min(2000, 1536, 151936, 0) == b
 
 
 FAKE = 1 << 20  # aligned non-null address; never dereferenced on the paths below
@@ -102,7 +107,9 @@ def test_is_loss_argument_checks(lib):
     assert call(loss=None) == 1
     assert call(grad_w=FAKE + 4) == 1  # misaligned
     assert call(H=704) == 2            # 11 * 64: no split into <= 384-column multiples of 64 with C <= 8
-    assert call(ws_bytes=ws_bytes - 1) == 3
+    ws_min = lib.bi_workspace_bytes_min(T, H, V, R)
+    assert 0 < ws_min < ws_bytes
+    assert call(ws_bytes=ws_min - 1) == 3
 
 
 def test_d3_argument_checks(lib):

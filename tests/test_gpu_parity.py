@@ -75,7 +75,8 @@ def test_bad_target_sets_status(cuda_device):
     assert np.isnan(f64(lp)[3]) and np.isfinite(np.delete(f64(lp), 3)).all()
 
 
-def _loss_case(batch, cuda_device, rollout_lp=None, resp_normalizer=0.0, check_dw=True, tight=1e-4):
+def _loss_case(batch, cuda_device, rollout_lp=None, resp_normalizer=0.0, check_dw=True, tight=1e-4,
+               minimal_ws=False):
     b = batch
     if rollout_lp is None:
         rollout_lp, _ = orc.token_logprob(b.hidden, b.w_roll, b.targets)
@@ -85,8 +86,9 @@ def _loss_case(batch, cuda_device, rollout_lp=None, resp_normalizer=0.0, check_d
     ref = orc.is_loss_fwd_bwd(b.hidden, b.w, b.targets, mu64, b.rewards, b.resp_offsets, b.group_offsets,
                               b.prompt_lens, resp_normalizer, want_grad_w=check_dw)
     d = b.to(cuda_device)
+    ws = bi.make_workspace(d.n_rows, d.hidden.shape[1], d.w.shape[0], d.R, cuda_device, minimal=minimal_ws)
     out = bi.is_loss_fwd_bwd(d.hidden, d.w, d.targets, mu.to(cuda_device), d.rewards, d.resp_offsets,
-                             d.group_offsets, d.prompt_lens, resp_normalizer)
+                             d.group_offsets, d.prompt_lens, resp_normalizer, ws=ws)
     torch.cuda.synchronize()
     bi.check_status(out.status)
     assert_close("loss", f64(out.loss), [ref["loss"]], LOSS_TOL, LOSS_TOL)
@@ -134,6 +136,19 @@ def test_loss_cluster_split_h2560(cuda_device):
     """H = 2560: 320 columns per CTA, two MMA column chunks of 192 and 128."""
     spec = spec_for("tiny", H=2560, V=2000, groups=2, per_group=2, len_lo=40, len_hi=150, prompt_len=16)
     _loss_case(make_batch(spec), cuda_device)
+
+
+@pytest.mark.parametrize("name,kw", [("tiny", dict(prompt_len=3)), ("h2560", dict(H=2560, V=2000, len_lo=40, len_hi=150)),
+                                     ("odd", dict(V=549, H=192, len_lo=1, len_hi=70))])
+def test_loss_low_memory_path(name, kw, cuda_device):
+    """The minimum workspace (dW recomputes the logits) against the oracle, and against the full
+    workspace (dW from the stored probability tiles): identical bits except grad_w."""
+    b = make_batch(spec_for("tiny", **kw))
+    lo, ref = _loss_case(b, cuda_device, minimal_ws=True)
+    hi, _ = _loss_case(b, cuda_device, minimal_ws=False)
+    for f in ("loss", "logprob", "is_weight", "token_loss", "grad_hidden", "d3_raw"):
+        assert torch.equal(getattr(lo, f), getattr(hi, f)), f
+    assert not torch.equal(lo.grad_w, hi.grad_w) or b.n_rows == 0  # two different dW kernels ran
 
 
 @pytest.mark.parametrize("H,V", [(256, 3001), (1536, 8000)])
