@@ -182,6 +182,21 @@ bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int 
            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The same bf16 row-major [rows][cols] tensor seen as [cols / 64][rows][64]: one load brings
+// `box_blocks` consecutive 64-column blocks of `box_rows` rows, each block a 128B-swizzled
+// [box_rows][64] tile of its own (the MN-major operand layout), in a single TMA instruction.
+bool make_map_blocks(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows, int box_blocks) {
+  EncodeTiledFn f = encode_fn();
+  if (!f || cols % 64 != 0) return false;
+  const cuuint64_t dims[3] = {64u, static_cast<cuuint64_t>(rows > 0 ? rows : 1), static_cast<cuuint64_t>(cols / 64)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(cols) * 2, 128u};
+  const cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(box_rows), static_cast<cuuint32_t>(box_blocks)};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // ---------------------------------------------------------------------------------------------
 // per-device set-up (kernel attributes, SM count, cluster occupancy), done once per device
 // ---------------------------------------------------------------------------------------------
@@ -567,7 +582,7 @@ bi_status bi_is_loss_fwd_bwd(const uint16_t* hidden, const uint16_t* w_lm, const
   }
   if (cudaGetLastError() != cudaSuccess) return BI_ERR_CUDA;
 
-  CUtensorMap tm_h128, tm_hz, tm_h64, tm_w128, tm_wz, tm_w64, tm_dz, tm_p64;
+  CUtensorMap tm_h128, tm_hz, tm_h64, tm_w128, tm_wz, tm_w64, tm_dz, tm_p64, tm_hblk;
   const int64_t trows = T > 0 ? T : 1;
   const int nvz = (V + pl.NZ - 1) / pl.NZ;
   const int64_t p_ld = static_cast<int64_t>(nvz) * pl.NZ;  // <= L.pcols
@@ -576,7 +591,10 @@ bi_status bi_is_loss_fwd_bwd(const uint16_t* hidden, const uint16_t* w_lm, const
       !make_map(&tm_h64, hsrc, trows, H, 64) || !make_map(&tm_w128, w_lm, V, H, 128) ||
       !make_map(&tm_wz, w_lm, V, H, pl.NZ) || !make_map(&tm_w64, w_lm, V, H, 64))
     return BI_ERR_CUDA;
-  if (store ? !(make_map(&tm_dz, w8 + L.pbuf, L.tpad, p_ld, 128) && make_map(&tm_p64, w8 + L.pbuf, L.tpad, p_ld, 64))
+  const int dw_hs = dw_split(H);
+  if (store ? !(make_map(&tm_dz, w8 + L.pbuf, L.tpad, p_ld, 128) &&
+                make_map_blocks(&tm_p64, w8 + L.pbuf, L.tpad, p_ld, 64, 4) &&
+                make_map_blocks(&tm_hblk, hsrc, trows, H, 64, dw_hs / 64))
             : !make_map(&tm_dz, w8 + L.dz, static_cast<int64_t>(kDzSlotsMax) * 128, pl.NZ, 128))
     return BI_ERR_CUDA;
   bi::LmArgs a{};
@@ -625,7 +643,7 @@ bi_status bi_is_loss_fwd_bwd(const uint16_t* hidden, const uint16_t* w_lm, const
     da.Tpad = L.tpad;
     da.d_rows = d_rows;
     da.nv128 = a.nv128;
-    da.nitems = a.nv128 * da.nsl;
+    da.nitems = ((a.nv128 + 1) / 2) * da.nsl;
     da.lse_c = F(L.lse_c);
     da.g_c = F(L.g_c);
     da.y_c = I(L.y_c);
@@ -660,7 +678,7 @@ bi_status bi_is_loss_fwd_bwd(const uint16_t* hidden, const uint16_t* w_lm, const
   if (st == BI_OK && store) {
     st = BI_ERR_UNSUPPORTED_SHAPE;
 #define BI_LAUNCH_DW(HS_) \
-    if (da.Hs == HS_) st = launch_dw<HS_>(tm_p64, tm_h64, da, di, s);
+    if (da.Hs == HS_) st = launch_dw<HS_>(tm_p64, tm_hblk, da, di, s);
     BI_DW_CONFIGS(BI_LAUNCH_DW)
 #undef BI_LAUNCH_DW
   }

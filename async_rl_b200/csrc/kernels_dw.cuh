@@ -10,14 +10,17 @@
 // ("Zero Mismatch, Simple Async RL", section "Alignment permits a simpler learning path": the
 // gradient of the unclipped token-level IS loss through the LM head.)
 //
-// Work item = (128-row vocabulary tile u, Hs-column slice q of H); a CTA owns one item at a time
-// (grid = one CTA per SM, items strided by the grid) and sweeps the tokens in chunks of 64:
-//   TMA warp     P^T chunk [128 v x 64 t] (two MN-major boxes) + H chunk [64 t x Hs] -> stage
+// Work item = (two 128-row vocabulary tiles 2w, 2w+1, Hs-column slice q of H); a CTA owns one
+// item at a time (grid = one CTA per SM, items strided by the grid) and sweeps the tokens in
+// chunks of 64:
+//   TMA warp     P^T chunk [256 v x 64 t] (four MN-major 64-column blocks) + H chunk [64 t x Hs]
 //   transform    8 warps rewrite the P chunk in place into bf16 dZ^T (per-token scale, target)
-//   MMA lane     O[128 x Hs] += dZ^T chunk * H chunk (A and B MN-major), O double-buffered in TMEM
-//   drain        4 warps write the finished O of an item to dW while the next item accumulates
-// The six slices of one vocabulary tile run on neighbouring CTAs at the same time, so a P chunk
-// is read from HBM once and from L2 by the other five.
+//   MMA lane     O_0, O_1 [128 x Hs] += dZ^T halves * H chunk (A and B MN-major)
+//   drain        4 warps write the finished O_0, O_1 of an item to dW
+// Shared-memory delivery, not the tensor cores, bounds this kernel (a stage of two 128-row
+// tiles and one H chunk carries 8.4 MFLOP per 66 KB, a third fewer bytes per flop than one
+// tile); the slices of one vocabulary pair run on neighbouring CTAs at the same time, so a P
+// chunk is read from HBM once and from L2 by the others.
 #pragma once
 
 #include "kernels_lm.cuh"
@@ -27,8 +30,8 @@ namespace bi {
 constexpr int kDwThreads = 448;  // TMA warp, MMA warp, 8 transform warps, 4 drain warps
 constexpr int kDwXfThreads = 256;
 constexpr int kDwAUnit = 8192;   // [64 tokens][64 vocabulary] bf16, 128B-swizzled
-constexpr int kDwABytes = 2 * kDwAUnit;
-constexpr int kDwTokBytes = 6 * 256;  // per chunk: lse, g, y, dZ_y, m (first half), m (second half) x 64 tokens
+constexpr int kDwABytes = 4 * kDwAUnit;   // two 128-row vocabulary tiles
+constexpr int kDwTokBytes = 8 * 256;      // per chunk: lse, g, y, dZ_y, m of each 64-column block x 64 tokens
 
 #define BI_DW_CONFIGS(X) X(64) X(128) X(192) X(256)
 
@@ -42,7 +45,7 @@ struct DwArgs {
                             // every per-row array below holds Tpad entries
   const int64_t* d_rows;    // number of scored rows on the device
   int32_t nv128;            // ceil(V / 128)
-  int32_t nitems;           // nv128 * nsl
+  int32_t nitems;           // ceil(nv128 / 2) * nsl
   const float* lse_c;       // [rows]
   const float* g_c;         // [rows]
   const int32_t* y_c;       // [rows]
@@ -57,7 +60,7 @@ struct DwShared {
   uint64_t full[kMaxStages];    // TMA -> transform (transaction bytes)
   uint64_t tready[kMaxStages];  // transform (256 threads) -> MMA
   uint64_t empty[kMaxStages];   // MMA commit -> TMA
-  uint64_t o_full[2], o_empty[2];
+  uint64_t o_full, o_empty;
   uint64_t mma_done;
   uint32_t tmem_base;
   volatile uint32_t abort_flag;
@@ -73,6 +76,7 @@ struct DwTile {
   static constexpr int nstages = fit < kMaxStages ? fit : kMaxStages;
   static constexpr int smem = nstages * stage_bytes + kDwSharedBytes;
   static_assert(kHS % 64 == 0 && kHS <= 256, "two accumulators of Hs columns fill at most 512 TMEM columns");
+  static_assert(kDwABytes % 1024 == 0 && (kHS * 128) % 1024 == 0, "operand blocks stay 1024-byte aligned");
   static_assert(nstages >= 2, "pipeline needs at least two stages");
 };
 
@@ -89,6 +93,8 @@ __device__ __forceinline__ void fence_proxy_async_shared() {
 template <int kHS>
 __global__ void __launch_bounds__(kDwThreads, 1)
     k_dw_stream(const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_h, DwArgs a) {
+  // tm_p: the P store as [p_ld / 64][Tpad][64], box {64, 64, 4}; tm_h: the (compact) hidden
+  // states as [H / 64][rows][64], box {64, 64, Hs / 64}
   extern __shared__ __align__(1024) uint8_t dsmem[];
   constexpr int nst = DwTile<kHS>::nstages;
   constexpr uint32_t sbytes = DwTile<kHS>::stage_bytes;
@@ -102,10 +108,8 @@ __global__ void __launch_bounds__(kDwThreads, 1)
       mbar_init(&sh.tready[i], kDwXfThreads);
       mbar_init(&sh.empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&sh.o_full[i], 1);
-      mbar_init(&sh.o_empty[i], 128);
-    }
+    mbar_init(&sh.o_full, 1);
+    mbar_init(&sh.o_empty, 128);
     mbar_init(&sh.mma_done, 1);
     sh.abort_flag = 0u;
     fence_mbar_init_cluster();
@@ -133,20 +137,16 @@ __global__ void __launch_bounds__(kDwThreads, 1)
       uint32_t stage = 0, phase = 0;
       bool ok = true;
       for (int it = blockIdx.x; ok && it < nitems; it += gridDim.x) {
-        const int u = it / a.nsl, q = it - (it / a.nsl) * a.nsl;
-        // forward steps of the two 64-column halves (a half past V reads a valid, unused row)
-        const int jm0 = min((u * 128) / a.NZf, a.nvz - 1);
-        const int jm1 = min((u * 128 + 64) / a.NZf, a.nvz - 1);
+        const int w = it / a.nsl, q = it - (it / a.nsl) * a.nsl;
 #pragma unroll 1
         for (int k = 0; k < nk; ++k) {
           if (!dw_wait(sh, a, &sh.empty[stage], phase ^ 1u)) { ok = false; break; }
           mbar_arrive_expect_tx(&sh.full[stage], DwTile<kHS>::tok_off + kDwTokBytes);
           const uint32_t dst = ring + stage * sbytes;
-          tma_load_2d(dst, &tm_p, &sh.full[stage], u * 128, k * 64);
-          tma_load_2d(dst + kDwAUnit, &tm_p, &sh.full[stage], u * 128 + 64, k * 64);
-#pragma unroll
-          for (int m = 0; m < kHS / 64; ++m)
-            tma_load_2d(dst + kDwABytes + m * kDwAUnit, &tm_h, &sh.full[stage], q * kHS + m * 64, k * 64);
+          // the four 64-column blocks of the P chunk, then the Hs / 64 column blocks of the H
+          // chunk, one instruction each (block-major tensor maps)
+          tma_load_3d(dst, &tm_p, &sh.full[stage], 0, k * 64, w * 4);
+          tma_load_3d(dst + kDwABytes, &tm_h, &sh.full[stage], 0, k * 64, q * (kHS / 64));
           // the chunk's per-token values (64 x 4 bytes each; the arrays hold Tpad >= 64 nk entries)
           const uint32_t tok = dst + DwTile<kHS>::tok_off;
           const int64_t t0 = static_cast<int64_t>(k) * 64;
@@ -154,8 +154,11 @@ __global__ void __launch_bounds__(kDwThreads, 1)
           bulk_load(tok + 256, a.g_c + t0, 256, &sh.full[stage]);
           bulk_load(tok + 512, a.y_c + t0, 256, &sh.full[stage]);
           bulk_load(tok + 768, a.dzy_c + t0, 256, &sh.full[stage]);
-          bulk_load(tok + 1024, a.mhist + static_cast<int64_t>(jm0) * a.Tpad + t0, 256, &sh.full[stage]);
-          bulk_load(tok + 1280, a.mhist + static_cast<int64_t>(jm1) * a.Tpad + t0, 256, &sh.full[stage]);
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {  // forward step of each block (a block past V reads a valid, unused row)
+            const int jm = min((w * 256 + h * 64) / a.NZf, a.nvz - 1);
+            bulk_load(tok + 1024 + h * 256, a.mhist + static_cast<int64_t>(jm) * a.Tpad + t0, 256, &sh.full[stage]);
+          }
           ring_advance(stage, phase, nst);
         }
       }
@@ -177,23 +180,24 @@ __global__ void __launch_bounds__(kDwThreads, 1)
       uint32_t stage = 0, phase = 0, n_it = 0;
       bool ok = true;
       for (int it = blockIdx.x; ok && it < nitems; it += gridDim.x, ++n_it) {
-        const uint32_t b = n_it & 1u;
-        if (!dw_wait(sh, a, &sh.o_empty[b], ((n_it >> 1) & 1u) ^ 1u)) break;
+        if (!dw_wait(sh, a, &sh.o_empty, (n_it & 1u) ^ 1u)) break;
         tc_fence_after();
-        const uint32_t acc = tmem + b * kHS;
 #pragma unroll 1
         for (int k = 0; k < nk; ++k) {
           if (!dw_wait(sh, a, &sh.tready[stage], phase)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)  // 16 tokens = 16 MN-major rows of 128 B = 2 KB
-            umma_bf16(acc, da0 + stage * sb + kk * (2048 >> 4), db0 + stage * sb + kk * (2048 >> 4), idesc,
-                      (k > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < 4; ++kk) {  // 16 tokens = 16 MN-major rows of 128 B = 2 KB
+            const uint32_t accum = (k > 0 || kk > 0) ? 1u : 0u;
+            const uint64_t db = db0 + stage * sb + kk * (2048 >> 4);
+            umma_bf16(tmem, da0 + stage * sb + kk * (2048 >> 4), db, idesc, accum);
+            umma_bf16(tmem + kHS, da0 + stage * sb + ((2 * kDwAUnit) >> 4) + kk * (2048 >> 4), db, idesc, accum);
+          }
           umma_commit(&sh.empty[stage]);
           ring_advance(stage, phase, nst);
         }
         if (!ok) break;
-        umma_commit(&sh.o_full[b]);
+        umma_commit(&sh.o_full);
       }
       umma_commit(&sh.mma_done);
       const uint64_t t0 = globaltimer_ns();
@@ -209,7 +213,7 @@ __global__ void __launch_bounds__(kDwThreads, 1)
     uint32_t stage = 0, phase = 0;
     bool ok = true;
     for (int it = blockIdx.x; ok && nk > 0 && it < nitems; it += gridDim.x) {
-      const int u = it / a.nsl;
+      const int w = it / a.nsl;
 #pragma unroll 1
       for (int k = 0; k < nk; ++k) {
         if (!dw_wait(sh, a, &sh.full[stage], phase)) { ok = false; break; }
@@ -217,7 +221,7 @@ __global__ void __launch_bounds__(kDwThreads, 1)
         const float* tok = reinterpret_cast<const float*>(dsmem + stage * sbytes + DwTile<kHS>::tok_off);
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
-          // 16-byte chunk c = tt + 256 i of each 8 KB half: token row tl, logical chunk cq
+          // 16-byte chunk c = tt + 256 i of each 8 KB block: token row tl, logical chunk cq
           const int c = tt + 256 * i;
           const int tl = c >> 3, cq = c & 7;
           const int64_t t = static_cast<int64_t>(k) * 64 + tl;
@@ -226,31 +230,31 @@ __global__ void __launch_bounds__(kDwThreads, 1)
           const int32_t yy = tv ? reinterpret_cast<const int32_t*>(tok)[128 + tl] : -1;
           const uint32_t off = static_cast<uint32_t>(tl * 128 + ((cq ^ (tl & 7)) << 4));
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            // a half at or past V has no forward step (and P there is zero-filled); the two halves
-            // each lie inside one forward step (NZf is a multiple of 64)
-            const bool hv = tv && (u * 128 + h * 64 < a.V);
+          for (int h = 0; h < 4; ++h) {
+            // a block at or past V has no forward step (and P there is zero-filled); each block
+            // lies inside one forward step (NZf is a multiple of 64)
+            const bool hv = tv && (w * 256 + h * 64 < a.V);
             const float sig = hv ? -g * ex2_approx((tok[256 + 64 * h + tl] - lse) * kLog2e) : 0.f;
             const uint32_t sig2 = pack_bf16x2(sig, sig);
             const uint32_t addr = base + h * kDwAUnit + off;
-            uint32_t w[4];
+            uint32_t pv[4];
             asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
-                         : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                         : "=r"(pv[0]), "=r"(pv[1]), "=r"(pv[2]), "=r"(pv[3])
                          : "r"(addr));
 #pragma unroll
-            for (int e = 0; e < 4; ++e) asm("mul.rn.bf16x2 %0, %0, %1;" : "+r"(w[e]) : "r"(sig2));
+            for (int e = 0; e < 4; ++e) asm("mul.rn.bf16x2 %0, %0, %1;" : "+r"(pv[e]) : "r"(sig2));
             // the target column (stored as 0) takes g (1 - p_y); rare, so a branch
-            const uint32_t dv = static_cast<uint32_t>(yy - (u * 128 + h * 64 + cq * 8));
+            const uint32_t dv = static_cast<uint32_t>(yy - (w * 256 + h * 64 + cq * 8));
             if (dv < 8u) {
               const uint32_t bz = pack_bf16x2(dzy, dzy);
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
                 const uint32_t m = ((dv == 2u * e) ? 0x0000ffffu : 0u) | ((dv == 2u * e + 1u) ? 0xffff0000u : 0u);
-                w[e] = (w[e] & ~m) | (bz & m);
+                pv[e] = (pv[e] & ~m) | (bz & m);
               }
             }
-            asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(w[0]), "r"(w[1]), "r"(w[2]),
-                         "r"(w[3])
+            asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(pv[0]), "r"(pv[1]), "r"(pv[2]),
+                         "r"(pv[3])
                          : "memory");
           }
         }
@@ -260,37 +264,43 @@ __global__ void __launch_bounds__(kDwThreads, 1)
       }
     }
   } else {
-    // ---------------- drain: O -> dW rows ----------------
+    // ---------------- drain: O_0, O_1 -> dW rows ----------------
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t tl = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     uint32_t n_it = 0;
     for (int it = blockIdx.x; it < nitems; it += gridDim.x, ++n_it) {
-      const int u = it / a.nsl, q = it - (it / a.nsl) * a.nsl;
-      const int64_t v = static_cast<int64_t>(u) * 128 + row;
-      float* dst = (v < a.V) ? a.grad_w + v * a.H + q * kHS : nullptr;
-      const uint32_t b = n_it & 1u;
-      if (nk == 0) {  // no scored rows: the gradient is zero
-        if (dst)
-          for (int c = 0; c < kHS / 4; ++c) reinterpret_cast<float4*>(dst)[c] = make_float4(0.f, 0.f, 0.f, 0.f);
-        continue;
+      const int w = it / a.nsl, q = it - (it / a.nsl) * a.nsl;
+      if (nk > 0) {
+        const WaitCtl wc{&sh.abort_flag, a.status, a.limit_ns};
+        if (!__all_sync(0xffffffffu, mbar_wait<false>(&sh.o_full, n_it & 1u, wc))) break;
+        tc_fence_after();
       }
-      const WaitCtl wc{&sh.abort_flag, a.status, a.limit_ns};
-      if (!__all_sync(0xffffffffu, mbar_wait<false>(&sh.o_full[b], (n_it >> 1) & 1u, wc))) break;
-      tc_fence_after();
 #pragma unroll 1
-      for (int c = 0; c < kHS / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tl + b * kHS + c * 32, r);
-        tmem_ld_wait();
-        if (dst) {
-          uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+      for (int half = 0; half < 2; ++half) {
+        const int64_t v = static_cast<int64_t>(w) * 256 + half * 128 + row;
+        float* dst = (v < a.V) ? a.grad_w + v * a.H + q * kHS : nullptr;
+        if (nk == 0) {  // no scored rows: the gradient is zero
+          if (dst)
+            for (int c = 0; c < kHS / 4; ++c) reinterpret_cast<float4*>(dst)[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+          continue;
+        }
+#pragma unroll 1
+        for (int c = 0; c < kHS / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tl + half * kHS + c * 32, r);
+          tmem_ld_wait();
+          if (dst) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) d4[e] = make_uint4(r[4 * e], r[4 * e + 1], r[4 * e + 2], r[4 * e + 3]);
+            for (int e = 0; e < 8; ++e) d4[e] = make_uint4(r[4 * e], r[4 * e + 1], r[4 * e + 2], r[4 * e + 3]);
+          }
         }
       }
-      tc_fence_before();
-      mbar_arrive(&sh.o_empty[b]);
+      if (nk > 0) {
+        tc_fence_before();
+        mbar_arrive(&sh.o_empty);
+      }
     }
   }
 
