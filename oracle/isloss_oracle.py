@@ -35,6 +35,21 @@ Readings where the pages are silent (each one is listed in the design notes):
   zero gradient row.
 * D3 statistics are over every scored token of the call: mean, max, count, and
   the number of non-finite terms (mean and max are non-finite when any term is).
+* rollout-to-learner KL (the pages plot a "sampled estimate" without a formula):
+  the plain sampled estimators of KL(mu || pi) from tokens drawn from mu, with
+  delta = log pi - log mu: k1 = -delta, k2 = delta^2 / 2, k3 = e^delta - 1 - delta
+  (the D3 term); means over the scored tokens.  E_mu[k1] = E_mu[k3] = KL(mu||pi).
+* comparison variants (the baselines the pages argue against; no formula given):
+  - "ppo_clip": the clipped surrogate per token,
+      l_t = -min(r A_i, clip(r, 1 - eps_low, 1 + eps_high) A_i) / (R* n_i),
+    r = w_t, differentiated through r only (the clip bound is a constant);
+  - "seq_gate": response i is rejected when its mean token log-ratio
+    rho_i = (1/n_i) sum_t delta_t has |rho_i| > gate (or is not finite); a
+    rejected response contributes no loss and no gradient and still counts in
+    R*.  The rejection rate is n_rejected / (responses with a scored token).
+* D3 peak/median across updates: max over the per-update D3 means divided by
+  their median; KL drift: median over the last window of updates divided by
+  the median over the first window.
 """
 from __future__ import annotations
 
@@ -182,13 +197,59 @@ def response_coefficients(A, resp_offsets, prompt_lens, resp_normalizer: float =
 # Full step: loss, per-token terms, D3 and gradients
 # ---------------------------------------------------------------------------
 
+def token_terms(variant: str, w, delta, A_row, n_row, rstar: float, resp_of_row, mask, c_row,
+                eps_low: float = 0.2, eps_high: float = 0.2, gate: float = math.inf) -> dict:
+    """Per-token loss l_t and gradient coefficient g_t = dL/dlog pi_t of each loss variant.
+
+    unclipped: l_t = -w A / (R* n),  g_t = l_t                         ([ZM-path], [RZ-core])
+    ppo_clip:  l_t = -min(w A, clip(w) A) / (R* n); g_t = -w A / (R* n) where the first
+               argument is the minimum (ties included), else 0
+    seq_gate:  the unclipped terms, zeroed on every row of a rejected response
+    """
+    T = w.shape[0]
+    with np.errstate(invalid="ignore", over="ignore", divide="ignore"):
+        denom = rstar * n_row
+        if variant == "unclipped":
+            l = np.where(mask, -c_row * w, 0.0)
+            return {"token_loss": l, "g": l.copy(), "n_clipped": 0, "n_rejected": 0,
+                    "rejected": np.zeros(0, dtype=bool)}
+        if variant == "ppo_clip":
+            first = w * A_row
+            second = np.clip(w, 1.0 - eps_low, 1.0 + eps_high) * A_row
+            sur = np.minimum(first, second)
+            active = first <= second
+            l = np.where(mask, -sur / np.where(mask, denom, 1.0), 0.0)
+            g = np.where(mask & active, -first / np.where(mask, denom, 1.0), 0.0)
+            n_clipped = int(np.sum(mask & ~active & (A_row != 0)))
+            return {"token_loss": l, "g": g, "n_clipped": n_clipped, "n_rejected": 0,
+                    "rejected": np.zeros(0, dtype=bool)}
+        if variant == "seq_gate":
+            R = int(np.max(resp_of_row)) + 1 if T else 0
+            R = max(R, 0)
+            sums = np.zeros(R)
+            cnt = np.zeros(R)
+            for t in range(T):
+                if mask[t]:
+                    sums[resp_of_row[t]] += delta[t]
+                    cnt[resp_of_row[t]] += 1
+            rho = np.where(cnt > 0, sums / np.maximum(cnt, 1), 0.0)
+            rejected = (cnt > 0) & ~(np.abs(rho) <= gate)
+            keep_row = mask & ~rejected[resp_of_row] if T else mask
+            l = np.where(keep_row, -c_row * w, 0.0)
+            return {"token_loss": l, "g": l.copy(), "n_clipped": 0, "n_rejected": int(np.sum(rejected)),
+                    "rejected": rejected, "rho": rho}
+    raise ValueError(f"unknown loss variant {variant!r}")
+
+
 def is_loss_fwd_bwd(hidden, w, targets, rollout_logprob, rewards, resp_offsets, group_offsets,
                     prompt_lens=None, resp_normalizer: float = 0.0, want_grads: bool = True,
-                    want_grad_w: bool = True) -> dict:
+                    want_grad_w: bool = True, variant: str = "unclipped", eps_low: float = 0.2,
+                    eps_high: float = 0.2, gate: float = math.inf) -> dict:
     """Everything the fused learner step returns, in float64.
 
-    L   = -sum_i c_i sum_{t in i, scored} w_t,          c_i = A_i / (R* n_i)
-    g_t = dL/dz_{t,y_t}-coefficient = -c_i w_t  (0 on unscored rows)
+    L   = sum_t l_t over the scored tokens (l_t of the variant, see ``token_terms``;
+          unclipped: l_t = -c_i w_t, c_i = A_i / (R* n_i))
+    g_t = dL/dlog pi_t  (0 on unscored rows)
     dZ  = g_t (onehot(y_t) - p_t),  p_t = softmax(z_t)
     dH  = dZ W,   dW = dZ^T H
     """
@@ -216,17 +277,24 @@ def is_loss_fwd_bwd(hidden, w, targets, rollout_logprob, rewards, resp_offsets, 
     w_s, d_s = is_weight(lp_all, logmu[mask])
     wgt[mask] = w_s
     delta[mask] = d_s
+    rstar = float(resp_normalizer) if resp_normalizer > 0 else float(off.shape[0] - 1)
+    terms = token_terms(variant, wgt, delta, A[resp_of_row], n[resp_of_row].astype(np.float64), rstar,
+                        resp_of_row, mask, c_row, eps_low, eps_high, gate)
+    token_loss = terms["token_loss"]
     with np.errstate(invalid="ignore", over="ignore"):
-        token_loss = np.where(mask, -c_row * wgt, 0.0)
         loss = float(np.sum(token_loss))
     d3 = d3_stats(lp_all, logmu[mask])
+    kl = kl_estimators(lp_all, logmu[mask])
 
     out = {"loss": loss, "logprob": logprob, "lse": lse, "is_weight": wgt, "delta": delta,
-           "token_loss": token_loss, "d3": d3, "advantages": A, "n_scored": n, "coef": c,
-           "mask": mask}
+           "token_loss": token_loss, "d3": d3, "kl": kl, "advantages": A, "n_scored": n, "coef": c,
+           "mask": mask, "n_clipped": terms["n_clipped"], "n_rejected": terms["n_rejected"],
+           "rejected": terms["rejected"]}
+    if "rho" in terms:
+        out["rho"] = terms["rho"]
     if not want_grads:
         return out
-    g = token_loss.copy()  # g_t = -c_i w_t
+    g = terms["g"]
     dH = np.zeros_like(Hm)
     dW = np.zeros_like(Wm) if want_grad_w else None
     rows = np.nonzero(mask)[0]
@@ -275,11 +343,30 @@ def kl_estimators(learner_logprob, rollout_logprob, mask=None) -> dict:
             "k3": float(np.mean(d3_terms(delta)))}
 
 
+def d3_peak_median(d3_means) -> dict:
+    """Peak over median of per-update D3 means ([ZM-gap]: 1.50x aligned, 442.54x standard)."""
+    d = np.asarray(d3_means, dtype=np.float64)
+    if d.shape[0] == 0:
+        return {"peak": 0.0, "median": 0.0, "ratio": float("nan")}
+    med = float(np.median(d))
+    peak = float(np.max(d))
+    return {"peak": peak, "median": med, "ratio": peak / med if med != 0 else float("inf")}
+
+
+def kl_drift(values, window: int) -> float:
+    """Median over the last ``window`` updates divided by the median over the first ``window``
+    ([ZM-path] Fig. 1: median rollout-to-learner KL rises 83.33x with standard kernels)."""
+    v = np.asarray(values, dtype=np.float64)
+    if v.shape[0] < window or window <= 0:
+        raise ValueError("need at least one full window of updates")
+    return float(np.median(v[-window:]) / np.median(v[:window]))
+
+
 def loss_only(hidden, w, targets, rollout_logprob, rewards, resp_offsets, group_offsets,
-              prompt_lens=None, resp_normalizer: float = 0.0) -> float:
+              prompt_lens=None, resp_normalizer: float = 0.0, **variant) -> float:
     """The scalar loss (no gradients); used by finite-difference pins."""
     return is_loss_fwd_bwd(hidden, w, targets, rollout_logprob, rewards, resp_offsets,
-                           group_offsets, prompt_lens, resp_normalizer, want_grads=False)["loss"]
+                           group_offsets, prompt_lens, resp_normalizer, want_grads=False, **variant)["loss"]
 
 
 def minus_log_v(V: int) -> float:

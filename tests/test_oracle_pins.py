@@ -291,3 +291,152 @@ def test_synthetic_generator_is_seeded():
     assert a.hidden.dtype == torch.bfloat16 and a.targets.dtype == torch.int32
     h, w, y = random_inputs(5, 64, 100, seed=1)
     assert h.shape == (5, 64) and w.shape == (100, 64) and int(y.max()) < 100
+
+
+# ---------------------------------------------------------------------------
+# Comparison variants and diagnostics (the pages' baselines and stability statistics)
+# ---------------------------------------------------------------------------
+
+def _variant_case(seed=21, lag=0.35):
+    """Tiny step whose rollout log-probabilities carry enough noise that some weights leave
+    [0.8, 1.2] (clipping) and some responses have a large mean log-ratio (gating)."""
+    rng = np.random.default_rng(seed)
+    T, H, V = 14, 6, 9
+    h = rng.normal(size=(T, H))
+    w = rng.normal(size=(V, H)) * 0.7
+    y = rng.integers(0, V, size=T)
+    off = np.array([0, 3, 7, 10, 14])
+    goff = np.array([0, 2, 4])
+    r = np.array([1.0, 0.0, 0.0, 1.0])
+    mu = orc.token_logprob(h, w, y)[0] + rng.normal(size=T) * lag
+    pl = np.array([1, 0, 0, 1])
+    args = dict(targets=y, rollout_logprob=mu, rewards=r, resp_offsets=off, group_offsets=goff,
+                prompt_lens=pl, resp_normalizer=4.0)
+    return h, w, args
+
+
+def test_ppo_clip_hand_example():
+    """Two responses of two tokens, R* = 2, clip range [0.8, 1.2].  A = +1: w = 1.5 is clipped
+    (l = -1.2/4, g = 0), w = 0.9 is not (l = g = -0.9/4).  A = -1: w = 0.5 is clipped at 0.8
+    (l = +0.8/4, g = 0), w = 1.5 is not (min picks -1.5: l = g = +1.5/4).  L = 0.05."""
+    w = np.array([1.5, 0.9, 0.5, 1.5])
+    A_row = np.array([1.0, 1.0, -1.0, -1.0])
+    n_row = np.full(4, 2.0)
+    resp = np.array([0, 0, 1, 1])
+    mask = np.ones(4, dtype=bool)
+    c_row = A_row / (2.0 * n_row)
+    t = orc.token_terms("ppo_clip", w, np.log(w), A_row, n_row, 2.0, resp, mask, c_row, 0.2, 0.2)
+    assert np.allclose(t["token_loss"], [-0.3, -0.225, 0.2, 0.375], rtol=0, atol=1e-15)
+    assert np.allclose(t["g"], [0.0, -0.225, 0.0, 0.375], rtol=0, atol=1e-15)
+    assert t["n_clipped"] == 2
+    assert abs(float(np.sum(t["token_loss"])) - 0.05) < 1e-15
+
+
+def test_ppo_clip_wide_range_is_unclipped():
+    h, w, args = _variant_case()
+    ref = orc.is_loss_fwd_bwd(h, w, **args)
+    wide = orc.is_loss_fwd_bwd(h, w, variant="ppo_clip", eps_low=1.0, eps_high=1e9, **args)
+    assert abs(wide["loss"] - ref["loss"]) <= 1e-15 * max(1.0, abs(ref["loss"]))
+    assert np.allclose(wide["grad_hidden"], ref["grad_hidden"], rtol=1e-14, atol=1e-18)
+    assert np.allclose(wide["grad_w"], ref["grad_w"], rtol=1e-14, atol=1e-18)
+    assert wide["n_clipped"] == 0
+
+
+def test_ppo_clip_finite_differences():
+    """The clipped loss is piecewise smooth in log pi; away from the kinks its gradient is the
+    oracle's dH/dW (a wrong clip side or a gradient through the constant bound fails here)."""
+    h, w, args = _variant_case()
+    v = dict(variant="ppo_clip", eps_low=0.2, eps_high=0.2)
+    out = orc.is_loss_fwd_bwd(h, w, **args, **v)
+    wts = out["is_weight"][out["mask"]]
+    assert np.min(np.abs(np.concatenate([wts - 0.8, wts - 1.2]))) > 1e-3  # no token at a kink
+    assert 0 < out["n_clipped"] < int(out["mask"].sum())                    # both branches occur
+    rng = np.random.default_rng(5)
+    eps = 1e-6
+    for _ in range(24):
+        i, k = rng.integers(0, h.shape[0]), rng.integers(0, h.shape[1])
+        hp, hm = h.copy(), h.copy()
+        hp[i, k] += eps
+        hm[i, k] -= eps
+        fd = (orc.loss_only(hp, w, **args, **v) - orc.loss_only(hm, w, **args, **v)) / (2 * eps)
+        assert abs(fd - out["grad_hidden"][i, k]) <= 1e-6 * max(1e-3, abs(fd)) + 1e-10
+    for _ in range(24):
+        a, k = rng.integers(0, w.shape[0]), rng.integers(0, w.shape[1])
+        wp, wm = w.copy(), w.copy()
+        wp[a, k] += eps
+        wm[a, k] -= eps
+        fd = (orc.loss_only(h, wp, **args, **v) - orc.loss_only(h, wm, **args, **v)) / (2 * eps)
+        assert abs(fd - out["grad_w"][a, k]) <= 1e-6 * max(1e-3, abs(fd)) + 1e-10
+
+
+def test_seq_gate_hand_example_and_limits():
+    """rho = mean delta of a response: (0.1 + 0.5) / 2 = 0.3 is rejected at gate 0.2 and kept at
+    0.4; an infinite gate is the unclipped loss; a zero gate rejects every response whose rho is
+    not exactly 0."""
+    w = np.exp(np.array([0.1, 0.5, -0.05, 0.05]))
+    A_row = np.array([1.0, 1.0, -1.0, -1.0])
+    n_row = np.full(4, 2.0)
+    resp = np.array([0, 0, 1, 1])
+    mask = np.ones(4, dtype=bool)
+    c_row = A_row / (2.0 * n_row)
+    lo = orc.token_terms("seq_gate", w, np.log(w), A_row, n_row, 2.0, resp, mask, c_row, gate=0.2)
+    hi = orc.token_terms("seq_gate", w, np.log(w), A_row, n_row, 2.0, resp, mask, c_row, gate=0.4)
+    assert lo["n_rejected"] == 1 and list(lo["rejected"]) == [True, False]
+    assert np.all(lo["token_loss"][:2] == 0.0) and np.all(lo["g"][:2] == 0.0)
+    assert np.allclose(lo["token_loss"][2:], -c_row[2:] * w[2:], rtol=0, atol=0)
+    assert hi["n_rejected"] == 0 and np.allclose(hi["token_loss"], -c_row * w, rtol=0, atol=0)
+    h, wm, args = _variant_case()
+    ref = orc.is_loss_fwd_bwd(h, wm, **args)
+    inf = orc.is_loss_fwd_bwd(h, wm, variant="seq_gate", gate=math.inf, **args)
+    assert inf["loss"] == ref["loss"] and inf["n_rejected"] == 0
+    assert np.array_equal(inf["grad_hidden"], ref["grad_hidden"])
+    zero = orc.is_loss_fwd_bwd(h, wm, variant="seq_gate", gate=0.0, **args)
+    assert zero["loss"] == 0.0 and zero["n_rejected"] == 4
+    assert not np.any(zero["grad_hidden"]) and not np.any(zero["grad_w"])
+
+
+def test_seq_gate_drops_exactly_the_rejected_responses():
+    """Rows of rejected responses get dH = 0; the rows of kept responses are unchanged from the
+    unclipped step (the gate removes terms, it does not rescale the others)."""
+    h, w, args = _variant_case()
+    ref = orc.is_loss_fwd_bwd(h, w, **args)
+    gated = orc.is_loss_fwd_bwd(h, w, variant="seq_gate", gate=0.15, **args)
+    rho = gated["rho"]
+    assert 0 < gated["n_rejected"] < 4
+    off = args["resp_offsets"]
+    for i in range(4):
+        rows = slice(off[i], off[i + 1])
+        if gated["rejected"][i]:
+            assert abs(rho[i]) > 0.15 and not np.any(gated["grad_hidden"][rows])
+        else:
+            assert np.array_equal(gated["grad_hidden"][rows], ref["grad_hidden"][rows])
+
+
+def test_kl_estimators_unbiased_on_exact_expectation():
+    """With tokens drawn from mu in exact proportions (counts 1..7 of 28), the plain means of k1
+    and k3 equal KL(mu || pi) = sum mu log(mu / pi); k2 equals it to second order only."""
+    rng = np.random.default_rng(3)
+    counts = np.arange(1, 8)
+    mu = counts / counts.sum()
+    pi = rng.dirichlet(np.ones(7))
+    kl = float(np.sum(mu * np.log(mu / pi)))
+    logmu = np.repeat(np.log(mu), counts)
+    logpi = np.repeat(np.log(pi), counts)
+    est = orc.kl_estimators(logpi, logmu)
+    assert abs(est["k1"] - kl) < 1e-14 and abs(est["k3"] - kl) < 1e-14
+    near = np.exp(np.log(mu) + 1e-3 * rng.normal(size=7))
+    near /= near.sum()
+    kl_near = float(np.sum(mu * np.log(mu / near)))
+    est_near = orc.kl_estimators(np.repeat(np.log(near), counts), logmu)
+    assert abs(est_near["k2"] - kl_near) < 1e-3 * kl_near
+    const = orc.kl_estimators(np.full(5, 0.3), np.zeros(5))
+    assert abs(const["k1"] + 0.3) < 1e-15 and abs(const["k2"] - 0.045) < 1e-15
+    assert abs(const["k3"] - (math.expm1(0.3) - 0.3)) < 1e-15
+
+
+def test_d3_peak_median_and_kl_drift():
+    s = orc.d3_peak_median([1.0, 2.0, 3.0, 100.0])
+    assert s["peak"] == 100.0 and s["median"] == 2.5 and s["ratio"] == 40.0
+    assert orc.kl_drift([1.0, 1.0, 2.0, 2.0, 10.0, 30.0], 2) == 20.0
+    with pytest.raises(ValueError):
+        orc.kl_drift([1.0], 2)
