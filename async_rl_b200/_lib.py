@@ -19,6 +19,15 @@ STATUS_NAMES = {0: "BI_OK", 1: "BI_ERR_INVALID_ARG", 2: "BI_ERR_UNSUPPORTED_SHAP
 
 _lib = None
 
+
+class LossCfg(ctypes.Structure):
+    """bi_loss_cfg"""
+    _fields_ = [("variant", ctypes.c_int32), ("eps_low", ctypes.c_float), ("eps_high", ctypes.c_float),
+                ("gate", ctypes.c_float)]
+
+
+LOSS_VARIANTS = {"unclipped": 0, "ppo_clip": 1, "seq_gate": 2}
+
 _p = ctypes.c_void_p
 _i32 = ctypes.c_int32
 _i64 = ctypes.c_int64
@@ -43,7 +52,7 @@ def load() -> ctypes.CDLL:
     lib.bi_logprob_fwd.restype = ctypes.c_int
     lib.bi_logprob_fwd_noalloc.argtypes = [_p, _p, _p, _i64, _i32, _i32, _p, _p, _p, _p]
     lib.bi_logprob_fwd_noalloc.restype = ctypes.c_int
-    lib.bi_is_loss_fwd_bwd.argtypes = [_p, _p, _p, _p, _p, _p, _p, _p, _i32, _i32, _f64, _i64, _i32, _i32,
+    lib.bi_is_loss_fwd_bwd.argtypes = [_p, _p, _p, _p, _p, _p, _p, _p, _i32, _i32, _f64, _p, _i64, _i32, _i32,
                                        _p, _p, _p, _p, _p, _p, _p, _p, _p, _sz, _p]
     lib.bi_is_loss_fwd_bwd.restype = ctypes.c_int
     lib.bi_d3_stats.argtypes = [_p, _p, _p, _i64, _p, _p, _p, _sz, _p]

@@ -12,7 +12,7 @@ import torch
 
 from . import _lib
 
-D3_DTYPE_BYTES = 24  # bi_d3: float mean, float max, int64 count, int64 n_nonfinite
+D3_DTYPE_BYTES = 40  # bi_d3: f32 mean, f32 max, i64 count, i64 n_nonfinite, f32 k1, f32 k2, i32 n_clipped, i32 n_rejected
 
 
 class BiError(RuntimeError):
@@ -96,10 +96,7 @@ class LossOutputs:
     status: torch.Tensor       # [1] i32
 
     def d3(self) -> dict:
-        raw = self.d3_raw.cpu()
-        f = raw[:8].view(torch.float32)
-        i = raw[8:24].view(torch.int64)
-        return {"mean": float(f[0]), "max": float(f[1]), "count": int(i[0]), "n_nonfinite": int(i[1])}
+        return decode_d3(self.d3_raw)
 
     @staticmethod
     def allocate(T: int, H: int, V: int, device) -> "LossOutputs":
@@ -110,8 +107,13 @@ class LossOutputs:
 
 def is_loss_fwd_bwd(hidden, w, targets, rollout_logprob, rewards, resp_offsets, group_offsets,
                     prompt_lens=None, resp_normalizer: float = 0.0, ws: Optional[torch.Tensor] = None,
-                    out: Optional[LossOutputs] = None) -> LossOutputs:
-    """Fused forward + backward of the unclipped token-level IS REINFORCE loss (see the C header)."""
+                    out: Optional[LossOutputs] = None, variant: str = "unclipped", eps_low: float = 0.2,
+                    eps_high: float = 0.2, gate: float = float("inf")) -> LossOutputs:
+    """Fused forward + backward of the token-level IS REINFORCE loss (see the C header).
+
+    ``variant`` is "unclipped" (the method), or one of the comparison baselines "ppo_clip"
+    (clip range [1 - eps_low, 1 + eps_high]) and "seq_gate" (rejects responses whose mean token
+    log-ratio exceeds ``gate`` in absolute value)."""
     dev = hidden.device
     T, H = hidden.shape
     V = w.shape[0]
@@ -130,9 +132,13 @@ def is_loss_fwd_bwd(hidden, w, targets, rollout_logprob, rewards, resp_offsets, 
     if ws is None:
         ws = make_workspace(T, H, V, R, dev)
     o = out if out is not None else LossOutputs.allocate(T, H, V, dev)
+    if variant not in _lib.LOSS_VARIANTS:
+        raise ValueError(f"unknown loss variant {variant!r}")
+    cfg = _lib.LossCfg(_lib.LOSS_VARIANTS[variant], float(eps_low), float(eps_high), float(gate))
+    import ctypes
     code = lib.bi_is_loss_fwd_bwd(_ptr(hidden), _ptr(w), _ptr(targets), _ptr(rollout_logprob), _ptr(rewards),
                                   _ptr(resp_offsets), _ptr(group_offsets), _ptr(prompt_lens), R, G,
-                                  float(resp_normalizer), T, H, V, _ptr(o.loss), _ptr(o.logprob),
+                                  float(resp_normalizer), ctypes.addressof(cfg), T, H, V, _ptr(o.loss), _ptr(o.logprob),
                                   _ptr(o.is_weight), _ptr(o.token_loss), _ptr(o.d3_raw), _ptr(o.grad_hidden),
                                   _ptr(o.grad_w), _ptr(o.status), _ptr(ws), ws.numel(), _stream(dev))
     _raise_host(code, "bi_is_loss_fwd_bwd")
@@ -148,9 +154,8 @@ def d3_stats(learner_logprob, rollout_logprob, mask=None, ws=None):
     if mask is not None:
         _check_cuda(mask, "mask", torch.uint8, dev)
     lib = _lib.load()
-    nred = (max(T, 1) + 255) // 256
     if ws is None:
-        ws = torch.empty(max(256, nred * 48), dtype=torch.uint8, device=dev)
+        ws = make_workspace(T, 64, 1, 0, dev)  # the R = 0 layout covers the block partials
     raw = torch.empty(D3_DTYPE_BYTES, dtype=torch.uint8, device=dev)
     st = torch.empty(1, dtype=torch.int32, device=dev)
     code = lib.bi_d3_stats(_ptr(learner_logprob), _ptr(rollout_logprob), _ptr(mask), T, _ptr(raw), _ptr(st),
@@ -160,10 +165,14 @@ def d3_stats(learner_logprob, rollout_logprob, mask=None, ws=None):
 
 
 def decode_d3(raw: torch.Tensor) -> dict:
+    """bi_d3 bytes -> {mean, max, count, n_nonfinite, k1, k2, n_clipped, n_rejected}."""
     raw = raw.cpu()
     f = raw[:8].view(torch.float32)
     i = raw[8:24].view(torch.int64)
-    return {"mean": float(f[0]), "max": float(f[1]), "count": int(i[0]), "n_nonfinite": int(i[1])}
+    k = raw[24:32].view(torch.float32)
+    c = raw[32:40].view(torch.int32)
+    return {"mean": float(f[0]), "max": float(f[1]), "count": int(i[0]), "n_nonfinite": int(i[1]),
+            "k1": float(k[0]), "k2": float(k[1]), "n_clipped": int(c[0]), "n_rejected": int(c[1])}
 
 
 def debug_force_timeout_once(limit_ns: int) -> None:

@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <array>
+#include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -29,10 +30,11 @@ thread_local uint64_t g_force_timeout_ns = 0;
 // optional per-kernel timing (events around each launch; measurement tools only)
 // ---------------------------------------------------------------------------------------------
 enum KernelKind : int { kKPrep, kKRowmap, kKZeroRows, kKGather, kKLmFwd, kKLmFwdDH, kKLmDW, kKDwStream,
-                        kKRowParts, kKReduce, kKD3Partial, kNumKinds };
+                        kKSeqGate, kKRowParts, kKReduce, kKD3Partial, kNumKinds };
 const char* const kKindNames[kNumKinds] = {"k_prep", "k_rowmap", "k_zero_prompt_rows", "k_gather_rows",
                                            "k_lm_fwd", "k_lm_fwd_dh", "k_lm_dw", "k_dw_stream",
-                                           "k_row_parts", "k_reduce_parts", "k_d3_partial"};
+                                           "k_seq_gate", "k_row_parts", "k_reduce_parts", "k_d3_partial"};
+static_assert(sizeof(bi::D3Out) == sizeof(bi_d3), "device-written diagnostics match the ABI struct");
 struct Pending {
   int kind;
   cudaEvent_t a, b;
@@ -81,7 +83,8 @@ struct ProfScope {  // records an event pair around one launch when profiling is
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct WsLayout {
-  size_t ctrl, lse_c, g_c, tl_c, d3_c, y_c, logmu_c, rowmap, respof, coef, cprefix, red, hc, dz, alpha, fin;
+  size_t ctrl, lse_c, g_c, tl_c, d3_c, delta_c, clip_c, y_c, logmu_c, rowmap, respof, coef, cprefix, red, hc, dz,
+      alpha, fin;
   size_t dzy_c, mhist, pbuf;  // the P store (loss layout with the store only)
   size_t total;
   int nred;
@@ -113,6 +116,8 @@ WsLayout ws_layout(int64_t T, int32_t H, int32_t V, int32_t R, bool store) {
     L.g_c = take(tp * 4);
     L.tl_c = take(t * 4);
     L.d3_c = take(t * 4);
+    L.delta_c = take(t * 4);
+    L.clip_c = take(t);
     L.y_c = take(tp * 4);
     L.logmu_c = take(t * 4);
     L.rowmap = take(t * 4);
@@ -525,11 +530,18 @@ bi_status bi_logprob_fwd_noalloc(const uint16_t* hidden, const uint16_t* w_lm, c
 bi_status bi_is_loss_fwd_bwd(const uint16_t* hidden, const uint16_t* w_lm, const int32_t* targets,
                              const float* rollout_logprob, const float* rewards, const int64_t* resp_offsets,
                              const int32_t* group_offsets, const int32_t* prompt_lens, int32_t R, int32_t G,
-                             double resp_normalizer, int64_t T, int32_t H, int32_t V, float* loss, float* logprob,
+                             double resp_normalizer, const bi_loss_cfg* cfg, int64_t T, int32_t H, int32_t V,
+                             float* loss, float* logprob,
                              float* is_weight, float* token_loss, bi_d3* d3, uint16_t* grad_hidden, float* grad_w,
                              int32_t* dev_status, void* ws, size_t ws_bytes, void* stream) {
   if (T < 0 || T >= (int64_t(1) << 31) || H <= 0 || V <= 0 || R < 1 || G < 1 || G > R) return BI_ERR_INVALID_ARG;
   if (!(resp_normalizer >= 0.0)) return BI_ERR_INVALID_ARG;
+  const bi_loss_cfg lc = cfg ? *cfg : bi_loss_cfg{BI_LOSS_UNCLIPPED, 0.f, 0.f, 0.f};
+  if (lc.variant < BI_LOSS_UNCLIPPED || lc.variant > BI_LOSS_SEQ_GATE) return BI_ERR_INVALID_ARG;
+  if (lc.variant == BI_LOSS_PPO_CLIP &&
+      !(lc.eps_low >= 0.f && lc.eps_high >= 0.f && std::isfinite(lc.eps_low) && std::isfinite(lc.eps_high)))
+    return BI_ERR_INVALID_ARG;
+  if (lc.variant == BI_LOSS_SEQ_GATE && !(lc.gate >= 0.f)) return BI_ERR_INVALID_ARG;
   if (!dev_status || !w_lm || !rewards || !resp_offsets || !group_offsets || !loss || !grad_w)
     return BI_ERR_INVALID_ARG;
   if (T > 0 && (!hidden || !targets || !rollout_logprob || !logprob || !grad_hidden)) return BI_ERR_INVALID_ARG;
@@ -617,6 +629,11 @@ bi_status bi_is_loss_fwd_bwd(const uint16_t* hidden, const uint16_t* w_lm, const
   a.g_c = F(L.g_c);
   a.tl_c = F(L.tl_c);
   a.d3_c = F(L.d3_c);
+  a.delta_c = F(L.delta_c);
+  a.clip_c = reinterpret_cast<uint8_t*>(w8 + L.clip_c);
+  a.variant = lc.variant;
+  a.eps_low = lc.eps_low;
+  a.eps_high = lc.eps_high;
   a.logprob = logprob;
   a.is_weight = is_weight;
   a.token_loss = token_loss;
@@ -661,13 +678,22 @@ bi_status bi_is_loss_fwd_bwd(const uint16_t* hidden, const uint16_t* w_lm, const
     st = BI_OK;                                                                                            \
     if (T > 0) st = launch_lm<bi::kModeFwdDH, NZ_, HS_>(tm_h128, tm_wz, tm_w64, tm_dz, a, (T + 127) / 128, di, s); \
     if (st == BI_OK) {                                                                                     \
+      if (lc.variant == BI_LOSS_SEQ_GATE && T > 0) {                                                      \
+        ProfScope ps(kKSeqGate, s);                                                                        \
+        bi::k_seq_gate<<<R, 256, 0, s>>>(reinterpret_cast<const int64_t*>(w8 + L.cprefix), F(L.delta_c),  \
+                                         I(L.rowmap), lc.gate, H, ctrl, F(L.g_c), F(L.tl_c),              \
+                                         store ? F(L.dzy_c) : nullptr, token_loss, grad_hidden);          \
+      }                                                                                                    \
       {                                                                                                    \
         ProfScope ps(kKRowParts, s);                                                                       \
-        bi::k_row_parts<<<L.nred, bi::kRedBlock, 0, s>>>(F(L.tl_c), F(L.d3_c), ctrl, parts);              \
+        bi::k_row_parts<<<L.nred, bi::kRedBlock, 0, s>>>(F(L.tl_c), F(L.d3_c), F(L.delta_c),             \
+                                                         reinterpret_cast<const uint8_t*>(w8 + L.clip_c), \
+                                                         ctrl, parts);                                     \
       }                                                                                                    \
       {                                                                                                    \
         ProfScope ps(kKReduce, s);                                                                         \
-        bi::k_reduce_parts<<<1, 1024, 0, s>>>(parts, L.nred, loss, reinterpret_cast<bi::D3Out*>(d3), dev_status); \
+        bi::k_reduce_parts<<<1, 1024, 0, s>>>(parts, L.nred, loss, reinterpret_cast<bi::D3Out*>(d3), ctrl, \
+                                              dev_status);                                                 \
       }                                                                                                    \
       if (cudaGetLastError() != cudaSuccess) st = BI_ERR_CUDA;                                             \
     }                                                                                                      \
@@ -700,7 +726,7 @@ bi_status bi_d3_stats(const float* learner_logprob, const float* rollout_logprob
   }
   ProfScope ps(kKReduce, s);
   bi::k_reduce_parts<<<1, 1024, 0, s>>>(parts, static_cast<int>(nred), nullptr, reinterpret_cast<bi::D3Out*>(out),
-                                        dev_status);
+                                        nullptr, dev_status);
   return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
 }
 

@@ -88,6 +88,10 @@ struct LmArgs {
   float* g_c;              // -c_i w_t (kModeFwdDH writes, kModeDW reads)
   float* tl_c;             // token loss, for the fixed-order reduction (kModeFwdDH)
   float* d3_c;             // D3 term, for the fixed-order reduction (kModeFwdDH)
+  float* delta_c;          // log pi - log mu, for the KL estimators and the sequence gate (kModeFwdDH)
+  uint8_t* clip_c;         // 1 where the PPO clip removed the token's gradient (kModeFwdDH)
+  int32_t variant;         // loss variant: 0 unclipped, 1 PPO clip, 2 sequence gate (applied after)
+  float eps_low, eps_high; // PPO clip range [1 - eps_low, 1 + eps_high]
   // outputs at output rows
   float* logprob;
   float* lse_out;          // nullable
@@ -649,17 +653,32 @@ __device__ __forceinline__ void lm_fwd_epilogue_role(LmShared& sh, const LmArgs&
           const float delta = lp - a.logmu[t];
           const float w = expf(delta);
           const float d3 = expm1f(delta) - delta;
-          const float tlv = static_cast<float>(-a.coef[a.respof[t]] * static_cast<double>(w));
+          const double c = a.coef[a.respof[t]];
+          float tlv = static_cast<float>(-c * static_cast<double>(w));
+          uint8_t clipped = 0;
           g = tlv;
+          if (a.variant == 1) {
+            // -min(w A, clip(w) A) / (R* n) = -c min(w, 1 + eps_high) for A > 0 and
+            // -c max(w, 1 - eps_low) for A < 0; the gradient flows only where w itself is the
+            // selected term (c = A / (R* n) carries the sign of A)
+            const float hi = 1.f + a.eps_high, lo = 1.f - a.eps_low;
+            const bool pos = c > 0.0, neg = c < 0.0;
+            const bool active = pos ? (w <= hi) : (neg && w >= lo);
+            tlv = static_cast<float>(-c * static_cast<double>(pos ? fminf(w, hi) : fmaxf(w, lo)));
+            g = active ? static_cast<float>(-c * static_cast<double>(w)) : 0.f;
+            clipped = (pos || neg) && !active ? 1 : 0;
+          }
           if (x.rank == 0) {
             a.logprob[r] = lp;
             if (a.is_weight) a.is_weight[r] = w;
             if (a.token_loss) a.token_loss[r] = tlv;
             a.lse_c[t] = lse;
-            a.g_c[t] = tlv;
+            a.g_c[t] = g;
             a.tl_c[t] = tlv;
             a.d3_c[t] = d3;
-            if (a.dzy_c) a.dzy_c[t] = tlv * (s_ex / s);
+            a.delta_c[t] = delta;
+            a.clip_c[t] = clipped;
+            if (a.dzy_c) a.dzy_c[t] = g * (s_ex / s);
           }
         }
         // dH_t = (g / s) (s' W_y - O') on this CTA's columns; O', s' and s share the reference m*

@@ -1,12 +1,14 @@
 // kernels_small.cuh -- the light, memory-bound steps around the tensor-core kernels: offsets
-// validation and per-response coefficients, the scored-row map, the gather of scored rows and
-// the fixed-order reductions of the loss and the D3 statistics.  No atomics take part in any
-// sum: every reduction has a fixed tree shape that depends only on the number of rows.
+// validation and per-response coefficients, the scored-row map, the gather of scored rows, the
+// sequence gate of the comparison variant, and the fixed-order reductions of the loss, the D3
+// statistics and the KL estimators.  No atomics take part in any sum: every reduction has a fixed
+// tree shape that depends only on the number of rows.
 //
 // Definitions: "Zero Mismatch, Simple Async RL", sections "Only one probability gap comes from
 // old weights" (w = pi / mu, D3 = mean of w - 1 - log w) and "Alignment permits a simpler
 // learning path" (advantage = reward - group mean, tokens averaged within each response,
-// no clipping, no gate).
+// no clipping, no gate; the clip and the gate exist here as the baselines the pages compare
+// with).
 #pragma once
 
 #include "sm100.cuh"
@@ -18,16 +20,20 @@ constexpr int kRedBlock = 256;
 struct RedPart {
   double loss;
   double d3sum;
+  double k1sum;        // sum of -delta
+  double k2sum;        // sum of delta^2 / 2
   float d3max;
   int32_t pad;
   int64_t count;
   int64_t nonfinite;
+  int64_t nclip;       // tokens whose gradient the clip removed
 };
+__device__ __forceinline__ RedPart red_zero() { return RedPart{0.0, 0.0, 0.0, 0.0, -INFINITY, 0, 0, 0, 0}; }
 
 struct Ctrl {          // small device-side control block at the start of the workspace
   int64_t n_scored;    // number of scored (compact) rows
   int32_t valid;       // offsets passed validation
-  int32_t pad;
+  int32_t n_rejected;  // responses rejected by the sequence gate
 };
 
 // Largest i in [0, R) with off[i] <= r (off[R] > r is guaranteed by validation).
@@ -65,6 +71,7 @@ __global__ void k_prep(const float* __restrict__ rewards, const int64_t* __restr
       raise_status(status, 8 /* BI_ERR_BAD_OFFSETS */);
       ctrl->n_scored = 0;
       ctrl->valid = 0;
+      ctrl->n_rejected = 0;
     }
     return;
   }
@@ -89,6 +96,7 @@ __global__ void k_prep(const float* __restrict__ rewards, const int64_t* __restr
     cprefix[R] = acc;
     ctrl->n_scored = acc;
     ctrl->valid = 1;
+    ctrl->n_rejected = 0;
   }
 }
 
@@ -152,9 +160,12 @@ __device__ __forceinline__ RedPart block_reduce(RedPart v) {
   for (int o = 16; o > 0; o >>= 1) {
     v.loss += __shfl_xor_sync(0xffffffffu, v.loss, o);
     v.d3sum += __shfl_xor_sync(0xffffffffu, v.d3sum, o);
+    v.k1sum += __shfl_xor_sync(0xffffffffu, v.k1sum, o);
+    v.k2sum += __shfl_xor_sync(0xffffffffu, v.k2sum, o);
     v.d3max = fmaxf(v.d3max, __shfl_xor_sync(0xffffffffu, v.d3max, o));
     v.count += __shfl_xor_sync(0xffffffffu, v.count, o);
     v.nonfinite += __shfl_xor_sync(0xffffffffu, v.nonfinite, o);
+    v.nclip += __shfl_xor_sync(0xffffffffu, v.nclip, o);
   }
   __shared__ RedPart wp[32];
   const int w = threadIdx.x >> 5, nw = blockDim.x >> 5;
@@ -165,28 +176,41 @@ __device__ __forceinline__ RedPart block_reduce(RedPart v) {
     for (int i = 1; i < nw; ++i) {
       out.loss += wp[i].loss;
       out.d3sum += wp[i].d3sum;
+      out.k1sum += wp[i].k1sum;
+      out.k2sum += wp[i].k2sum;
       out.d3max = fmaxf(out.d3max, wp[i].d3max);
       out.count += wp[i].count;
       out.nonfinite += wp[i].nonfinite;
+      out.nclip += wp[i].nclip;
     }
   }
   return out;
 }
 
-// One thread per compact row: the block partial of the token losses and D3 terms that the
-// forward kernel left per row (loss = sum of token losses; D3 mean, max and non-finite count).
-__global__ void k_row_parts(const float* __restrict__ tl_c, const float* __restrict__ d3_c, const Ctrl* ctrl,
-                            RedPart* parts) {
+// Per-token diagnostic terms of one scored row: the D3 term (w - 1 - log w = expm1(delta) -
+// delta) and the sampled KL estimators k1 = -delta, k2 = delta^2 / 2.
+__device__ __forceinline__ void add_token(RedPart& v, float delta, float d3) {
+  const double dd = static_cast<double>(delta);
+  v.d3sum = static_cast<double>(d3);
+  v.d3max = d3;
+  v.k1sum = -dd;
+  v.k2sum = 0.5 * dd * dd;
+  v.count = 1;
+  v.nonfinite = isfinite(d3) ? 0 : 1;
+}
+
+// One thread per compact row: the block partial of the token losses and diagnostic terms that
+// the forward kernel left per row (loss = sum of token losses; D3, KL estimators, clip count).
+__global__ void k_row_parts(const float* __restrict__ tl_c, const float* __restrict__ d3_c,
+                            const float* __restrict__ delta_c, const uint8_t* __restrict__ clip_c,
+                            const Ctrl* ctrl, RedPart* parts) {
   const int64_t k = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t ns = ctrl->n_scored;
-  RedPart v{0.0, 0.0, -INFINITY, 0, 0, 0};
+  RedPart v = red_zero();
   if (k < ns) {
-    const float d3 = d3_c[k];
+    add_token(v, delta_c[k], d3_c[k]);
     v.loss = static_cast<double>(tl_c[k]);
-    v.d3sum = static_cast<double>(d3);
-    v.d3max = d3;
-    v.count = 1;
-    v.nonfinite = isfinite(d3) ? 0 : 1;
+    v.nclip = clip_c[k];
   }
   const RedPart b = block_reduce(v);
   if (threadIdx.x == 0) parts[blockIdx.x] = b;
@@ -196,47 +220,97 @@ __global__ void k_row_parts(const float* __restrict__ tl_c, const float* __restr
 __global__ void k_d3_partial(const float* __restrict__ lp, const float* __restrict__ mu,
                              const uint8_t* __restrict__ mask, int64_t T, RedPart* parts) {
   const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  RedPart v{0.0, 0.0, -INFINITY, 0, 0, 0};
+  RedPart v = red_zero();
   if (t < T && (mask == nullptr || mask[t] != 0)) {
     const float delta = lp[t] - mu[t];
-    const float d3 = expm1f(delta) - delta;
-    v.d3sum = static_cast<double>(d3);
-    v.d3max = d3;
-    v.count = 1;
-    v.nonfinite = isfinite(d3) ? 0 : 1;
+    add_token(v, delta, expm1f(delta) - delta);
   }
   const RedPart b = block_reduce(v);
   if (threadIdx.x == 0) parts[blockIdx.x] = b;
 }
 
-// One block: sum the block partials in a fixed order; write loss and D3 statistics.
-struct D3Out {
+// One block per response (sequence-gate variant).  rho_i = mean of delta over the response's
+// scored rows, summed in a fixed order in float64; a response with |rho_i| > gate (or a
+// non-finite rho_i) is rejected: its rows get no loss and no gradient (token loss, g, dZ at the
+// target and the dH rows set to 0).  Runs after the forward and before the reductions and dW.
+__global__ void k_seq_gate(const int64_t* __restrict__ cprefix, const float* __restrict__ delta_c,
+                           const int32_t* __restrict__ rowmap, float gate, int H, Ctrl* ctrl,
+                           float* __restrict__ g_c, float* __restrict__ tl_c, float* __restrict__ dzy_c,
+                           float* __restrict__ token_loss, uint16_t* __restrict__ grad_hidden) {
+  if (!ctrl->valid) return;
+  const int i = blockIdx.x;
+  const int64_t k0 = cprefix[i], k1 = cprefix[i + 1];
+  if (k1 <= k0) return;
+  double part = 0.0;
+  for (int64_t k = k0 + threadIdx.x; k < k1; k += blockDim.x) part += static_cast<double>(delta_c[k]);
+  for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+  __shared__ double wsum[32];
+  __shared__ int reject;
+  if ((threadIdx.x & 31) == 0) wsum[threadIdx.x >> 5] = part;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double tot = 0.0;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) tot += wsum[w];
+    const double rho = tot / static_cast<double>(k1 - k0);
+    reject = !(fabs(rho) <= static_cast<double>(gate));
+    if (reject) atomicAdd(&ctrl->n_rejected, 1);
+  }
+  __syncthreads();
+  if (!reject) return;
+  for (int64_t k = k0 + threadIdx.x; k < k1; k += blockDim.x) {
+    g_c[k] = 0.f;
+    tl_c[k] = 0.f;
+    if (dzy_c) dzy_c[k] = 0.f;
+    if (token_loss) token_loss[rowmap[k]] = 0.f;
+  }
+  const int q8 = H / 8;
+  for (int64_t e = threadIdx.x; e < (k1 - k0) * q8; e += blockDim.x) {
+    const int64_t k = k0 + e / q8;
+    reinterpret_cast<uint4*>(grad_hidden + static_cast<int64_t>(rowmap[k]) * H)[e % q8] = make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+// One block: sum the block partials in a fixed order; write the loss and the diagnostics.
+struct D3Out {  // layout of bi_d3
   float mean;
   float max;
   int64_t count;
   int64_t n_nonfinite;
+  float k1_mean;
+  float k2_mean;
+  int32_t n_clipped;
+  int32_t n_rejected;
 };
 
 __global__ void k_reduce_parts(const RedPart* __restrict__ parts, int nparts, float* loss, D3Out* d3,
-                               int32_t* status) {
-  RedPart v{0.0, 0.0, -INFINITY, 0, 0, 0};
+                               const Ctrl* ctrl, int32_t* status) {
+  RedPart v = red_zero();
   for (int i = threadIdx.x; i < nparts; i += blockDim.x) {
     const RedPart p = parts[i];
     v.loss += p.loss;
     v.d3sum += p.d3sum;
+    v.k1sum += p.k1sum;
+    v.k2sum += p.k2sum;
     v.d3max = fmaxf(v.d3max, p.d3max);
     v.count += p.count;
     v.nonfinite += p.nonfinite;
+    v.nclip += p.nclip;
   }
   const RedPart b = block_reduce(v);
   if (threadIdx.x == 0) {
     if (loss) *loss = static_cast<float>(b.loss);
     if (d3) {
       D3Out o;
-      o.mean = (b.count > 0) ? static_cast<float>(b.d3sum / static_cast<double>(b.count)) : 0.f;
-      o.max = (b.count > 0) ? b.d3max : 0.f;
+      const bool any = b.count > 0;
+      const double n = static_cast<double>(b.count);
+      o.mean = any ? static_cast<float>(b.d3sum / n) : 0.f;
+      o.max = any ? b.d3max : 0.f;
       o.count = b.count;
       o.n_nonfinite = b.nonfinite;
+      o.k1_mean = any ? static_cast<float>(b.k1sum / n) : 0.f;
+      o.k2_mean = any ? static_cast<float>(b.k2sum / n) : 0.f;
+      o.n_clipped = static_cast<int32_t>(b.nclip);
+      o.n_rejected = ctrl ? ctrl->n_rejected : 0;
       *d3 = o;
     }
     if (b.nonfinite > 0 || (loss && !isfinite(b.loss))) raise_status(status, 7 /* BI_ERR_NONFINITE */);

@@ -74,16 +74,46 @@ typedef enum {
   BI_ERR_BAD_OFFSETS = 8        /* device: offsets not monotone / not covering the rows */
 } bi_status;
 
-/* D3 statistics of one call ("Zero Mismatch", section "Only one probability gap ..."):
- * mean and max of d3_t = w_t - 1 - log w_t over the scored tokens, the number of scored tokens and
- * the number of non-finite terms.  mean and max are non-finite when any term is.  Written by the
- * library to device memory. */
+/* Diagnostics of one call, written by the library to device memory.
+ *   mean, max, count, n_nonfinite: D3 statistics ("Zero Mismatch", section "Only one probability
+ *     gap ..."): mean and max of d3_t = w_t - 1 - log w_t over the scored tokens, the number of
+ *     scored tokens and the number of non-finite terms; mean and max are non-finite when any term
+ *     is.
+ *   k1_mean, k2_mean: the other sampled estimators of the rollout-to-learner KL(mu || pi) from the
+ *     rollout's tokens (the pages plot a "sampled estimate" of this KL): means of -delta and of
+ *     delta^2 / 2, delta = log pi - log mu.  D3 is the third one, k3.
+ *   n_clipped: tokens whose gradient the PPO clip removed (BI_LOSS_PPO_CLIP), else 0.
+ *   n_rejected: responses the sequence gate rejected (BI_LOSS_SEQ_GATE), else 0.
+ * bi_d3_stats fills mean ... k2_mean and sets both counters to 0. */
 typedef struct {
   float mean;
   float max;
   int64_t count;
   int64_t n_nonfinite;
+  float k1_mean;
+  float k2_mean;
+  int32_t n_clipped;
+  int32_t n_rejected;
 } bi_d3;
+
+/* Loss of bi_is_loss_fwd_bwd.  The method is the unclipped one; the two others are the baselines
+ * the pages compare it with ("Zero Mismatch", section "Alignment permits a simpler learning path":
+ * clipping suppresses excursions but biases, rejection gates discard samples).  The pages give no
+ * formula for either; the readings:
+ *   BI_LOSS_UNCLIPPED  l_t = -c_i w_t, c_i = A_i / (R* n_i)
+ *   BI_LOSS_PPO_CLIP   l_t = -min(w_t A_i, clip(w_t, 1 - eps_low, 1 + eps_high) A_i) / (R* n_i),
+ *                      differentiated through w_t only (no gradient where the clipped term is the
+ *                      smaller one)
+ *   BI_LOSS_SEQ_GATE   the unclipped terms, except that response i contributes nothing (loss and
+ *                      gradient) when its mean token log-ratio rho_i = mean_t (log pi_t - log mu_t)
+ *                      has |rho_i| > gate or is not finite; it still counts in R*. */
+typedef enum { BI_LOSS_UNCLIPPED = 0, BI_LOSS_PPO_CLIP = 1, BI_LOSS_SEQ_GATE = 2 } bi_loss_variant;
+typedef struct {
+  int32_t variant;  /* bi_loss_variant */
+  float eps_low;    /* PPO_CLIP: >= 0 */
+  float eps_high;   /* PPO_CLIP: >= 0 */
+  float gate;       /* SEQ_GATE: >= 0 (may be +inf) */
+} bi_loss_cfg;
 
 /* Size in bytes of the scratch workspace for these sizes (R = number of responses; pass 0 for
  * bi_logprob_fwd / bi_d3_stats).  Deterministic and free of side effects; the caller allocates
@@ -134,7 +164,8 @@ BI_API bi_status bi_logprob_fwd_noalloc(const uint16_t* hidden, const uint16_t* 
                                         float* logprob, float* lse, int32_t* dev_status,
                                         void* stream);
 
-/* Fused forward + backward of the unclipped token-level IS REINFORCE loss.
+/* Fused forward + backward of the token-level IS REINFORCE loss (unclipped unless cfg says
+ * otherwise).
  *   hidden, w_lm, targets, T, H, V   as in bi_logprob_fwd (T = all packed rows)
  *   rollout_logprob [T] float   log mu of each row's target under the rollout policy
  *   rewards        [R] float    one reward per response
@@ -146,12 +177,13 @@ BI_API bi_status bi_logprob_fwd_noalloc(const uint16_t* hidden, const uint16_t* 
  *                               scored (0 <= prompt_lens[i] <= its length)
  *   resp_normalizer  R* in c_i = A_i / (R* n_i); 0 means R.  Data-parallel callers pass the
  *                               global number of responses.
+ *   cfg              (may be NULL: BI_LOSS_UNCLIPPED) host pointer, read during the call
  * Outputs (device):
  *   loss        [1]    float   L (sum over scored tokens in a fixed order, float64 accumulation)
  *   logprob     [T]    float   log pi_t on scored rows, 0 on prompt rows
  *   is_weight   [T]    float   (may be NULL) w_t, 0 on prompt rows
- *   token_loss  [T]    float   (may be NULL) -c_i w_t, 0 on prompt rows
- *   d3          [1]    bi_d3   (may be NULL) D3 statistics over the scored rows
+ *   token_loss  [T]    float   (may be NULL) l_t of the loss variant, 0 on prompt rows
+ *   d3          [1]    bi_d3   (may be NULL) D3, KL estimators and variant counters
  *   grad_hidden [T, H] bf16    dL/dh_t (zero rows for prompt rows)
  *   grad_w      [V, H] float   dL/dW, overwritten (not accumulated)
  * A response with no scored row contributes 0 and still counts in R*. */
@@ -159,8 +191,8 @@ BI_API bi_status bi_is_loss_fwd_bwd(const uint16_t* hidden, const uint16_t* w_lm
                              const float* rollout_logprob, const float* rewards,
                              const int64_t* resp_offsets, const int32_t* group_offsets,
                              const int32_t* prompt_lens, int32_t R, int32_t G,
-                             double resp_normalizer, int64_t T, int32_t H, int32_t V,
-                             float* loss, float* logprob, float* is_weight, float* token_loss,
+                             double resp_normalizer, const bi_loss_cfg* cfg, int64_t T, int32_t H,
+                             int32_t V, float* loss, float* logprob, float* is_weight, float* token_loss,
                              bi_d3* d3, uint16_t* grad_hidden, float* grad_w,
                              int32_t* dev_status, void* ws, size_t ws_bytes, void* stream);
 

@@ -90,12 +90,13 @@ def test_logprob_argument_checks(lib):
 def test_is_loss_argument_checks(lib):
     T, H, V, R = 40, 128, 512, 4
     ws_bytes = lib.bi_workspace_bytes(T, H, V, R)
-    args = [FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, R, 2, 0.0, T, H, V,
+    args = [FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, R, 2, 0.0, None, T, H, V,
             FAKE, FAKE, None, None, None, FAKE, FAKE, FAKE, FAKE, ws_bytes, None]
 
     def call(**kw):
         a = list(args)
-        idx = {"hidden": 0, "R": 8, "G": 9, "rnorm": 10, "H": 12, "grad_w": 20, "ws_bytes": 23, "loss": 14}
+        idx = {"hidden": 0, "R": 8, "G": 9, "rnorm": 10, "cfg": 11, "H": 13, "grad_w": 21, "ws_bytes": 24,
+               "loss": 15}
         for k, v in kw.items():
             a[idx[k]] = v
         return lib.bi_is_loss_fwd_bwd(*a)
@@ -107,6 +108,12 @@ def test_is_loss_argument_checks(lib):
     assert call(loss=None) == 1
     assert call(grad_w=FAKE + 4) == 1  # misaligned
     assert call(H=704) == 2            # 11 * 64: no split into <= 384-column multiples of 64 with C <= 8
+    bad_variant = _lib.LossCfg(7, 0.2, 0.2, 1.0)
+    assert call(cfg=ctypes.addressof(bad_variant)) == 1
+    bad_eps = _lib.LossCfg(1, -0.1, 0.2, 1.0)
+    assert call(cfg=ctypes.addressof(bad_eps)) == 1
+    bad_gate = _lib.LossCfg(2, 0.2, 0.2, float("nan"))
+    assert call(cfg=ctypes.addressof(bad_gate)) == 1
     ws_min = lib.bi_workspace_bytes_min(T, H, V, R)
     assert 0 < ws_min < ws_bytes
     assert call(ws_bytes=ws_min - 1) == 3

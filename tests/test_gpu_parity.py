@@ -2,6 +2,8 @@
 
 Sizes span several tiles and ragged tails (rows not a multiple of 128, vocabularies not a
 multiple of 256 or 32) and include the full H = 1536, V = 151936 head."""
+import math
+
 import numpy as np
 import pytest
 import torch
@@ -76,19 +78,20 @@ def test_bad_target_sets_status(cuda_device):
 
 
 def _loss_case(batch, cuda_device, rollout_lp=None, resp_normalizer=0.0, check_dw=True, tight=1e-4,
-               minimal_ws=False):
+               minimal_ws=False, variant_kw=None):
     b = batch
     if rollout_lp is None:
         rollout_lp, _ = orc.token_logprob(b.hidden, b.w_roll, b.targets)
         rollout_lp = rollout_lp + b.logmu_noise.double().numpy()
     mu = torch.tensor(rollout_lp, dtype=torch.float32)
     mu64 = mu.double().numpy()   # the oracle sees exactly the fp32 values the GPU sees
+    vkw = dict(variant_kw or {})
     ref = orc.is_loss_fwd_bwd(b.hidden, b.w, b.targets, mu64, b.rewards, b.resp_offsets, b.group_offsets,
-                              b.prompt_lens, resp_normalizer, want_grad_w=check_dw)
+                              b.prompt_lens, resp_normalizer, want_grad_w=check_dw, **vkw)
     d = b.to(cuda_device)
     ws = bi.make_workspace(d.n_rows, d.hidden.shape[1], d.w.shape[0], d.R, cuda_device, minimal=minimal_ws)
     out = bi.is_loss_fwd_bwd(d.hidden, d.w, d.targets, mu.to(cuda_device), d.rewards, d.resp_offsets,
-                             d.group_offsets, d.prompt_lens, resp_normalizer, ws=ws)
+                             d.group_offsets, d.prompt_lens, resp_normalizer, ws=ws, **vkw)
     torch.cuda.synchronize()
     bi.check_status(out.status)
     assert_close("loss", f64(out.loss), [ref["loss"]], LOSS_TOL, LOSS_TOL)
@@ -103,6 +106,9 @@ def _loss_case(batch, cuda_device, rollout_lp=None, resp_normalizer=0.0, check_d
     d3 = out.d3()
     assert d3["count"] == ref["d3"]["count"] and d3["n_nonfinite"] == 0
     assert_close("d3.mean", [d3["mean"]], [ref["d3"]["mean"]], 1e-7, 5e-2)
+    assert_close("kl.k1", [d3["k1"]], [ref["kl"]["k1"]], 1e-6, 5e-2)
+    assert_close("kl.k2", [d3["k2"]], [ref["kl"]["k2"]], 1e-7, 5e-2)
+    assert d3["n_clipped"] == ref["n_clipped"] and d3["n_rejected"] == ref["n_rejected"]
     assert_grad_close("grad_hidden", f64(out.grad_hidden), ref["grad_hidden"])
     if check_dw:
         assert_grad_close("grad_w", f64(out.grad_w), ref["grad_w"])
@@ -149,6 +155,56 @@ def test_loss_low_memory_path(name, kw, cuda_device):
     for f in ("loss", "logprob", "is_weight", "token_loss", "grad_hidden", "d3_raw"):
         assert torch.equal(getattr(lo, f), getattr(hi, f)), f
     assert not torch.equal(lo.grad_w, hi.grad_w) or b.n_rows == 0  # two different dW kernels ran
+
+
+def _variant_batch(H=256, V=3001, noise=0.35):
+    """A batch whose rollout log-probabilities carry N(0, noise) on top of the lagged head, so that
+    weights leave the clip range and responses differ in their mean log-ratio."""
+    b = make_batch(spec_for("tiny", H=H, V=V, groups=3, per_group=4, len_lo=8, len_hi=40, prompt_len=2))
+    mu, _ = orc.token_logprob(b.hidden, b.w_roll, b.targets)
+    mu = mu + np.random.default_rng(99).normal(size=mu.shape[0]) * noise
+    return b, mu
+
+
+def _away_from(values, x, margin):
+    return bool(np.all(np.abs(np.asarray(values, dtype=np.float64) - x) > margin))
+
+
+@pytest.mark.parametrize("minimal_ws", [False, True])
+def test_loss_ppo_clip(minimal_ws, cuda_device):
+    """The clipped-surrogate baseline: token losses, the gradient only where w itself is the
+    selected term, and the count of clipped tokens (no weight within 1e-3 of the clip bounds, so
+    the fp32 and fp64 decisions agree)."""
+    b, mu = _variant_batch()
+    mu32 = torch.tensor(mu, dtype=torch.float32).double().numpy()
+    w_ref = orc.is_loss_fwd_bwd(b.hidden, b.w, b.targets, mu32, b.rewards, b.resp_offsets, b.group_offsets,
+                                b.prompt_lens, want_grads=False)["is_weight"]
+    eps = 0.2
+    while not (_away_from(w_ref[w_ref != 0], 1 - eps, 1e-3) and _away_from(w_ref[w_ref != 0], 1 + eps, 1e-3)):
+        eps += 0.0037
+    out, ref = _loss_case(b, cuda_device, rollout_lp=mu, minimal_ws=minimal_ws,
+                          variant_kw=dict(variant="ppo_clip", eps_low=eps, eps_high=eps))
+    assert 0 < ref["n_clipped"] < int(ref["mask"].sum())
+
+
+@pytest.mark.parametrize("minimal_ws", [False, True])
+def test_loss_sequence_gate(minimal_ws, cuda_device):
+    """The rejection-gate baseline with the threshold half-way between two responses' |rho|:
+    rejected responses have zero token losses and zero dH rows; the rejection count matches."""
+    b, mu = _variant_batch()
+    mu32 = torch.tensor(mu, dtype=torch.float32).double().numpy()
+    probe = orc.is_loss_fwd_bwd(b.hidden, b.w, b.targets, mu32, b.rewards, b.resp_offsets, b.group_offsets,
+                                b.prompt_lens, want_grads=False, variant="seq_gate", gate=math.inf)
+    a = np.sort(np.abs(probe["rho"]))
+    gate = float(0.5 * (a[len(a) // 2 - 1] + a[len(a) // 2]))
+    assert _away_from(np.abs(probe["rho"]), gate, 1e-4)
+    out, ref = _loss_case(b, cuda_device, rollout_lp=mu, minimal_ws=minimal_ws,
+                          variant_kw=dict(variant="seq_gate", gate=gate))
+    assert 0 < ref["n_rejected"] < b.R
+    off = b.resp_offsets.numpy()
+    dh = f64(out.grad_hidden)
+    for i in np.nonzero(ref["rejected"])[0]:
+        assert not np.any(dh[off[i]:off[i + 1]])
 
 
 @pytest.mark.parametrize("H,V", [(256, 3001), (1536, 8000)])
