@@ -29,10 +29,10 @@ thread_local uint64_t g_force_timeout_ns = 0;
 // ---------------------------------------------------------------------------------------------
 // optional per-kernel timing (events around each launch; measurement tools only)
 // ---------------------------------------------------------------------------------------------
-enum KernelKind : int { kKPrep, kKRowmap, kKZeroRows, kKGather, kKLmFwd, kKLmFwdDH, kKLmDW, kKDwStream,
-                        kKSeqGate, kKRowParts, kKReduce, kKD3Partial, kNumKinds };
+enum KernelKind : int { kKPrep, kKRowmap, kKZeroRows, kKGather, kKLmFwd, kKLmFwdDH, kKLmDW, kKDwRows,
+                        kKDwStream, kKSeqGate, kKRowParts, kKReduce, kKD3Partial, kNumKinds };
 const char* const kKindNames[kNumKinds] = {"k_prep", "k_rowmap", "k_zero_prompt_rows", "k_gather_rows",
-                                           "k_lm_fwd", "k_lm_fwd_dh", "k_lm_dw", "k_dw_stream",
+                                           "k_lm_fwd", "k_lm_fwd_dh", "k_lm_dw", "k_dw_rows", "k_dw_stream",
                                            "k_seq_gate", "k_row_parts", "k_reduce_parts", "k_d3_partial"};
 static_assert(sizeof(bi::D3Out) == sizeof(bi_d3), "device-written diagnostics match the ABI struct");
 struct Pending {
@@ -85,7 +85,7 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 struct WsLayout {
   size_t ctrl, lse_c, g_c, tl_c, d3_c, delta_c, clip_c, y_c, logmu_c, rowmap, respof, coef, cprefix, red, hc, dz,
       alpha, fin;
-  size_t dzy_c, mhist, pbuf;  // the P store (loss layout with the store only)
+  size_t sxr_c, mhist, hs, pbuf;  // the P store (loss layout with the store only)
   size_t total;
   int nred;
   int64_t tpad, pcols;        // rows and columns the P store is sized for
@@ -95,7 +95,8 @@ constexpr size_t kFinBytes = static_cast<size_t>(kMaxSms) * 2 * 384 * sizeof(flo
 
 // R == 0: the logprob-only layout (per-CTA partials only).  R > 0: the loss layout; with
 // `store`, followed by the P store of the fused forward ([Tpad][V + 256] bf16, enough for any
-// logit-tile width NZ <= 256) and the per-step reference history ([ceil(V / 128)][Tpad] float).
+// logit-tile width NZ <= 256), the per-step reference history ([ceil(V / 128)][Tpad] float) and
+// the scaled hidden states of the dW GEMM ([Tpad][H] bf16).
 WsLayout ws_layout(int64_t T, int32_t H, int32_t V, int32_t R, bool store) {
   WsLayout L{};
   const size_t t = static_cast<size_t>(T > 0 ? T : 1);
@@ -132,7 +133,8 @@ WsLayout ws_layout(int64_t T, int32_t H, int32_t V, int32_t R, bool store) {
     if (store) {
       L.tpad = static_cast<int64_t>((t + 127) / 128 * 128);
       L.pcols = (static_cast<int64_t>(V) + 127) / 128 * 128 + 256;
-      L.dzy_c = take(tp * 4);
+      L.sxr_c = take(tp * 4);
+      L.hs = take(static_cast<size_t>(L.tpad) * static_cast<size_t>(H) * 2);
       L.mhist = take(static_cast<size_t>((V + 127) / 128) * static_cast<size_t>(L.tpad) * 4);
       L.pbuf = take(static_cast<size_t>(L.tpad) * static_cast<size_t>(L.pcols) * 2);
     }
@@ -606,7 +608,7 @@ bi_status bi_is_loss_fwd_bwd(const uint16_t* hidden, const uint16_t* w_lm, const
   const int dw_hs = dw_split(H);
   if (store ? !(make_map(&tm_dz, w8 + L.pbuf, L.tpad, p_ld, 128) &&
                 make_map_blocks(&tm_p64, w8 + L.pbuf, L.tpad, p_ld, 64, 4) &&
-                make_map_blocks(&tm_hblk, hsrc, trows, H, 64, dw_hs / 64))
+                make_map_blocks(&tm_hblk, w8 + L.hs, L.tpad, H, 64, dw_hs / 64))
             : !make_map(&tm_dz, w8 + L.dz, static_cast<int64_t>(kDzSlotsMax) * 128, pl.NZ, 128))
     return BI_ERR_CUDA;
   bi::LmArgs a{};
@@ -650,7 +652,7 @@ bi_status bi_is_loss_fwd_bwd(const uint16_t* hidden, const uint16_t* w_lm, const
     a.p_ld = p_ld;
     a.mhist = F(L.mhist);
     a.Tpad = L.tpad;
-    a.dzy_c = F(L.dzy_c);
+    a.sxr_c = F(L.sxr_c);
     da.H = H;
     da.V = V;
     da.Hs = dw_split(H);
@@ -661,11 +663,8 @@ bi_status bi_is_loss_fwd_bwd(const uint16_t* hidden, const uint16_t* w_lm, const
     da.d_rows = d_rows;
     da.nv128 = a.nv128;
     da.nitems = ((a.nv128 + 1) / 2) * da.nsl;
-    da.lse_c = F(L.lse_c);
-    da.g_c = F(L.g_c);
-    da.y_c = I(L.y_c);
-    da.dzy_c = F(L.dzy_c);
     da.mhist = F(L.mhist);
+    da.y_c = I(L.y_c);
     da.grad_w = grad_w;
     da.status = dev_status;
     da.limit_ns = kWaitLimitNs;
@@ -681,8 +680,8 @@ bi_status bi_is_loss_fwd_bwd(const uint16_t* hidden, const uint16_t* w_lm, const
       if (lc.variant == BI_LOSS_SEQ_GATE && T > 0) {                                                      \
         ProfScope ps(kKSeqGate, s);                                                                        \
         bi::k_seq_gate<<<R, 256, 0, s>>>(reinterpret_cast<const int64_t*>(w8 + L.cprefix), F(L.delta_c),  \
-                                         I(L.rowmap), lc.gate, H, ctrl, F(L.g_c), F(L.tl_c),              \
-                                         store ? F(L.dzy_c) : nullptr, token_loss, grad_hidden);          \
+                                         I(L.rowmap), lc.gate, H, ctrl, F(L.g_c), F(L.tl_c), token_loss,  \
+                                         grad_hidden);                                                     \
       }                                                                                                    \
       {                                                                                                    \
         ProfScope ps(kKRowParts, s);                                                                       \
@@ -702,6 +701,15 @@ bi_status bi_is_loss_fwd_bwd(const uint16_t* hidden, const uint16_t* w_lm, const
   BI_LM_CONFIGS(BI_LAUNCH)
 #undef BI_LAUNCH
   if (st == BI_OK && store) {
+    {
+      // scaled hidden states H' and the target entries of the P store, then the dW GEMM
+      ProfScope ps(kKDwRows, s);
+      bi::k_dw_rows<<<blocks_for(L.tpad * 32, 256), 256, 0, s>>>(
+          static_cast<const uint16_t*>(hsrc), H, d_rows, L.tpad, F(L.lse_c), F(L.g_c), F(L.sxr_c), I(L.y_c),
+          F(L.mhist), nvz, V, reinterpret_cast<uint16_t*>(w8 + L.hs), reinterpret_cast<uint16_t*>(w8 + L.pbuf),
+          p_ld);
+      if (cudaGetLastError() != cudaSuccess) return BI_ERR_CUDA;
+    }
     st = BI_ERR_UNSUPPORTED_SHAPE;
 #define BI_LAUNCH_DW(HS_) \
     if (da.Hs == HS_) st = launch_dw<HS_>(tm_p64, tm_hblk, da, di, s);

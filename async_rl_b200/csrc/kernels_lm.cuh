@@ -104,7 +104,7 @@ struct LmArgs {
   int64_t p_ld;            // nvz * NZ
   float* mhist;            // [nvz][Tpad] reference of each row at each step
   int64_t Tpad;            // ceil(T / 128) * 128
-  float* dzy_c;            // [rows] dZ at the target column, g (1 - p_y)
+  float* sxr_c;            // [rows] s' / s = 1 - p_y (P store only)
   // scratch
   uint16_t* dz_scratch;    // [clusters * C * kSlotsPerCta * 128][NZ] bf16 (P or dZ tiles)
   float* alpha;            // [clusters * C * kSlotsPerCta][128] per-row O rescale factors (kModeFwdDH)
@@ -678,7 +678,7 @@ __device__ __forceinline__ void lm_fwd_epilogue_role(LmShared& sh, const LmArgs&
             a.d3_c[t] = d3;
             a.delta_c[t] = delta;
             a.clip_c[t] = clipped;
-            if (a.dzy_c) a.dzy_c[t] = g * (s_ex / s);
+            if (a.sxr_c) a.sxr_c[t] = s_ex / s;
           }
         }
         // dH_t = (g / s) (s' W_y - O') on this CTA's columns; O', s' and s share the reference m*

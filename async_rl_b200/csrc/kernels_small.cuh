@@ -231,12 +231,12 @@ __global__ void k_d3_partial(const float* __restrict__ lp, const float* __restri
 
 // One block per response (sequence-gate variant).  rho_i = mean of delta over the response's
 // scored rows, summed in a fixed order in float64; a response with |rho_i| > gate (or a
-// non-finite rho_i) is rejected: its rows get no loss and no gradient (token loss, g, dZ at the
-// target and the dH rows set to 0).  Runs after the forward and before the reductions and dW.
+// non-finite rho_i) is rejected: its rows get no loss and no gradient (token loss, g and the dH
+// rows set to 0).  Runs after the forward and before the reductions and dW.
 __global__ void k_seq_gate(const int64_t* __restrict__ cprefix, const float* __restrict__ delta_c,
                            const int32_t* __restrict__ rowmap, float gate, int H, Ctrl* ctrl,
-                           float* __restrict__ g_c, float* __restrict__ tl_c, float* __restrict__ dzy_c,
-                           float* __restrict__ token_loss, uint16_t* __restrict__ grad_hidden) {
+                           float* __restrict__ g_c, float* __restrict__ tl_c, float* __restrict__ token_loss,
+                           uint16_t* __restrict__ grad_hidden) {
   if (!ctrl->valid) return;
   const int i = blockIdx.x;
   const int64_t k0 = cprefix[i], k1 = cprefix[i + 1];
@@ -260,7 +260,6 @@ __global__ void k_seq_gate(const int64_t* __restrict__ cprefix, const float* __r
   for (int64_t k = k0 + threadIdx.x; k < k1; k += blockDim.x) {
     g_c[k] = 0.f;
     tl_c[k] = 0.f;
-    if (dzy_c) dzy_c[k] = 0.f;
     if (token_loss) token_loss[rowmap[k]] = 0.f;
   }
   const int q8 = H / 8;
