@@ -146,7 +146,7 @@ def is_loss_fwd_bwd(hidden, w, targets, rollout_logprob, rewards, resp_offsets, 
 
 
 def d3_stats(learner_logprob, rollout_logprob, mask=None, ws=None):
-    """D3 statistics of two logprob arrays.  Returns (d3 dict tensor bytes [24] u8, status)."""
+    """D3 and KL statistics of two logprob arrays.  Returns (bi_d3 bytes [40] u8, status)."""
     dev = learner_logprob.device
     T = learner_logprob.shape[0]
     _check_cuda(learner_logprob, "learner_logprob", torch.float32, dev)

@@ -64,6 +64,28 @@ def measured_peaks():
     return {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}, "fallback"
 
 
+TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "dram_traffic_qwen1.5b_step.md")
+CSRC_HASHED = ("sm100.cuh", "kernels_lm.cuh", "kernels_dw.cuh", "kernels_small.cuh", "bi_api.cu")
+
+
+def recorded_traffic(kernel: str):
+    """DRAM bytes per launch of `kernel` from the committed full-size ncu record, or None when the
+    CUDA sources changed since that capture (the record carries their sha256)."""
+    import hashlib
+    if not os.path.exists(TRAFFIC_RECORD):
+        return None
+    h = hashlib.sha256()
+    for f in CSRC_HASHED:
+        with open(os.path.join(ROOT, "async_rl_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    with open(TRAFFIC_RECORD) as fh:
+        for ln in fh:
+            parts = ln.split()
+            if len(parts) == 4 and parts[0] == "traffic" and parts[1] == kernel and parts[3] == h.hexdigest():
+                return int(parts[2])
+    return None
+
+
 class ClockSampler:
     """nvidia-smi clock / throttle-reason samples during the timed region."""
 
@@ -266,7 +288,7 @@ def run_ours(args):
         host["logmu"] = logmu.cpu().pin_memory()
         dbuf = {k: torch.empty_like(v, device=dev) for k, v in host.items()}
         loss_h = torch.empty(1, dtype=torch.float32).pin_memory()
-        d3_h = torch.empty(24, dtype=torch.uint8).pin_memory()
+        d3_h = torch.empty(out.d3_raw.numel(), dtype=torch.uint8).pin_memory()
         h2d = sum(v.numel() * v.element_size() for v in host.values())
         d2h = loss_h.numel() * 4 + d3_h.numel()
 
@@ -320,7 +342,8 @@ def run_ours(args):
                        "l2": "inputs larger than L2 (hidden 0.23 GB, W 0.47 GB); no flush"},
             "pct_bf16_peak": 100.0 * step_tflops / peak_tf,
             "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak_tf,
-                         "unit": "TFLOP/s", "frac": achieved / peak_tf, "traffic": None,
+                         "unit": "TFLOP/s", "frac": achieved / peak_tf,
+                         "traffic": recorded_traffic(dom) if (CONFIG == "qwen1.5b" and not args.small) else None,
                          "peak_source": f"{peak_src} bf16_tflops_sustained",
                          "algorithmic_flops_per_launch": alg[dom],
                          "executed_frac": executed[dom] / (davg * 1e-3) / 1e12 / peak_tf},
