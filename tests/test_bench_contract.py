@@ -1,0 +1,44 @@
+"""bench.py keeps its contract: one JSON line with the keys the driver reads.  The reference arm
+(the fp64 oracle on host cores) runs here on CPU; the CUDA arm runs its small profiling case on
+the GPU (the same code path as the full line, T = 4096)."""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+REQUIRED = ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+            "scaling", "vs_baseline", "dtype", "data", "config", "e2e")
+
+
+def _run(args, timeout):
+    proc = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py")] + args, cwd=ROOT, capture_output=True,
+                          text=True, timeout=timeout)
+    assert proc.returncode == 0, proc.stderr[-2000:]
+    lines = [ln for ln in proc.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, proc.stdout[-2000:]
+    return json.loads(lines[0])
+
+
+@pytest.mark.slow
+def test_reference_arm_line():
+    line = _run(["--impl", "reference", "--steps", "1", "--warmup", "0"], timeout=600)
+    for k in REQUIRED:
+        assert k in line, k
+    assert line["impl"] == "reference" and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+@pytest.mark.gpu
+def test_cuda_arm_line_small_case():
+    line = _run(["--small", "--steps", "2", "--warmup", "3", "--no-cpu-baseline"], timeout=900)
+    for k in REQUIRED + ("roofline", "clocks", "gpu_launches"):
+        assert k in line, k
+    assert line["value"] > 0 and line["gpu_launches"] > 0
+    roof = line["roofline"]
+    for k in ("bound", "achieved", "peak", "unit", "frac", "traffic"):
+        assert k in roof, k
+    assert 0 < roof["frac"] < 2
+    assert line["e2e"]["value"] > 0 and line["e2e"]["h2d_bytes_per_step"] > 0
