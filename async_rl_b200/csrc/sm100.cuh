@@ -48,10 +48,6 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
-// named barrier among `nthreads` threads (multiple of 32)
-__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
 
 // ----------------------------------------------------------------------------------------------
 // mbarrier
