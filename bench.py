@@ -280,51 +280,72 @@ def run_ours(args):
         total_tokens, ms_max = float(T), ms
     value = total_tokens / (ms_max * 1e-3)
 
-    # end to end through the public API with host buffers (pinned), per-step H2D + D2H
+    # end to end through the public API with host buffers (pinned): every step copies its inputs
+    # host -> device and reads its loss and diagnostics back.  The copy of step i+1's inputs runs on
+    # a second stream while step i computes (two device buffer sets), as a prefetching data loader
+    # would; every copy and read of the K steps lies inside the timed region.
     e2e = None
     if not args.no_e2e:
         host = {k: getattr(b, k).cpu().pin_memory() for k in ("hidden", "targets", "rewards", "resp_offsets",
                                                               "group_offsets")}
         host["logmu"] = logmu.cpu().pin_memory()
-        dbuf = {k: torch.empty_like(v, device=dev) for k, v in host.items()}
+        dbufs = [{k: torch.empty_like(v, device=dev) for k, v in host.items()} for _ in range(2)]
         loss_h = torch.empty(1, dtype=torch.float32).pin_memory()
         d3_h = torch.empty(out.d3_raw.numel(), dtype=torch.uint8).pin_memory()
         h2d = sum(v.numel() * v.element_size() for v in host.values())
         d2h = loss_h.numel() * 4 + d3_h.numel()
+        main_s = torch.cuda.current_stream(dev)
+        copy_s = torch.cuda.Stream(device=dev)
+        copied = [torch.cuda.Event(), torch.cuda.Event()]
+        used = [torch.cuda.Event(), torch.cuda.Event()]
 
-        def e2e_step():
-            for k in host:
-                dbuf[k].copy_(host[k], non_blocking=True)
-            bi.is_loss_fwd_bwd(dbuf["hidden"], b.w, dbuf["targets"], dbuf["logmu"], dbuf["rewards"],
-                               dbuf["resp_offsets"], dbuf["group_offsets"], None, rnorm, ws=ws, out=out)
-            if pg is not None:
-                pg.all_reduce(out.grad_w)
-                pg.all_reduce(out.loss)
-            loss_h.copy_(out.loss, non_blocking=True)
-            d3_h.copy_(out.d3_raw, non_blocking=True)
+        def issue_copy(i, after=None):
+            bufs = dbufs[i % 2]
+            with torch.cuda.stream(copy_s):
+                if after is not None:
+                    copy_s.wait_event(after)
+                copy_s.wait_event(used[i % 2])  # the step that last read these buffers
+                for k in host:
+                    bufs[k].copy_(host[k], non_blocking=True)
+                copied[i % 2].record(copy_s)
 
-        for _ in range(2):
-            e2e_step()
+        def e2e_run(nsteps, start_event=None):
+            issue_copy(0, start_event)
+            for i in range(nsteps):
+                if i + 1 < nsteps:
+                    issue_copy(i + 1)
+                main_s.wait_event(copied[i % 2])
+                d = dbufs[i % 2]
+                bi.is_loss_fwd_bwd(d["hidden"], b.w, d["targets"], d["logmu"], d["rewards"], d["resp_offsets"],
+                                   d["group_offsets"], None, rnorm, ws=ws, out=out)
+                used[i % 2].record(main_s)
+                if pg is not None:
+                    pg.all_reduce(out.grad_w)
+                    pg.all_reduce(out.loss)
+                loss_h.copy_(out.loss, non_blocking=True)
+                d3_h.copy_(out.d3_raw, non_blocking=True)
+
+        e2e_run(2)
         torch.cuda.synchronize()
         f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        f0.record()
-        for _ in range(args.steps):
-            e2e_step()
-        f1.record()
+        f0.record(main_s)
+        e2e_run(args.steps, start_event=f0)
+        f1.record(main_s)
         torch.cuda.synchronize()
         ems = torch.tensor([f0.elapsed_time(f1) / args.steps], dtype=torch.float64, device=dev)
         if pg is not None:
             pg.all_reduce(ems, op=pg.ReduceOp.MAX)
         e2e = {"value": total_tokens / (float(ems.item()) * 1e-3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
-               "d2h_bytes_per_step": int(d2h)}
+               "d2h_bytes_per_step": int(d2h), "h2d": "pinned host buffers, prefetched one step ahead on a copy stream"}
 
     peaks, peak_src = measured_peaks()
     peak_tf = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
     flops_tvh = 2.0 * T * V * H  # one LM-head contraction over the batch
     # algorithmic: logits + dH in the fused forward, dW in the second kernel; executed adds the
     # logit recompute of the dW kernel
-    alg = {"k_lm_fwd": flops_tvh, "k_lm_fwd_dh": 2 * flops_tvh, "k_lm_dw": flops_tvh}
-    executed = {"k_lm_fwd": flops_tvh, "k_lm_fwd_dh": 2 * flops_tvh, "k_lm_dw": 2 * flops_tvh}
+    alg = {"k_lm_fwd": flops_tvh, "k_lm_fwd_dh": 2 * flops_tvh, "k_lm_dw": flops_tvh, "k_dw_stream": flops_tvh}
+    executed = {"k_lm_fwd": flops_tvh, "k_lm_fwd_dh": 2 * flops_tvh, "k_lm_dw": 2 * flops_tvh,
+                "k_dw_stream": flops_tvh}
     dom = max(alg, key=lambda k: prof.get(k, (0.0, 1))[0])
     dms, dn = prof.get(dom, (float("nan"), 1))
     davg = dms / max(dn, 1)
