@@ -11,7 +11,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libbi_islos
 
 EXPORTED = ("bi_workspace_bytes", "bi_workspace_bytes_min", "bi_logprob_fwd", "bi_logprob_fwd_noalloc", "bi_is_loss_fwd_bwd", "bi_d3_stats",
             "bi_status_string", "bi_version", "bi_debug_force_timeout_once", "bi_profile_enable",
-            "bi_profile_reset", "bi_profile_read")
+            "bi_profile_reset", "bi_profile_read", "bi_gemm_bf16", "bi_rmsnorm")
 
 STATUS_NAMES = {0: "BI_OK", 1: "BI_ERR_INVALID_ARG", 2: "BI_ERR_UNSUPPORTED_SHAPE", 3: "BI_ERR_WORKSPACE",
                 4: "BI_ERR_CUDA", 5: "BI_ERR_TIMEOUT", 6: "BI_ERR_BAD_TARGET", 7: "BI_ERR_NONFINITE",
@@ -70,5 +70,9 @@ def load() -> ctypes.CDLL:
     lib.bi_profile_read.argtypes = [ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(ctypes.c_double),
                                     ctypes.POINTER(ctypes.c_int64), _i32]
     lib.bi_profile_read.restype = _i32
+    lib.bi_gemm_bf16.argtypes = [_p, _p, _p, _i64, _i32, _i32, _p, _p]
+    lib.bi_gemm_bf16.restype = ctypes.c_int
+    lib.bi_rmsnorm.argtypes = [_p, _p, ctypes.c_float, _p, _i64, _i32, _p, _p]
+    lib.bi_rmsnorm.restype = ctypes.c_int
     _lib = lib
     return lib

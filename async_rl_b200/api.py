@@ -175,6 +175,43 @@ def decode_d3(raw: torch.Tensor) -> dict:
             "k1": float(k[0]), "k2": float(k[1]), "n_clipped": int(c[0]), "n_rejected": int(c[1])}
 
 
+def gemm_bf16(x: torch.Tensor, w: torch.Tensor, out: Optional[torch.Tensor] = None,
+              status: Optional[torch.Tensor] = None):
+    """Y = X W^T (include/bi_model.h).  Returns (y [M, N] bf16, status [1] i32)."""
+    dev = w.device
+    M, K = x.shape
+    N = w.shape[0]
+    _check_cuda(x, "x", torch.bfloat16, dev)
+    _check_cuda(w, "w", torch.bfloat16, dev)
+    if w.shape[1] != K:
+        raise ValueError(f"x has K = {K} columns, w has {w.shape[1]}")
+    y = out if out is not None else torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    _check_cuda(y, "out", torch.bfloat16, dev)
+    if tuple(y.shape) != (M, N):
+        raise ValueError(f"out must be [{M}, {N}]")
+    st = status if status is not None else torch.empty(1, dtype=torch.int32, device=dev)
+    code = _lib.load().bi_gemm_bf16(_ptr(x), _ptr(w), _ptr(y), M, N, K, _ptr(st), _stream(dev))
+    _raise_host(code, "bi_gemm_bf16")
+    return y, st
+
+
+def rmsnorm(x: torch.Tensor, g: torch.Tensor, eps: float, out: Optional[torch.Tensor] = None,
+            status: Optional[torch.Tensor] = None):
+    """y = x / sqrt(mean(x^2) + eps) * g per row (include/bi_model.h).  Returns (y, status)."""
+    dev = x.device
+    M, H = x.shape
+    _check_cuda(x, "x", torch.bfloat16, dev)
+    _check_cuda(g, "g", torch.bfloat16, dev)
+    if g.shape != (H,):
+        raise ValueError(f"g must be [{H}]")
+    y = out if out is not None else torch.empty(M, H, dtype=torch.bfloat16, device=dev)
+    _check_cuda(y, "out", torch.bfloat16, dev)
+    st = status if status is not None else torch.empty(1, dtype=torch.int32, device=dev)
+    code = _lib.load().bi_rmsnorm(_ptr(x), _ptr(g), float(eps), _ptr(y), M, H, _ptr(st), _stream(dev))
+    _raise_host(code, "bi_rmsnorm")
+    return y, st
+
+
 def debug_force_timeout_once(limit_ns: int) -> None:
     """Test hook: the next logprob_fwd on this thread exercises the bounded-wait timeout path."""
     _lib.load().bi_debug_force_timeout_once(int(limit_ns))

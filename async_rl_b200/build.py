@@ -14,7 +14,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libbi_isloss.so")
 SOURCES = ["bi_api.cu"]
-HEADERS = ["sm100.cuh", "kernels_lm.cuh", "kernels_dw.cuh", "kernels_small.cuh"]
+HEADERS = ["sm100.cuh", "kernels_lm.cuh", "kernels_dw.cuh", "kernels_model.cuh", "kernels_small.cuh"]
 
 
 def nvcc_path() -> str:
@@ -28,7 +28,7 @@ def needs_build() -> bool:
     if not os.path.exists(LIB):
         return True
     t = os.path.getmtime(LIB)
-    deps = [os.path.join(CSRC, f) for f in SOURCES + HEADERS] + [os.path.join(ROOT, "include", "bi_isloss.h")]
+    deps = [os.path.join(CSRC, f) for f in SOURCES + HEADERS] + [os.path.join(ROOT, "include", h) for h in ("bi_isloss.h", "bi_model.h")]
     return any(os.path.getmtime(d) > t for d in deps if os.path.exists(d))
 
 

@@ -1,5 +1,6 @@
-// bi_api.cu -- the C ABI declared in include/bi_isloss.h: argument checks, workspace layout,
-// tensor maps and the fixed launch sequence.  Nothing here allocates device memory.
+// bi_api.cu -- the C ABI declared in include/bi_isloss.h and include/bi_model.h: argument checks,
+// workspace layout, tensor maps and the fixed launch sequences.  Nothing here allocates device
+// memory.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -11,8 +12,10 @@
 #include <vector>
 
 #include "bi_isloss.h"
+#include "bi_model.h"
 #include "kernels_dw.cuh"
 #include "kernels_lm.cuh"
+#include "kernels_model.cuh"
 #include "kernels_small.cuh"
 
 namespace {
@@ -30,10 +33,11 @@ thread_local uint64_t g_force_timeout_ns = 0;
 // optional per-kernel timing (events around each launch; measurement tools only)
 // ---------------------------------------------------------------------------------------------
 enum KernelKind : int { kKPrep, kKRowmap, kKZeroRows, kKGather, kKLmFwd, kKLmFwdDH, kKLmDW, kKDwRows,
-                        kKDwStream, kKSeqGate, kKRowParts, kKReduce, kKD3Partial, kNumKinds };
+                        kKDwStream, kKSeqGate, kKRowParts, kKReduce, kKD3Partial, kKGemm, kKRmsNorm, kNumKinds };
 const char* const kKindNames[kNumKinds] = {"k_prep", "k_rowmap", "k_zero_prompt_rows", "k_gather_rows",
                                            "k_lm_fwd", "k_lm_fwd_dh", "k_lm_dw", "k_dw_rows", "k_dw_stream",
-                                           "k_seq_gate", "k_row_parts", "k_reduce_parts", "k_d3_partial"};
+                                           "k_seq_gate", "k_row_parts", "k_reduce_parts", "k_d3_partial",
+                                           "k_gemm_pair", "k_rmsnorm"};
 static_assert(sizeof(bi::D3Out) == sizeof(bi_d3), "device-written diagnostics match the ABI struct");
 struct Pending {
   int kind;
@@ -212,6 +216,7 @@ struct DevInfo {
   bool ok = false;
   int sms = 0;
   int max_clusters[3][bi::kMaxCluster + 1] = {};  // [mode][C]
+  int gemm_clusters = 0;                            // resident CTA pairs of the GEMM kernel
 };
 std::mutex g_dev_mu;
 std::array<DevInfo, 64> g_dev;
@@ -267,7 +272,26 @@ bool set_lm_attributes() {
                                   dw_smem<HS_>()) == cudaSuccess;
   BI_DW_CONFIGS(BI_SET_DW_ATTR)
 #undef BI_SET_DW_ATTR
+  ok = ok && cudaFuncSetAttribute(bi::k_gemm_pair, cudaFuncAttributeMaxDynamicSharedMemorySize, bi::kGemmSmem) ==
+                 cudaSuccess;
   return ok;
+}
+
+int query_gemm_clusters() {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2, 1, 1);
+  cfg.blockDim = dim3(bi::kGemmThreads, 1, 1);
+  cfg.dynamicSmemBytes = bi::kGemmSmem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, bi::k_gemm_pair, &cfg) != cudaSuccess) return 0;
+  return n;
 }
 
 const DevInfo* device_info() {
@@ -284,6 +308,7 @@ const DevInfo* device_info() {
     d.max_clusters[bi::kModeFwdDH][c] = query_clusters<bi::kModeFwdDH>(c);
     d.max_clusters[bi::kModeDW][c] = query_clusters<bi::kModeDW>(c);
   }
+  d.gemm_clusters = query_gemm_clusters();
   cudaGetLastError();
   d.ok = d.sms > 0 && d.sms <= kMaxSms;
   return d.ok ? &d : nullptr;
@@ -735,6 +760,66 @@ bi_status bi_d3_stats(const float* learner_logprob, const float* rollout_logprob
   ProfScope ps(kKReduce, s);
   bi::k_reduce_parts<<<1, 1024, 0, s>>>(parts, static_cast<int>(nred), nullptr, reinterpret_cast<bi::D3Out*>(out),
                                         nullptr, dev_status);
+  return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+}
+
+bi_status bi_gemm_bf16(const uint16_t* x, const uint16_t* w, uint16_t* y, int64_t M, int32_t N, int32_t K,
+                       int32_t* dev_status, void* stream) {
+  if (!dev_status || !w || (M > 0 && (!x || !y))) return BI_ERR_INVALID_ARG;
+  if (!aligned16(w) || (M > 0 && (!aligned16(x) || !aligned16(y)))) return BI_ERR_INVALID_ARG;
+  // tile row coordinates (M rounded up to 256) must stay inside int32
+  if (M < 0 || M > (int64_t{1} << 31) - 256) return BI_ERR_INVALID_ARG;
+  if (N <= 0 || N % 8 != 0 || K <= 0 || K % 8 != 0) return BI_ERR_UNSUPPORTED_SHAPE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s) != cudaSuccess) return BI_ERR_CUDA;
+  if (M == 0) return BI_OK;
+  const DevInfo* di = device_info();
+  if (!di || di->gemm_clusters <= 0) return BI_ERR_CUDA;
+  CUtensorMap tm_x, tm_w;
+  if (!make_map(&tm_x, x, M, K, 128) || !make_map(&tm_w, w, N, K, 128)) return BI_ERR_CUDA;
+  bi::GemmArgs a{};
+  a.y = y;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.status = dev_status;
+  a.limit_ns = kWaitLimitNs;
+  const int64_t tiles = ((M + bi::kGemmTileM - 1) / bi::kGemmTileM) * ((N + bi::kGemmTileN - 1) / bi::kGemmTileN);
+  const int64_t ncl = tiles < di->gemm_clusters ? tiles : di->gemm_clusters;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * ncl), 1, 1);
+  cfg.blockDim = dim3(bi::kGemmThreads, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(bi::kGemmSmem);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  ProfScope ps(kKGemm, s);
+  return cudaLaunchKernelEx(&cfg, bi::k_gemm_pair, tm_x, tm_w, a) == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+}
+
+bi_status bi_rmsnorm(const uint16_t* x, const uint16_t* g, float eps, uint16_t* y, int64_t M, int32_t H,
+                     int32_t* dev_status, void* stream) {
+  if (!dev_status || !g || (M > 0 && (!x || !y))) return BI_ERR_INVALID_ARG;
+  if (!aligned16(g) || (M > 0 && (!aligned16(x) || !aligned16(y)))) return BI_ERR_INVALID_ARG;
+  if (M < 0 || !(eps >= 0.f) || !std::isfinite(eps)) return BI_ERR_INVALID_ARG;
+  if (H <= 0 || H % 8 != 0) return BI_ERR_UNSUPPORTED_SHAPE;
+  if (M > 0 && static_cast<const void*>(x) == static_cast<const void*>(y)) return BI_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s) != cudaSuccess) return BI_ERR_CUDA;
+  if (M == 0) return BI_OK;
+  const DevInfo* di = device_info();
+  if (!di) return BI_ERR_CUDA;
+  // a warp per row, 8 rows per block; at most 8 blocks per SM, rows strided over the grid
+  const int64_t want = (M + bi::kNormThreads / 32 - 1) / (bi::kNormThreads / 32);
+  const int64_t cap = static_cast<int64_t>(di->sms) * 8;
+  const unsigned blocks = static_cast<unsigned>(want < cap ? want : cap);
+  ProfScope ps(kKRmsNorm, s);
+  bi::k_rmsnorm<<<blocks, bi::kNormThreads, 0, s>>>(x, g, eps, y, M, H);
   return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
 }
 

@@ -10,7 +10,8 @@ from async_rl_b200 import _lib
 from async_rl_b200.build import build
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADER = os.path.join(ROOT, "include", "bi_isloss.h")
+HEADERS = [os.path.join(ROOT, "include", h) for h in sorted(os.listdir(os.path.join(ROOT, "include")))
+           if h.endswith(".h")]
 
 
 @pytest.fixture(scope="module")
@@ -20,14 +21,17 @@ def lib():
 
 
 def declared_functions():
-    text = open(HEADER).read()
-    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(bi_[a-z0-9_]+)\s*\(", text)))
+    names = set()
+    for h in HEADERS:
+        text = re.sub(r"/\*.*?\*/", "", open(h).read(), flags=re.S)
+        names |= set(re.findall(r"\b(bi_[a-z0-9_]+)\s*\(", text))
+    return sorted(names)
 
 
 def test_header_declares_the_boundary():
     names = declared_functions()
-    for must in ("bi_logprob_fwd", "bi_is_loss_fwd_bwd", "bi_d3_stats", "bi_workspace_bytes", "bi_status_string"):
+    for must in ("bi_logprob_fwd", "bi_is_loss_fwd_bwd", "bi_d3_stats", "bi_workspace_bytes", "bi_status_string",
+                 "bi_gemm_bf16", "bi_rmsnorm"):
         assert must in names
 
 
@@ -123,3 +127,34 @@ def test_d3_argument_checks(lib):
     assert lib.bi_d3_stats(None, FAKE, None, 10, FAKE, FAKE, FAKE, 256, None) == 1
     assert lib.bi_d3_stats(FAKE, FAKE, None, 10, None, FAKE, FAKE, 256, None) == 1
     assert lib.bi_d3_stats(FAKE, FAKE, None, 1000, FAKE, FAKE, FAKE, 16, None) == 3
+
+
+def test_gemm_argument_checks(lib):
+    """Host checks of bi_gemm_bf16 (include/bi_model.h) return before any CUDA call."""
+    p = ctypes.c_void_p(4096)      # 16-byte aligned stand-in pointers, never dereferenced
+    odd = ctypes.c_void_p(4104)
+    st = ctypes.c_void_p(8192)
+    f = lib.bi_gemm_bf16
+    assert f(p, p, p, 16, 256, 64, None, None) == 1            # no status pointer
+    assert f(None, p, p, 16, 256, 64, st, None) == 1           # no input
+    assert f(p, odd, p, 16, 256, 64, st, None) == 1            # misaligned weight
+    assert f(p, p, p, -1, 256, 64, st, None) == 1              # negative M
+    assert f(p, p, p, 16, 250, 64, st, None) == 2              # N not a multiple of 8
+    assert f(p, p, p, 16, 256, 60, st, None) == 2              # K not a multiple of 8
+    assert f(p, p, p, 16, 0, 64, st, None) == 2
+    assert f(p, p, p, 16, 256, 0, st, None) == 2
+
+
+def test_rmsnorm_argument_checks(lib):
+    p = ctypes.c_void_p(4096)
+    q = ctypes.c_void_p(1 << 20)
+    odd = ctypes.c_void_p(4100)
+    st = ctypes.c_void_p(8192)
+    f = lib.bi_rmsnorm
+    assert f(p, p, 1e-6, q, 4, 64, None, None) == 1            # no status pointer
+    assert f(p, None, 1e-6, q, 4, 64, st, None) == 1           # no gain
+    assert f(odd, p, 1e-6, q, 4, 64, st, None) == 1            # misaligned input
+    assert f(p, p, -1.0, q, 4, 64, st, None) == 1              # negative eps
+    assert f(p, p, float("nan"), q, 4, 64, st, None) == 1
+    assert f(p, p, 1e-6, p, 4, 64, st, None) == 1              # output aliases input
+    assert f(p, p, 1e-6, q, 4, 60, st, None) == 2              # H not a multiple of 8

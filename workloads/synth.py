@@ -176,3 +176,21 @@ def random_inputs(T: int, H: int, V: int, seed: int, w_std: float = 0.02, device
     w = _randn_bf16(gen, (V, H), w_std, device)
     targets = torch.randint(0, V, (T,), generator=gen, device=device, dtype=torch.int64).to(torch.int32)
     return hidden, w, targets
+
+
+def dense_inputs(M: int, K: int, N: int, seed: int, w_std: float = 0.02, device="cpu"):
+    """(x [M, K], w [N, K]) for the linear-layer GEMM: x ~ N(0, 1), W ~ N(0, w_std), both bf16."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    return _randn_bf16(gen, (M, K), 1.0, device), _randn_bf16(gen, (N, K), w_std, device)
+
+
+def norm_inputs(M: int, H: int, seed: int, device="cpu"):
+    """(x [M, H], g [H]) for RMSNorm: rows x ~ N(0, s_m^2) with a per-row scale s_m ~ U[0.05, 20]
+    (hidden states of very different magnitudes), gains g ~ 1 + N(0, 0.1), both bf16."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    x = torch.randn((M, H), generator=gen, device=device)
+    x.mul_(torch.rand((M, 1), generator=gen, device=device) * 19.95 + 0.05)
+    g = 1.0 + 0.1 * torch.randn((H,), generator=gen, device=device)
+    return x.to(torch.bfloat16), g.to(torch.bfloat16)
