@@ -7,10 +7,14 @@ forward logits + log-softmax + target gather, IS weight, D3, advantages, loss, d
 Inputs (hidden 0.2 GB, W 0.47 GB) are larger than the 126 MB L2, so no flush is needed between
 steps.  Prints one JSON line (rank 0).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload loss|dense]
 
 N > 1 runs one process per GPU (torchrun): each rank scores its own batch (weak scaling) and the
 ranks sum dW and the three loss/D3 scalars with NCCL, the one exchange step of data parallelism.
+
+--workload dense times the batch-invariant dense layers instead (not the default line): one step is
+RMSNorm of the 1.5B-shape hidden states [76239, 1536] followed by the gate/up projection
+Y = X W^T with W [8960, 1536] (bi_rmsnorm + bi_gemm_bf16); ranks are independent replicas.
 """
 from __future__ import annotations
 
@@ -45,6 +49,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--small", action="store_true",
                     help="profiling case: same head, 4 responses of 1024 rows (T=4096); not a bench line")
+    ap.add_argument("--workload", choices=["loss", "dense"], default="loss",
+                    help="loss: the fused LM-head step (default line); dense: RMSNorm + linear layer")
     return ap.parse_args()
 
 
@@ -380,9 +386,184 @@ def run_ours(args):
         pg.destroy_process_group()
 
 
+DENSE_M, DENSE_K, DENSE_N = 76239, 1536, 8960  # 1.5B shape: tokens, hidden size, MLP width
+DENSE_METRIC = "batch-invariant RMSNorm + bf16 GEMM (gate/up) TFLOP/s at M76239 K1536 N8960"
+DENSE_CPU_ROWS = 32768
+
+
+def run_dense_reference(args):
+    """--impl reference --workload dense: the fp64 oracle on the machine's host cores, a bounded slice
+    of rows per step (rank 0 only)."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    from workloads import dense_inputs, norm_inputs
+    M, K, N = DENSE_M, DENSE_K, DENSE_N
+    rows = 4096
+    x, g = norm_inputs(rows, K, seed=1234)
+    _, w = dense_inputs(8, K, N, seed=4321)
+    times, cores = [], 1
+    for i in range(args.warmup + args.steps):
+        dt, cores = dense_cpu_sample(x, g, w, rows)
+        if i >= args.warmup:
+            times.append(dt)
+    ms = 1e3 * statistics.mean(times)
+    val = 2.0 * rows * N * K / (ms * 1e-3) / 1e12
+    print(json.dumps({"impl": "reference", "metric": DENSE_METRIC, "value": val, "unit": "TFLOP/s",
+                      "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+                      "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                      "data": "synthetic",
+                      "config": {"workload": f"dense: RMSNorm + GEMM, {rows}-row slice of [{M}, {K}] x [{N}, {K}]^T "
+                                             "per step on host cores"},
+                      "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                                       "sample": f"{rows} rows per step"},
+                      "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),
+          flush=True)
+
+
+def dense_cpu_sample(x, g, w, rows):
+    """The fp64 oracle (test infrastructure) on the first `rows` rows of the dense step."""
+    from oracle import model_oracle as mo
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max((d.get("num_threads", 1) for d in threadpool_info()), default=os.cpu_count())
+    except Exception:  # pragma: no cover
+        cores = os.cpu_count()
+    xs, gs, ws = x[:rows].cpu(), g.cpu(), w.cpu()
+    t0 = time.perf_counter()
+    for r0 in range(0, rows, 8192):  # row chunks keep the fp64 output small
+        h = mo.rmsnorm(xs[r0:r0 + 8192], gs, 1e-6)
+        mo.gemm(torch.tensor(h, dtype=torch.float32).to(torch.bfloat16), ws)
+    dt = time.perf_counter() - t0
+    return dt, int(cores)
+
+
+def run_dense(args):
+    """--workload dense: RMSNorm then the gate/up GEMM on one synthetic batch per step."""
+    rank, world, local = dist_env()
+    import async_rl_b200 as bi
+    from async_rl_b200.build import build
+    from workloads import dense_inputs, norm_inputs
+
+    if rank == 0:
+        build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        dist.barrier()
+        pg = dist
+    M, K, N = DENSE_M, DENSE_K, DENSE_N
+    x, g = norm_inputs(M, K, seed=1234 + 1000 * rank)
+    _, w = dense_inputs(8, K, N, seed=4321)
+    xd, gd, wd = x.to(dev), g.to(dev), w.to(dev)
+    h = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+    y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    st = torch.empty(1, dtype=torch.int32, device=dev)
+
+    def step(src):
+        bi.rmsnorm(src, gd, 1e-6, out=h, status=st)
+        bi.gemm_bf16(h, wd, out=y, status=st)
+
+    for _ in range(args.warmup):
+        step(xd)
+    torch.cuda.synchronize()
+    bi.check_status(st)
+    clocks = ClockSampler(local)
+    if pg is not None:
+        pg.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    bi.profile_reset()
+    bi.profile_enable(True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        step(xd)
+    e1.record()
+    torch.cuda.synchronize()
+    bi.profile_enable(False)
+    clk = clocks.stop()
+    ms = torch.tensor([e0.elapsed_time(e1) / args.steps], dtype=torch.float64, device=dev)
+    if pg is not None:
+        pg.all_reduce(ms, op=pg.ReduceOp.MAX)
+    ms = float(ms.item())
+    prof = bi.profile_read()
+    flops = 2.0 * M * N * K
+    value = world * flops / (ms * 1e-3) / 1e12
+
+    # end to end: x copied in from pinned host memory and all of y read back, every step
+    xh = x.pin_memory()
+    yh = torch.empty(M, N, dtype=torch.bfloat16).pin_memory()
+    xin = torch.empty_like(xd)
+
+    def e2e_step():
+        xin.copy_(xh, non_blocking=True)
+        step(xin)
+        yh.copy_(y, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record()
+    for _ in range(args.steps):
+        e2e_step()
+    f1.record()
+    torch.cuda.synchronize()
+    ems = torch.tensor([f0.elapsed_time(f1) / args.steps], dtype=torch.float64, device=dev)
+    if pg is not None:
+        pg.all_reduce(ems, op=pg.ReduceOp.MAX)
+    e2e = {"value": world * flops / (float(ems.item()) * 1e-3) / 1e12, "unit": "TFLOP/s",
+           "h2d_bytes_per_step": int(x.numel() * 2), "d2h_bytes_per_step": int(y.numel() * 2),
+           "h2d": "pinned host buffers, copies in series with the step (x in, all of y out)"}
+
+    peaks, peak_src = measured_peaks()
+    peak_tf = float(peaks.get("bf16_tflops"))
+    peak_gb = float(peaks.get("hbm_gbs"))
+    gms, gn = prof.get("k_gemm_pair", (float("nan"), 1))
+    nms, nn = prof.get("k_rmsnorm", (float("nan"), 1))
+    g_tf = flops / (gms / max(gn, 1) * 1e-3) / 1e12
+    n_gb = 2.0 * 2 * M * K / (nms / max(nn, 1) * 1e-3) / 1e9
+    line = {"metric": DENSE_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"dense: RMSNorm [{M}, {K}] then Y = X W^T, W [{N}, {K}] (1.5B shape gate/up)",
+                       "parallelism": f"replicas{world}",
+                       "l2": "inputs larger than L2 (x 0.23 GB, y 1.37 GB); no flush"},
+            "roofline": {"bound": "tensor", "kernel": "k_gemm_pair", "achieved": g_tf, "peak": peak_tf,
+                         "unit": "TFLOP/s", "frac": g_tf / peak_tf, "traffic": None,
+                         "peak_source": f"{peak_src} bf16_tflops (burst: short kernel timed alone)",
+                         "algorithmic_flops_per_launch": flops},
+            "rmsnorm_roofline": {"bound": "hbm", "kernel": "k_rmsnorm", "achieved": n_gb, "peak": peak_gb,
+                                 "unit": "GB/s", "frac": n_gb / peak_gb,
+                                 "algorithmic_bytes_per_launch": 2.0 * 2 * M * K},
+            "kernels": {k: {"ms_per_launch": v[0] / max(v[1], 1), "launches": v[1]} for k, v in prof.items()},
+            "gpu_launches": int(sum(v[1] for v in prof.values())), "clocks": clk, "e2e": e2e}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rows = DENSE_CPU_ROWS
+        dt, cores = dense_cpu_sample(x, g, w, rows)
+        line["cpu_baseline"] = {"value": 2.0 * rows * N * K / dt / 1e12, "unit": "TFLOP/s", "cores": cores,
+                                "kind": "oracle",
+                                "sample": f"first {rows} rows of the dense step (fp64 NumPy RMSNorm + GEMM), {dt:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.barrier()
+        pg.destroy_process_group()
+
+
 def main():
     args = parse()
-    if args.impl == "reference":
+    if args.workload == "dense":
+        if args.impl == "reference":
+            run_dense_reference(args)
+        else:
+            run_dense(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

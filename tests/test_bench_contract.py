@@ -42,3 +42,21 @@ def test_cuda_arm_line_small_case():
         assert k in roof, k
     assert 0 < roof["frac"] < 2
     assert line["e2e"]["value"] > 0 and line["e2e"]["h2d_bytes_per_step"] > 0
+
+
+@pytest.mark.slow
+def test_dense_reference_arm_line():
+    line = _run(["--impl", "reference", "--workload", "dense", "--steps", "1", "--warmup", "0"], timeout=600)
+    for k in REQUIRED:
+        assert k in line, k
+    assert line["impl"] == "reference" and line["unit"] == "TFLOP/s" and line["value"] > 0
+
+
+@pytest.mark.gpu
+def test_dense_workload_line():
+    line = _run(["--workload", "dense", "--steps", "3", "--warmup", "3", "--no-cpu-baseline"], timeout=900)
+    for k in REQUIRED + ("roofline", "rmsnorm_roofline", "clocks", "gpu_launches"):
+        assert k in line, k
+    assert line["gpu_launches"] == 6 and line["value"] > 0
+    assert 0 < line["roofline"]["frac"] < 2 and 0 < line["rmsnorm_roofline"]["frac"] < 2
+    assert line["e2e"]["d2h_bytes_per_step"] == 76239 * 8960 * 2
