@@ -278,6 +278,71 @@ __device__ __forceinline__ uint4 ldg_nc_u4(const void* p) {
   return r;
 }
 
+// Rows of at most 256 kVec elements: the row stays in registers (one read of x), and the next
+// row's vectors are requested before the current row is reduced.  Same per-lane order and shuffle
+// tree as the general kernel below.
+constexpr int kNormRegMaxVec = 8;  // rows of up to 2048 elements stay in registers
+template <int kVec>
+__global__ void __launch_bounds__(kNormThreads, 2)
+    k_rmsnorm_reg(const uint16_t* __restrict__ x, const uint16_t* __restrict__ g, float eps,
+                  uint16_t* __restrict__ y, int64_t M, int32_t H) {
+  const int lane = threadIdx.x & 31;
+  const int64_t w0 = (static_cast<int64_t>(blockIdx.x) * kNormThreads + threadIdx.x) >> 5;
+  const int64_t nw = (static_cast<int64_t>(gridDim.x) * kNormThreads) >> 5;
+  const int nvec = H / 8;
+  const float inv_h = 1.0f / static_cast<float>(H);
+  uint4 cur[kVec];
+  auto load_row = [&](int64_t r, uint4 (&q)[kVec]) {
+#pragma unroll
+    for (int i = 0; i < kVec; ++i) {
+      const int v = lane + 32 * i;
+      q[i] = (r < M && v < nvec) ? ldg_nc_u4(x + r * H + 8 * v) : make_uint4(0u, 0u, 0u, 0u);
+    }
+  };
+  load_row(w0, cur);
+  for (int64_t r = w0; r < M; r += nw) {
+    uint4 nxt[kVec];
+    load_row(r + nw, nxt);
+    float ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < kVec; ++i) {
+      const uint32_t u[4] = {cur[i].x, cur[i].y, cur[i].z, cur[i].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float lo = __uint_as_float(u[e] << 16);
+        const float hi = __uint_as_float(u[e] & 0xffff0000u);
+        ss = fmaf(lo, lo, ss);
+        ss = fmaf(hi, hi, ss);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    ss = __shfl_sync(0xffffffffu, ss, 0);
+    const float rs = rsqrtf(ss * inv_h + eps);
+    uint16_t* yr = y + r * H;
+#pragma unroll
+    for (int i = 0; i < kVec; ++i) {
+      const int v = lane + 32 * i;
+      if (v < nvec) {
+        const uint4 gq = ldg_nc_u4(g + 8 * v);
+        const uint32_t u[4] = {cur[i].x, cur[i].y, cur[i].z, cur[i].w};
+        const uint32_t gw[4] = {gq.x, gq.y, gq.z, gq.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float lo = (__uint_as_float(u[e] << 16) * rs) * __uint_as_float(gw[e] << 16);
+          const float hi = (__uint_as_float(u[e] & 0xffff0000u) * rs) * __uint_as_float(gw[e] & 0xffff0000u);
+          o[e] = pack_bf16x2(lo, hi);
+        }
+        *reinterpret_cast<uint4*>(yr + 8 * v) = make_uint4(o[0], o[1], o[2], o[3]);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kVec; ++i) cur[i] = nxt[i];
+  }
+}
+
+// Any H (a multiple of 8): two passes over the row, the second from L1/L2.
 __global__ void __launch_bounds__(kNormThreads)
     k_rmsnorm(const uint16_t* __restrict__ x, const uint16_t* __restrict__ g, float eps, uint16_t* __restrict__ y,
               int64_t M, int32_t H) {
