@@ -155,6 +155,12 @@ __global__ void k_gather_rows(const uint16_t* __restrict__ hidden, int64_t T, in
   }
 }
 
+// Maximum that keeps a NaN operand (fmaxf would drop it): a NaN D3 term makes the max NaN, as it
+// makes the mean NaN.
+__device__ __forceinline__ float max_keep_nan(float a, float b) {
+  return isnan(a) ? a : (isnan(b) ? b : fmaxf(a, b));
+}
+
 // Fixed-shape block reduction of a RedPart (warp butterflies, then warps in order).
 __device__ __forceinline__ RedPart block_reduce(RedPart v) {
   for (int o = 16; o > 0; o >>= 1) {
@@ -162,7 +168,7 @@ __device__ __forceinline__ RedPart block_reduce(RedPart v) {
     v.d3sum += __shfl_xor_sync(0xffffffffu, v.d3sum, o);
     v.k1sum += __shfl_xor_sync(0xffffffffu, v.k1sum, o);
     v.k2sum += __shfl_xor_sync(0xffffffffu, v.k2sum, o);
-    v.d3max = fmaxf(v.d3max, __shfl_xor_sync(0xffffffffu, v.d3max, o));
+    v.d3max = max_keep_nan(v.d3max, __shfl_xor_sync(0xffffffffu, v.d3max, o));
     v.count += __shfl_xor_sync(0xffffffffu, v.count, o);
     v.nonfinite += __shfl_xor_sync(0xffffffffu, v.nonfinite, o);
     v.nclip += __shfl_xor_sync(0xffffffffu, v.nclip, o);
@@ -178,7 +184,7 @@ __device__ __forceinline__ RedPart block_reduce(RedPart v) {
       out.d3sum += wp[i].d3sum;
       out.k1sum += wp[i].k1sum;
       out.k2sum += wp[i].k2sum;
-      out.d3max = fmaxf(out.d3max, wp[i].d3max);
+      out.d3max = max_keep_nan(out.d3max, wp[i].d3max);
       out.count += wp[i].count;
       out.nonfinite += wp[i].nonfinite;
       out.nclip += wp[i].nclip;
@@ -290,7 +296,7 @@ __global__ void k_reduce_parts(const RedPart* __restrict__ parts, int nparts, fl
     v.d3sum += p.d3sum;
     v.k1sum += p.k1sum;
     v.k2sum += p.k2sum;
-    v.d3max = fmaxf(v.d3max, p.d3max);
+    v.d3max = max_keep_nan(v.d3max, p.d3max);
     v.count += p.count;
     v.nonfinite += p.nonfinite;
     v.nclip += p.nclip;

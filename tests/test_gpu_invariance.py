@@ -151,7 +151,9 @@ def test_nonfinite_rollout_logprob_is_reported(cuda_device):
     out = bi.is_loss_fwd_bwd(b.hidden, b.w, b.targets, mu, b.rewards, b.resp_offsets, b.group_offsets)
     torch.cuda.synchronize()
     assert int(out.status.item()) == 7
-    assert out.d3()["n_nonfinite"] == 1
+    d3 = out.d3()
+    assert d3["n_nonfinite"] == 1
+    assert not np.isfinite(d3["mean"]) and not np.isfinite(d3["max"])  # the NaN term is kept in both
     assert torch.isinf(out.is_weight[4])
 
 

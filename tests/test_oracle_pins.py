@@ -144,7 +144,7 @@ def test_weights_are_not_clipped():
 
 def test_nonfinite_rollout_logprob_propagates():
     st = orc.d3_stats(np.array([-1.0, -2.0]), np.array([-np.inf, -2.0]))
-    assert st["n_nonfinite"] == 1 and not np.isfinite(st["mean"])
+    assert st["n_nonfinite"] == 1 and not np.isfinite(st["mean"]) and np.isnan(st["max"])
 
 
 # --- advantages, coefficients, loss ---------------------------------------------
