@@ -14,7 +14,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libbi_isloss.so")
 SOURCES = ["bi_api.cu"]
-HEADERS = ["sm100.cuh", "kernels_lm.cuh", "kernels_dw.cuh", "kernels_model.cuh", "kernels_small.cuh"]
+HEADERS = ["sm100.cuh", "kernels_lm.cuh", "kernels_decode.cuh", "kernels_dw.cuh", "kernels_model.cuh",
+           "kernels_small.cuh"]
 
 
 def nvcc_path() -> str:

@@ -13,6 +13,7 @@
 
 #include "bi_isloss.h"
 #include "bi_model.h"
+#include "kernels_decode.cuh"
 #include "kernels_dw.cuh"
 #include "kernels_lm.cuh"
 #include "kernels_model.cuh"
@@ -24,6 +25,7 @@ using bi::Ctrl;
 using bi::RedPart;
 
 constexpr uint64_t kWaitLimitNs = 4000000000ull;  // 4 s for any single in-kernel wait
+constexpr size_t kZscanSmemMax = 160 * 1024;      // per-row scan of decode-style scoring
 constexpr int kMaxSms = 160;                      // upper bound used to size the dZ scratch
 constexpr int kDzSlotsMax = 2 * kMaxSms;          // clusters * C * slots-per-CTA <= 2 * SMs
 
@@ -33,11 +35,11 @@ thread_local uint64_t g_force_timeout_ns = 0;
 // optional per-kernel timing (events around each launch; measurement tools only)
 // ---------------------------------------------------------------------------------------------
 enum KernelKind : int { kKPrep, kKRowmap, kKZeroRows, kKGather, kKLmFwd, kKLmFwdDH, kKLmDW, kKDwRows,
-                        kKDwStream, kKSeqGate, kKRowParts, kKReduce, kKD3Partial, kKGemm, kKRmsNorm, kNumKinds };
+                        kKDwStream, kKSeqGate, kKRowParts, kKReduce, kKD3Partial, kKGemm, kKRmsNorm, kKLmZtiles, kKLmZscan, kNumKinds };
 const char* const kKindNames[kNumKinds] = {"k_prep", "k_rowmap", "k_zero_prompt_rows", "k_gather_rows",
                                            "k_lm_fwd", "k_lm_fwd_dh", "k_lm_dw", "k_dw_rows", "k_dw_stream",
                                            "k_seq_gate", "k_row_parts", "k_reduce_parts", "k_d3_partial",
-                                           "k_gemm_pair", "k_rmsnorm"};
+                                           "k_gemm_pair", "k_rmsnorm", "k_lm_ztiles", "k_lm_zscan"};
 static_assert(sizeof(bi::D3Out) == sizeof(bi_d3), "device-written diagnostics match the ABI struct");
 struct Pending {
   int kind;
@@ -90,6 +92,8 @@ struct WsLayout {
   size_t ctrl, lse_c, g_c, tl_c, d3_c, delta_c, clip_c, y_c, logmu_c, rowmap, respof, coef, cprefix, red, hc, dz,
       alpha, fin;
   size_t sxr_c, mhist, hs, pbuf;  // the P store (loss layout with the store only)
+  size_t zbuf, zmax;              // decode-style scoring (logprob layout, T <= 128 rows)
+  bool decode;
   size_t total;
   int nred;
   int64_t tpad, pcols;        // rows and columns the P store is sized for
@@ -101,7 +105,9 @@ constexpr size_t kFinBytes = static_cast<size_t>(kMaxSms) * 2 * 384 * sizeof(flo
 // `store`, followed by the P store of the fused forward ([Tpad][V + 256] bf16, enough for any
 // logit-tile width NZ <= 256), the per-step reference history ([ceil(V / 128)][Tpad] float) and
 // the scaled hidden states of the dW GEMM ([Tpad][H] bf16).
-WsLayout ws_layout(int64_t T, int32_t H, int32_t V, int32_t R, bool store) {
+// R == 0 with `decode` and 0 < T <= 128: followed by the logits of the few rows ([T][V + 256]
+// fp32) and their per-tile maxima ([T][ceil(V / 128)] fp32) for the all-SM scoring path.
+WsLayout ws_layout(int64_t T, int32_t H, int32_t V, int32_t R, bool store, bool decode = false) {
   WsLayout L{};
   const size_t t = static_cast<size_t>(T > 0 ? T : 1);
   size_t o = 0;
@@ -142,6 +148,11 @@ WsLayout ws_layout(int64_t T, int32_t H, int32_t V, int32_t R, bool store) {
       L.mhist = take(static_cast<size_t>((V + 127) / 128) * static_cast<size_t>(L.tpad) * 4);
       L.pbuf = take(static_cast<size_t>(L.tpad) * static_cast<size_t>(L.pcols) * 2);
     }
+  }
+  if (R == 0 && decode && T > 0 && T <= bi::kDecodeRows) {
+    L.decode = true;
+    L.zbuf = take(t * (static_cast<size_t>(V) + 256) * 4);
+    L.zmax = take(t * static_cast<size_t>((V + 127) / 128) * 4);
   }
   L.total = o;
   return L;
@@ -274,6 +285,18 @@ bool set_lm_attributes() {
 #undef BI_SET_DW_ATTR
   ok = ok && cudaFuncSetAttribute(bi::k_gemm_pair, cudaFuncAttributeMaxDynamicSharedMemorySize, bi::kGemmSmem) ==
                  cudaSuccess;
+  ok = ok && cudaFuncSetAttribute(bi::k_lm_ztiles<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  bi::ZtTile<256>::smem) == cudaSuccess;
+  ok = ok && cudaFuncSetAttribute(bi::k_lm_ztiles<192>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  bi::ZtTile<192>::smem) == cudaSuccess;
+  ok = ok && cudaFuncSetAttribute(bi::k_lm_ztiles<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  bi::ZtTile<128>::smem) == cudaSuccess;
+  ok = ok && cudaFuncSetAttribute(bi::k_lm_zscan<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(kZscanSmemMax)) == cudaSuccess;
+  ok = ok && cudaFuncSetAttribute(bi::k_lm_zscan<192>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(kZscanSmemMax)) == cudaSuccess;
+  ok = ok && cudaFuncSetAttribute(bi::k_lm_zscan<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(kZscanSmemMax)) == cudaSuccess;
   return ok;
 }
 
@@ -417,6 +440,53 @@ bi_status logprob_forward(const uint16_t* hidden, const uint16_t* w_lm, const in
   return st;
 }
 
+// Decode-style scoring (T <= 128 rows) on every SM: the logit tiles of the rows with the cluster
+// kernel's instruction sequence, then the chain, the class sums and the combine of its epilogue,
+// expression for expression (kernels_decode.cuh).  The same plan (C, NZ) as the cluster kernel,
+// so the same bits.  Returns kDecodeUnsupported when the shape needs the cluster kernel.
+constexpr int kDecodeUnsupported = -1;
+
+int logprob_decode(const uint16_t* hidden, const uint16_t* w_lm, const int32_t* targets, int64_t T, int32_t H,
+                   int32_t V, float* logprob, float* lse, int32_t* dev_status, float* zbuf, float* zmax,
+                   const DevInfo* di, cudaStream_t s) {
+  const LmPlan pl = plan_lm(H, di);
+  if (pl.C == 0 || pl.C > 8) return kDecodeUnsupported;
+  const int nvz = (V + pl.NZ - 1) / pl.NZ;
+  const size_t zsm = bi::zscan_smem(nvz, pl.NZ);
+  if (zsm > kZscanSmemMax) return kDecodeUnsupported;
+  CUtensorMap tm_h, tm_w;
+  if (!make_map(&tm_h, hidden, T, H, 128) || !make_map(&tm_w, w_lm, V, H, pl.NZ)) return BI_ERR_CUDA;
+  bi::ZtArgs a{};
+  a.T = T;
+  a.V = V;
+  a.nvz = nvz;
+  a.KB = H / 64;
+  a.z = zbuf;
+  a.z_ld = static_cast<int64_t>(nvz) * pl.NZ;
+  a.tmax = zmax;
+  a.status = dev_status;
+  a.limit_ns = kWaitLimitNs;
+  const unsigned grid = static_cast<unsigned>(nvz < di->sms ? nvz : di->sms);
+  {
+    ProfScope ps(kKLmZtiles, s);
+    switch (pl.NZ) {
+      case 256: bi::k_lm_ztiles<256><<<grid, bi::kZtThreads, bi::ZtTile<256>::smem, s>>>(tm_h, tm_w, a); break;
+      case 192: bi::k_lm_ztiles<192><<<grid, bi::kZtThreads, bi::ZtTile<192>::smem, s>>>(tm_h, tm_w, a); break;
+      case 128: bi::k_lm_ztiles<128><<<grid, bi::kZtThreads, bi::ZtTile<128>::smem, s>>>(tm_h, tm_w, a); break;
+      default: return kDecodeUnsupported;
+    }
+    if (cudaGetLastError() != cudaSuccess) return BI_ERR_CUDA;
+  }
+  ProfScope ps(kKLmZscan, s);
+  const unsigned rows = static_cast<unsigned>(T);
+  switch (pl.NZ) {
+    case 256: bi::k_lm_zscan<256><<<rows, bi::kZsThreads, zsm, s>>>(zbuf, a.z_ld, zmax, targets, T, V, nvz, pl.C, logprob, lse, dev_status); break;
+    case 192: bi::k_lm_zscan<192><<<rows, bi::kZsThreads, zsm, s>>>(zbuf, a.z_ld, zmax, targets, T, V, nvz, pl.C, logprob, lse, dev_status); break;
+    default:  bi::k_lm_zscan<128><<<rows, bi::kZsThreads, zsm, s>>>(zbuf, a.z_ld, zmax, targets, T, V, nvz, pl.C, logprob, lse, dev_status); break;
+  }
+  return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+}
+
 }  // namespace
 
 namespace {
@@ -506,7 +576,7 @@ int32_t bi_profile_read(const char** names_out, double* ms_out, int64_t* launche
 
 size_t bi_workspace_bytes(int64_t T, int32_t H, int32_t V, int32_t R) {
   if (T < 0 || H <= 0 || V <= 0 || R < 0) return 0;
-  return ws_layout(T, H, V, R, R > 0).total;
+  return ws_layout(T, H, V, R, R > 0, true).total;
 }
 
 size_t bi_workspace_bytes_min(int64_t T, int32_t H, int32_t V, int32_t R) {
@@ -530,6 +600,14 @@ bi_status bi_logprob_fwd(const uint16_t* hidden, const uint16_t* w_lm, const int
   if (!di) return BI_ERR_CUDA;
   if (cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s) != cudaSuccess) return BI_ERR_CUDA;
   if (T == 0) return BI_OK;
+  // a few rows: the same bits from every SM when the workspace holds their logits
+  const WsLayout Ld = ws_layout(T, H, V, 0, false, true);
+  if (Ld.decode && ws_bytes >= Ld.total && force == 0) {
+    uint8_t* w8 = static_cast<uint8_t*>(ws);
+    const int r = logprob_decode(hidden, w_lm, targets, T, H, V, logprob, lse, dev_status,
+                                 reinterpret_cast<float*>(w8 + Ld.zbuf), reinterpret_cast<float*>(w8 + Ld.zmax), di, s);
+    if (r != kDecodeUnsupported) return static_cast<bi_status>(r);
+  }
   float* fin = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + L.fin);
   return logprob_forward(hidden, w_lm, targets, T, H, V, logprob, lse, dev_status, fin, force, di, s);
 }

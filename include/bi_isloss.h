@@ -121,14 +121,18 @@ typedef struct {
  * For bi_is_loss_fwd_bwd this is the workspace of the fastest path: besides O(T) per-row arrays
  * it holds every bf16 probability tile of the forward (about 2 T (V + 384) bytes, 23 GB for
  * T = 76,000 rows of a 151,936-token vocabulary), so that dW is one GEMM over stored tiles instead
- * of a second pass over the logits. */
+ * of a second pass over the logits.
+ * For bi_logprob_fwd with 1 <= T <= 128 rows (decode-style scoring) it also holds the rows' fp32
+ * logits (about 4 T (V + 256) bytes), so that the call runs on every SM instead of one cluster;
+ * the bits are the same either way. */
 BI_API size_t bi_workspace_bytes(int64_t T, int32_t H, int32_t V, int32_t R);
 
 /* Smallest workspace bi_is_loss_fwd_bwd accepts (O(T H) bytes).  Any ws_bytes from this size up
  * to just below bi_workspace_bytes(...) selects the low-memory path, whose dW kernel recomputes
  * the logits (about a third more tensor work per step).  Both paths produce the same bits for
- * every output except grad_w, where they differ by rounding only.  For R = 0 it equals
- * bi_workspace_bytes. */
+ * every output except grad_w, where they differ by rounding only.  For R = 0 it is the per-CTA
+ * partials only; bi_logprob_fwd accepts it for any T (with T <= 128 it then scores the rows on one
+ * cluster, with the same bits). */
 BI_API size_t bi_workspace_bytes_min(int64_t T, int32_t H, int32_t V, int32_t R);
 
 /* Token log-probabilities log pi(y_t | h_t) under the LM head W (definition above).
@@ -137,8 +141,13 @@ BI_API size_t bi_workspace_bytes_min(int64_t T, int32_t H, int32_t V, int32_t R)
  *   targets  [T]    int32     token ids; an id outside [0, V) sets BI_ERR_BAD_TARGET and NaN
  *   logprob  [T]    float     out: z_{t,y_t} - lse_t
  *   lse      [T]    float     out (may be NULL): log-sum-exp of the row's logits
- * The same kernels serve T = 1 (one row per call, decode style) and packed batches, and produce
- * identical bits for a row in both. */
+ * A row gets identical bits whether it is scored alone (T = 1, decode style) or packed.  Packed
+ * batches run on the cluster kernel (one cluster sweeps the vocabulary for each 128-row tile).
+ * With 1 <= T <= 128 and a workspace of bi_workspace_bytes(T, H, V, 0) bytes the rows are scored
+ * on every SM instead: the logit tiles with the cluster kernel's instruction sequence, then the
+ * reference chain, the class partial sums and their combine in the cluster kernel's order, which
+ * reproduces its bits ("Zero Mismatch, Simple Async RL", section "Alignment permits a simpler
+ * learning path"). */
 BI_API bi_status bi_logprob_fwd(const uint16_t* hidden, const uint16_t* w_lm, const int32_t* targets,
                          int64_t T, int32_t H, int32_t V, float* logprob, float* lse,
                          int32_t* dev_status, void* ws, size_t ws_bytes, void* stream);
@@ -151,7 +160,7 @@ BI_API bi_status bi_logprob_fwd(const uint16_t* hidden, const uint16_t* w_lm, co
  * library (480 KB, one [2][3][128] float block per CTA of a full-device grid, held by every GPU
  * that loads the library until the process exits).  Its size does not depend on T: any T that
  * bi_logprob_fwd accepts is accepted, and the results are bit-identical to bi_logprob_fwd's
- * (same kernel, same tiles).
+ * (it always runs the cluster kernel, whose bits both of bi_logprob_fwd's paths have).
  *   - The call allocates nothing (no cudaMalloc, no library allocator).  Its first call on a
  *     device looks up the array's device address with that device current; make that first call
  *     before any stream capture.

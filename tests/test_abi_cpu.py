@@ -67,6 +67,9 @@ def test_workspace_bytes(lib):
     lo = lib.bi_workspace_bytes_min(2000, 1536, 151936, 64)
     assert d - lo >= 2048 * 151936 * 2 and lo < 2000 * 1536 * 2 * 4 + (64 << 20)
     assert lib.bi_workspace_bytes_min(2000, 1536, 151936, 0) == b
+    # up to 128 rows the logprob workspace also holds the rows' logits for the all-SM path
+    assert lib.bi_workspace_bytes(128, 1536, 151936, 0) >= 128 * (151936 + 256) * 4
+    assert lib.bi_workspace_bytes_min(128, 1536, 151936, 0) == b
 
 
 FAKE = 1 << 20  # aligned non-null address; never dereferenced on the paths below
@@ -82,8 +85,11 @@ def test_logprob_argument_checks(lib):
     # unsupported H
     assert lib.bi_logprob_fwd(FAKE, FAKE, FAKE, 10, 100, 512, FAKE, None, st, FAKE, ws_bytes, None) == 2
     assert lib.bi_logprob_fwd(FAKE, FAKE, FAKE, 10, 704, 512, FAKE, None, st, FAKE, ws_bytes, None) == 2
-    # workspace too small / missing / misaligned
-    assert lib.bi_logprob_fwd(FAKE, FAKE, FAKE, 10, 128, 512, FAKE, None, st, FAKE, ws_bytes - 1, None) == 3
+    # workspace too small (below the minimum; between the minimum and bi_workspace_bytes the call
+    # runs on the cluster kernel instead of every SM) / missing / misaligned
+    ws_min = lib.bi_workspace_bytes_min(10, 128, 512, 0)
+    assert ws_min < ws_bytes
+    assert lib.bi_logprob_fwd(FAKE, FAKE, FAKE, 10, 128, 512, FAKE, None, st, FAKE, ws_min - 1, None) == 3
     assert lib.bi_logprob_fwd(FAKE, FAKE, FAKE, 10, 128, 512, FAKE, None, st, None, ws_bytes, None) == 3
     assert lib.bi_logprob_fwd(FAKE, FAKE, FAKE, 10, 128, 512, FAKE, None, st, FAKE + 16, ws_bytes, None) == 3
     # negative sizes

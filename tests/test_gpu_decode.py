@@ -1,0 +1,70 @@
+"""Decode-style scoring (bi_logprob_fwd with T <= 128 rows, computed on every SM) gives the same bits
+as the cluster kernel that scores packed batches ("Zero Mismatch, Simple Async RL", section
+"Alignment permits a simpler learning path": rollout and learner logprobs bit-identical whether a
+row is scored alone or packed), for the tilings of several hidden sizes, and matches the oracle."""
+import numpy as np
+import pytest
+import torch
+
+import async_rl_b200 as bi
+from oracle import isloss_oracle as orc
+from workloads.synth import random_inputs
+
+from .util import LOGPROB_TOL, assert_close
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from async_rl_b200.build import build
+    build()
+
+
+def _lp(h, w, y, dev, ws_rows=None):
+    T = h.shape[0]
+    ws = bi.make_workspace(ws_rows if ws_rows is not None else T, h.shape[1], w.shape[0], 0, dev)
+    lp, lse, st = bi.logprob_fwd(h, w, y, want_lse=True, ws=ws)
+    torch.cuda.synchronize()
+    bi.check_status(st)
+    return lp, lse
+
+
+# (H, V): tilings C = 1 (H = 128, 192), C = 6 (1536, NZ = 256), C = 8 with NZ = 192 (2560); V ragged
+@pytest.mark.parametrize("H,V", [(128, 549), (192, 4099), (1536, 32771), (2560, 20011)])
+def test_few_rows_bitwise_equal_to_packed_batch(H, V, cuda_device):
+    h, w, y = random_inputs(300, H, V, seed=H + V)
+    h, w, y = h.to(cuda_device), w.to(cuda_device), y.to(cuda_device)
+    packed_lp, packed_lse = _lp(h, w, y, cuda_device)          # 300 rows: the cluster kernel
+    for rows in ([0], [5, 17, 299], list(range(128)), list(range(172, 300))):
+        r = torch.tensor(rows, device=cuda_device)
+        lp, lse = _lp(h[r].contiguous(), w, y[r].contiguous(), cuda_device)   # <= 128 rows: every SM
+        assert torch.equal(lp, packed_lp[r]), f"logprob bits differ (H={H}, V={V}, {len(rows)} rows)"
+        assert torch.equal(lse, packed_lse[r]), f"lse bits differ (H={H}, V={V}, {len(rows)} rows)"
+    # and the few-row path against the fp64 oracle
+    lp, _ = _lp(h[:7].contiguous(), w, y[:7].contiguous(), cuda_device)
+    ref, _ = orc.token_logprob(h[:7].cpu(), w.cpu(), y[:7].cpu())
+    assert_close("logprob", lp.double().cpu().numpy(), ref, LOGPROB_TOL, LOGPROB_TOL)
+
+
+def test_few_rows_with_minimum_workspace_take_the_cluster_kernel(cuda_device):
+    """A workspace without room for the rows' logits is accepted; the bits are the same."""
+    h, w, y = random_inputs(5, 1536, 8192, seed=3)
+    h, w, y = h.to(cuda_device), w.to(cuda_device), y.to(cuda_device)
+    fast, _ = _lp(h, w, y, cuda_device)
+    ws = torch.empty(max(bi.workspace_bytes(1000, 1536, 8192, 0), 256), dtype=torch.uint8, device=cuda_device)
+    small = ws[: bi.workspace_bytes(1000, 1536, 8192, 0)]
+    assert small.numel() < bi.workspace_bytes(5, 1536, 8192, 0)
+    lp, _, st = bi.logprob_fwd(h, w, y, ws=small)
+    torch.cuda.synchronize()
+    bi.check_status(st)
+    assert torch.equal(lp, fast)
+
+
+def test_few_rows_bad_target_sets_status(cuda_device):
+    h, w, y = random_inputs(3, 128, 512, seed=9)
+    y[1] = 512
+    lp, _, st = bi.logprob_fwd(h.to(cuda_device), w.to(cuda_device), y.to(cuda_device))
+    torch.cuda.synchronize()
+    assert int(st.item()) == 6
+    assert torch.isnan(lp[1]).item() and torch.isfinite(lp[0]).item() and torch.isfinite(lp[2]).item()
