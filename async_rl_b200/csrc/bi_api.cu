@@ -893,11 +893,11 @@ bi_status bi_rmsnorm(const uint16_t* x, const uint16_t* g, float eps, uint16_t* 
   const DevInfo* di = device_info();
   if (!di) return BI_ERR_CUDA;
   // a warp per row, 8 rows per block, rows strided over the grid.  The variant depends on H only:
-  // rows of up to 2048 elements stay in registers (2 resident blocks per SM), longer rows take
-  // two passes (8 resident blocks per SM).
+  // rows of up to 3072 elements stay in registers (2 resident blocks per SM up to 2048, then 1),
+  // longer rows take two passes (8 resident blocks per SM).
   const int64_t want = (M + bi::kNormThreads / 32 - 1) / (bi::kNormThreads / 32);
   const int kvec = (H + 255) / 256;
-  const int64_t cap = static_cast<int64_t>(di->sms) * (kvec <= bi::kNormRegMaxVec ? 2 : 8);
+  const int64_t cap = static_cast<int64_t>(di->sms) * (kvec <= bi::kNormRegMaxVec ? bi::kNormRegBlocks(kvec) : 8);
   const unsigned blocks = static_cast<unsigned>(want < cap ? want : cap);
   ProfScope ps(kKRmsNorm, s);
   switch (kvec) {
@@ -905,8 +905,8 @@ bi_status bi_rmsnorm(const uint16_t* x, const uint16_t* g, float eps, uint16_t* 
   case V_:                                                                                \
     bi::k_rmsnorm_reg<V_><<<blocks, bi::kNormThreads, 0, s>>>(x, g, eps, y, M, H);        \
     break;
-    BI_NORM_CASE(1) BI_NORM_CASE(2) BI_NORM_CASE(3) BI_NORM_CASE(4)
-    BI_NORM_CASE(5) BI_NORM_CASE(6) BI_NORM_CASE(7) BI_NORM_CASE(8)
+    BI_NORM_CASE(1) BI_NORM_CASE(2) BI_NORM_CASE(3) BI_NORM_CASE(4) BI_NORM_CASE(5) BI_NORM_CASE(6)
+    BI_NORM_CASE(7) BI_NORM_CASE(8) BI_NORM_CASE(9) BI_NORM_CASE(10) BI_NORM_CASE(11) BI_NORM_CASE(12)
 #undef BI_NORM_CASE
     default:
       bi::k_rmsnorm<<<blocks, bi::kNormThreads, 0, s>>>(x, g, eps, y, M, H);

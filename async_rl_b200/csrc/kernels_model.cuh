@@ -281,9 +281,10 @@ __device__ __forceinline__ uint4 ldg_nc_u4(const void* p) {
 // Rows of at most 256 kVec elements: the row stays in registers (one read of x), and the next
 // row's vectors are requested before the current row is reduced.  Same per-lane order and shuffle
 // tree as the general kernel below.
-constexpr int kNormRegMaxVec = 8;  // rows of up to 2048 elements stay in registers
+constexpr int kNormRegMaxVec = 12;  // rows of up to 3072 elements stay in registers
+constexpr int kNormRegBlocks(int vec) { return vec <= 8 ? 2 : 1; }  // resident blocks per SM
 template <int kVec>
-__global__ void __launch_bounds__(kNormThreads, 2)
+__global__ void __launch_bounds__(kNormThreads, kNormRegBlocks(kVec))
     k_rmsnorm_reg(const uint16_t* __restrict__ x, const uint16_t* __restrict__ g, float eps,
                   uint16_t* __restrict__ y, int64_t M, int32_t H) {
   const int lane = threadIdx.x & 31;
