@@ -140,6 +140,13 @@ __device__ __forceinline__ void gemm_mma_role(GemmShared& sh, const GemmArgs& a,
   umma_commit_pair(&sh.mma_done, pair_mask);
 }
 
+// 32-byte global store (sm_100 256-bit vector store); the address must be 32-byte aligned.
+__device__ __forceinline__ void st_global_v8(uint16_t* dst, const uint32_t* p) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "r"(p[0]), "r"(p[1]),
+               "r"(p[2]), "r"(p[3]), "r"(p[4]), "r"(p[5]), "r"(p[6]), "r"(p[7])
+               : "memory");
+}
+
 // ---- epilogue (128 threads per CTA): this CTA's 128 rows of the tile, fp32 -> bf16 ----
 __device__ __forceinline__ void gemm_epilogue_role(GemmShared& sh, const GemmArgs& a, const GemmCtx& x,
                                                    uint32_t tmem) {
@@ -150,6 +157,7 @@ __device__ __forceinline__ void gemm_epilogue_role(GemmShared& sh, const GemmArg
   const int et = threadIdx.x - 64;
   const uint32_t tl = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
   const uint32_t lead_empty = mapa_shared(smem_u32(&sh.acc_empty[0]), 0u);
+  const bool wide = (a.N % 16 == 0) && ((reinterpret_cast<uintptr_t>(a.y) & 31u) == 0);
   uint32_t tc = 0, epc = 0;
   for (int64_t t = x.cl; t < x.ntiles; t += x.ncl, ++tc) {
     const int64_t mt = t / x.tiles_n;
@@ -168,15 +176,19 @@ __device__ __forceinline__ void gemm_epilogue_role(GemmShared& sh, const GemmArg
       tmem_ld_wait();
       const int cb = col0 + c * 32;
       if (rvalid) {
+        uint32_t p[16];
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          if (cb + 8 * g < a.N) {  // N is a multiple of 8: an 8-column group is all in or all out
-            const uint4 q = make_uint4(pack_bf16x2(__uint_as_float(v[8 * g + 0]), __uint_as_float(v[8 * g + 1])),
-                                       pack_bf16x2(__uint_as_float(v[8 * g + 2]), __uint_as_float(v[8 * g + 3])),
-                                       pack_bf16x2(__uint_as_float(v[8 * g + 4]), __uint_as_float(v[8 * g + 5])),
-                                       pack_bf16x2(__uint_as_float(v[8 * g + 6]), __uint_as_float(v[8 * g + 7])));
-            *reinterpret_cast<uint4*>(dst + c * 32 + 8 * g) = q;
-          }
+        for (int e = 0; e < 16; ++e) p[e] = pack_bf16x2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
+        if (wide) {
+          // N a multiple of 16 and y 32-byte aligned: whole 32-byte sectors, 16 columns a store
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+            if (cb + 16 * h < a.N) st_global_v8(dst + c * 32 + 16 * h, p + 8 * h);
+        } else {
+#pragma unroll
+          for (int g = 0; g < 4; ++g)
+            if (cb + 8 * g < a.N)  // N is a multiple of 8: an 8-column group is all in or all out
+              *reinterpret_cast<uint4*>(dst + c * 32 + 8 * g) = make_uint4(p[4 * g], p[4 * g + 1], p[4 * g + 2], p[4 * g + 3]);
         }
       }
     }
