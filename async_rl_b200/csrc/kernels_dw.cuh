@@ -267,6 +267,8 @@ __global__ void __launch_bounds__(kDwThreads, 1)
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t tl = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    // row chunks are 128-byte multiples from the base: whole sectors when the base allows
+    const bool sectors = (reinterpret_cast<uintptr_t>(a.grad_w) & 31u) == 0;
     uint32_t n_it = 0;
     for (int it = blockIdx.x; it < nitems; it += gridDim.x, ++n_it) {
       const int w = it / a.nsl, q = it - (it / a.nsl) * a.nsl;
@@ -290,9 +292,14 @@ __global__ void __launch_bounds__(kDwThreads, 1)
           tmem_ld32(tl + half * kHS + c * 32, r);
           tmem_ld_wait();
           if (dst) {
-            uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+            if (sectors) {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) d4[e] = make_uint4(r[4 * e], r[4 * e + 1], r[4 * e + 2], r[4 * e + 3]);
+              for (int e = 0; e < 4; ++e) st_global_v8(dst + c * 32 + 8 * e, r + 8 * e);
+            } else {
+              uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) d4[e] = make_uint4(r[4 * e], r[4 * e + 1], r[4 * e + 2], r[4 * e + 3]);
+            }
           }
         }
       }

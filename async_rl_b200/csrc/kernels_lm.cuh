@@ -457,7 +457,17 @@ __device__ __forceinline__ void lm_rescale_role(LmShared& sh, const LmArgs& a, c
 }
 
 // ---------------- epilogue helpers ----------------
-// Store one 32-value chunk of bf16 to global memory (64 bytes).
+// Store one 32-value chunk of bf16 to a 32-byte aligned address as two whole 32-byte sectors
+// (sm_100 256-bit stores); the P store and the dZ scratch are laid out so that every chunk is.
+__device__ __forceinline__ void store_bf16x32_sectors(uint16_t* dst, const float (&d)[32]) {
+  uint32_t p[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) p[e] = pack_bf16x2(d[2 * e], d[2 * e + 1]);
+  st_global_v8(dst, p);
+  st_global_v8(dst + 16, p + 8);
+}
+
+// Store one 32-value chunk of bf16 to global memory (64 bytes, 16-byte aligned).
 __device__ __forceinline__ void store_bf16x32(uint16_t* dst, const float (&d)[32]) {
   uint4* d4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll
@@ -593,7 +603,7 @@ __device__ __forceinline__ void lm_fwd_epilogue_role(LmShared& sh, const LmArgs&
           if (tgt) zyp = z;
         }
         sp += cs;
-        if (kMode == kModeFwdDH) store_bf16x32(dzrow + c * 32, d);
+        if (kMode == kModeFwdDH) store_bf16x32_sectors(dzrow + c * 32, d);
       }
       tc_fence_before();
       mbar_arrive(&sh.z_empty[b]);
@@ -687,6 +697,8 @@ __device__ __forceinline__ void lm_fwd_epilogue_role(LmShared& sh, const LmArgs&
         const float gs = g / s;
         const uint16_t* wy = (valid && !ybad) ? a.w_lm + static_cast<int64_t>(y) * a.H + x.slice0 : nullptr;
         uint16_t* dst = valid ? a.grad_hidden + r * a.H + x.slice0 : nullptr;
+        // row chunks are 64-byte multiples from the base: whole sectors when the base allows
+        const bool sectors = (reinterpret_cast<uintptr_t>(a.grad_hidden) & 31u) == 0;
 #pragma unroll 1
         for (int c = 0; c < kHS / 32; ++c) {
           uint32_t v[32];
@@ -712,7 +724,10 @@ __device__ __forceinline__ void lm_fwd_epilogue_role(LmShared& sh, const LmArgs&
 #pragma unroll
               for (int h = 0; h < 32; ++h) d[h] = __int_as_float(0x7fc00000);
             }
-            store_bf16x32(dst + c * 32, d);
+            if (sectors)
+              store_bf16x32_sectors(dst + c * 32, d);
+            else
+              store_bf16x32(dst + c * 32, d);
           }
         }
         tc_fence_before();
@@ -821,7 +836,7 @@ __device__ __forceinline__ void lm_dw_epilogue_role(LmShared& sh, const LmArgs& 
           const float oh = (static_cast<int64_t>(yc) == vrow) ? 1.f : 0.f;
           d[q] = (v_ok && yc != INT32_MIN) ? sh.col_g[tc] * (oh - pr) : 0.f;
         }
-        store_bf16x32(dzrow + c * 32, d);
+        store_bf16x32_sectors(dzrow + c * 32, d);
       }
       tc_fence_before();
       mbar_arrive(&sh.z_empty[0]);

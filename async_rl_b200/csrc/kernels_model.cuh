@@ -140,13 +140,6 @@ __device__ __forceinline__ void gemm_mma_role(GemmShared& sh, const GemmArgs& a,
   umma_commit_pair(&sh.mma_done, pair_mask);
 }
 
-// 32-byte global store (sm_100 256-bit vector store); the address must be 32-byte aligned.
-__device__ __forceinline__ void st_global_v8(uint16_t* dst, const uint32_t* p) {
-  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "r"(p[0]), "r"(p[1]),
-               "r"(p[2]), "r"(p[3]), "r"(p[4]), "r"(p[5]), "r"(p[6]), "r"(p[7])
-               : "memory");
-}
-
 // ---- epilogue (128 threads per CTA): this CTA's 128 rows of the tile, fp32 -> bf16 ----
 __device__ __forceinline__ void gemm_epilogue_role(GemmShared& sh, const GemmArgs& a, const GemmCtx& x,
                                                    uint32_t tmem) {

@@ -317,6 +317,14 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
+// 32-byte global store (sm_100 256-bit vector store): one whole sector per instruction.  The
+// address must be 32-byte aligned.
+__device__ __forceinline__ void st_global_v8(void* dst, const uint32_t* p) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "r"(p[0]), "r"(p[1]),
+               "r"(p[2]), "r"(p[3]), "r"(p[4]), "r"(p[5]), "r"(p[6]), "r"(p[7])
+               : "memory");
+}
+
 constexpr float kLog2e = 1.4426950408889634f;
 
 }  // namespace bi
