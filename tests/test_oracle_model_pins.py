@@ -102,3 +102,20 @@ def test_rmsnorm_zero_row_and_row_independence():
     assert np.all(y[2] == 0.0)
     for r in range(5):
         assert np.array_equal(mo.rmsnorm(x[r:r + 1], g, 1e-6)[0], y[r])
+
+
+def test_dense_input_generators_are_seeded_and_follow_the_recipe():
+    """The seeded generators behind the dense-layer tests and the dense bench: deterministic, bf16,
+    and the stated distributions (x ~ N(0, 1), W ~ N(0, 0.02); RMSNorm rows N(0, s^2) with
+    s ~ U[0.05, 20], gains 1 + N(0, 0.1))."""
+    from workloads import dense_inputs, norm_inputs
+    x1, w1 = dense_inputs(2000, 512, 300, seed=7)
+    x2, w2 = dense_inputs(2000, 512, 300, seed=7)
+    assert torch.equal(x1, x2) and torch.equal(w1, w2)
+    assert x1.dtype == torch.bfloat16 and w1.shape == (300, 512)
+    assert abs(float(x1.float().std()) - 1.0) < 0.01 and abs(float(w1.float().std()) - 0.02) < 0.001
+    x, g = norm_inputs(4000, 256, seed=8)
+    assert torch.equal(x, norm_inputs(4000, 256, seed=8)[0]) and g.shape == (256,)
+    s = x.float().pow(2).mean(dim=1).sqrt()
+    assert float(s.min()) > 0.04 and float(s.max()) < 21.0 and float(s.median()) > 5.0
+    assert abs(float(g.float().mean()) - 1.0) < 0.03 and 0.07 < float(g.float().std()) < 0.13
