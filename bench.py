@@ -15,6 +15,9 @@ ranks sum dW and the three loss/D3 scalars with NCCL, the one exchange step of d
 --workload dense times the batch-invariant dense layers instead (not the default line): one step is
 RMSNorm of the 1.5B-shape hidden states [76239, 1536] followed by the gate/up projection
 Y = X W^T with W [8960, 1536] (bi_rmsnorm + bi_gemm_bf16); ranks are independent replicas.
+
+--workload decode times decode-style scoring (not the default line): one bi_logprob_fwd call per
+step on one row of the 1.5B head (the all-SM path), with the cluster kernel's latency beside it.
 """
 from __future__ import annotations
 
@@ -49,8 +52,9 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--small", action="store_true",
                     help="profiling case: same head, 4 responses of 1024 rows (T=4096); not a bench line")
-    ap.add_argument("--workload", choices=["loss", "dense"], default="loss",
-                    help="loss: the fused LM-head step (default line); dense: RMSNorm + linear layer")
+    ap.add_argument("--workload", choices=["loss", "dense", "decode"], default="loss",
+                    help="loss: the fused LM-head step (default line); dense: RMSNorm + linear layer; "
+                         "decode: one-row logprob scoring latency")
     return ap.parse_args()
 
 
@@ -556,9 +560,132 @@ def run_dense(args):
         pg.destroy_process_group()
 
 
+DECODE_METRIC = "decode-style logprob scoring latency, one row per call, at H1536 V151936"
+
+
+def run_decode_reference(args):
+    """--impl reference --workload decode: the fp64 oracle scoring one row per step on the host cores."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    from oracle import isloss_oracle as orc
+    from workloads.synth import random_inputs
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max((d.get("num_threads", 1) for d in threadpool_info()), default=os.cpu_count())
+    except Exception:  # pragma: no cover
+        cores = os.cpu_count()
+    h, w, y = random_inputs(1, 1536, 151936, seed=1234)
+    times = []
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        orc.token_logprob(h, w, y)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    ms = 1e3 * statistics.mean(times)
+    print(json.dumps({"impl": "reference", "metric": DECODE_METRIC, "value": ms, "unit": "ms per call",
+                      "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+                      "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                      "data": "synthetic",
+                      "config": {"workload": "decode: 1 row per call, H=1536 V=151936, fp64 oracle on host cores"},
+                      "cpu_baseline": {"value": ms, "unit": "ms per call", "cores": int(cores), "kind": "oracle",
+                                       "sample": "one row per step"},
+                      "e2e": {"value": ms, "unit": "ms per call", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),
+          flush=True)
+
+
+def run_decode(args):
+    """--workload decode: one-row bi_logprob_fwd calls (all-SM path), ms per call."""
+    rank, world, local = dist_env()
+    import async_rl_b200 as bi
+    from async_rl_b200.build import build
+    from workloads.synth import random_inputs
+
+    if rank == 0:
+        build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    H, V = 1536, 151936
+    h, w, y = random_inputs(128, H, V, seed=1234 + rank)
+    h, w, y = h.to(dev), w.to(dev), y.to(dev)
+    h1, y1 = h[:1].contiguous(), y[:1].contiguous()
+    out = torch.empty(1, dtype=torch.float32, device=dev)
+    st = torch.empty(1, dtype=torch.int32, device=dev)
+    ws_fast = bi.make_workspace(1, H, V, 0, dev)
+    ws_min = torch.empty(bi.workspace_bytes(1, H, V, 0, minimal=True), dtype=torch.uint8, device=dev)
+
+    def timed(ws, n, T=1):
+        hh, yy = h[:T].contiguous(), y[:T].contiguous()
+        o = torch.empty(T, dtype=torch.float32, device=dev)
+        for _ in range(args.warmup):
+            bi.logprob_fwd(hh, w, yy, ws=ws, out=o, status=st)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(n):
+            bi.logprob_fwd(hh, w, yy, ws=ws, out=o, status=st)
+        e1.record()
+        torch.cuda.synchronize()
+        bi.check_status(st)
+        return e0.elapsed_time(e1) / n
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    bi.profile_reset()
+    bi.profile_enable(True)
+    ms = timed(ws_fast, args.steps)
+    bi.profile_enable(False)
+    clk = clocks.stop()
+    prof = bi.profile_read()
+    ms_128 = timed(bi.make_workspace(128, H, V, 0, dev), args.steps, T=128)
+    ms_cluster = timed(ws_min, args.steps)
+    # end to end: the row copied in from pinned memory and its logprob read back, every call
+    hh = h1.cpu().pin_memory()
+    yh = y1.cpu().pin_memory()
+    oh = torch.empty(1, dtype=torch.float32).pin_memory()
+    hd, yd = torch.empty_like(h1), torch.empty_like(y1)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        hd.copy_(hh, non_blocking=True)
+        yd.copy_(yh, non_blocking=True)
+        bi.logprob_fwd(hd, w, yd, ws=ws_fast, out=out, status=st)
+        oh.copy_(out, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    ems = e0.elapsed_time(e1) / args.steps
+    peaks, peak_src = measured_peaks()
+    w_bytes = 2.0 * V * H
+    zt = prof.get("k_lm_ztiles", (float("nan"), 1))
+    zt_ms = zt[0] / max(zt[1], 1)
+    line = {"metric": DECODE_METRIC, "value": ms, "unit": "ms per call", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": False, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"decode: 1 row per bi_logprob_fwd call, H={H} V={V}, all-SM path",
+                       "parallelism": f"replicas{world}", "l2": "W 0.47 GB exceeds L2; no flush"},
+            "rows_128_ms": ms_128, "cluster_kernel_ms": ms_cluster,
+            "roofline": {"bound": "hbm", "kernel": "k_lm_ztiles", "achieved": w_bytes / (zt_ms * 1e-3) / 1e9,
+                         "peak": float(peaks.get("hbm_gbs")), "unit": "GB/s",
+                         "frac": w_bytes / (zt_ms * 1e-3) / 1e9 / float(peaks.get("hbm_gbs")), "traffic": None,
+                         "peak_source": f"{peak_src} hbm_gbs", "algorithmic_bytes_per_launch": w_bytes},
+            "kernels": {k: {"ms_per_launch": v[0] / max(v[1], 1), "launches": v[1]} for k, v in prof.items()},
+            "gpu_launches": int(sum(v[1] for v in prof.values())), "clocks": clk,
+            "e2e": {"value": ems, "unit": "ms per call", "h2d_bytes_per_step": int(H * 2 + 4),
+                    "d2h_bytes_per_step": 4, "h2d": "pinned host row and target in, logprob out, every call"}}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
-    if args.workload == "dense":
+    if args.workload == "decode":
+        if args.impl == "reference":
+            run_decode_reference(args)
+        else:
+            run_decode(args)
+    elif args.workload == "dense":
         if args.impl == "reference":
             run_dense_reference(args)
         else:

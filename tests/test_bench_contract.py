@@ -60,3 +60,20 @@ def test_dense_workload_line():
     assert line["gpu_launches"] == 6 and line["value"] > 0
     assert 0 < line["roofline"]["frac"] < 2 and 0 < line["rmsnorm_roofline"]["frac"] < 2
     assert line["e2e"]["d2h_bytes_per_step"] == 76239 * 8960 * 2
+
+
+@pytest.mark.slow
+def test_decode_reference_arm_line():
+    line = _run(["--impl", "reference", "--workload", "decode", "--steps", "1", "--warmup", "0"], timeout=600)
+    for k in REQUIRED:
+        assert k in line, k
+    assert line["impl"] == "reference" and line["higher_is_better"] is False and line["value"] > 0
+
+
+@pytest.mark.gpu
+def test_decode_workload_line():
+    line = _run(["--workload", "decode", "--steps", "20", "--warmup", "3"], timeout=900)
+    for k in REQUIRED + ("roofline", "clocks", "gpu_launches", "cluster_kernel_ms", "rows_128_ms"):
+        assert k in line, k
+    assert line["gpu_launches"] == 40 and line["value"] < line["cluster_kernel_ms"]
+    assert 0 < line["roofline"]["frac"] < 2 and line["e2e"]["h2d_bytes_per_step"] > 0
