@@ -614,28 +614,30 @@ def run_decode(args):
     ws_fast = bi.make_workspace(1, H, V, 0, dev)
     ws_min = torch.empty(bi.workspace_bytes(1, H, V, 0, minimal=True), dtype=torch.uint8, device=dev)
 
-    def timed(ws, n, T=1):
+    def timed(ws, n, T=1, profiled=False):
         hh, yy = h[:T].contiguous(), y[:T].contiguous()
         o = torch.empty(T, dtype=torch.float32, device=dev)
         for _ in range(args.warmup):
             bi.logprob_fwd(hh, w, yy, ws=ws, out=o, status=st)
         torch.cuda.synchronize()
+        if profiled:  # only the timed calls are recorded
+            bi.profile_reset()
+            bi.profile_enable(True)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         for _ in range(n):
             bi.logprob_fwd(hh, w, yy, ws=ws, out=o, status=st)
         e1.record()
         torch.cuda.synchronize()
+        if profiled:
+            bi.profile_enable(False)
         bi.check_status(st)
         return e0.elapsed_time(e1) / n
 
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.3)
-    bi.profile_reset()
-    bi.profile_enable(True)
-    ms = timed(ws_fast, args.steps)
-    bi.profile_enable(False)
+    ms = timed(ws_fast, args.steps, profiled=True)
     clk = clocks.stop()
     prof = bi.profile_read()
     ms_128 = timed(bi.make_workspace(128, H, V, 0, dev), args.steps, T=128)
