@@ -199,7 +199,7 @@ __global__ void __launch_bounds__(kZtThreads, 1)
   }
 }
 
-constexpr int kZsThreads = 256;
+constexpr int kZsThreads = 1024;
 
 // Dynamic shared memory of k_lm_zscan: the references and the chunk sums of one row.
 __host__ __device__ constexpr size_t zscan_smem(int nvz, int nz) {
@@ -226,6 +226,7 @@ __global__ void __launch_bounds__(kZsThreads)
   __syncthreads();
   if (threadIdx.x == 0) {
     float mprev = -INFINITY;
+#pragma unroll 8
     for (int j = 0; j < nvz; ++j) {
       const float M = mref[j];
       const float mnew = (M > mprev + kTau) ? M : mprev;
@@ -265,12 +266,14 @@ __global__ void __launch_bounds__(kZsThreads)
   if (threadIdx.x < C) {
     const int k = threadIdx.x;
     float mp = -INFINITY, sp = 0.f;
+#pragma unroll 4
     for (int j = k; j < nvz; j += C) {
       const float mnew = mref[j];
       if (mnew != mp) {
         sp = (mp == -INFINITY) ? 0.f : sp * ex2_approx((mp - mnew) * kLog2e);
         mp = mnew;
       }
+#pragma unroll
       for (int c = 0; c < kChunks; ++c) sp += csum[j * kChunks + c];
     }
     cls[k] = mp;
