@@ -1,4 +1,4 @@
-"""bench.py keeps its contract: one JSON line with the keys the driver reads.  The reference arm
+"""bench.py keeps its contract: one JSON line with every key its consumers read.  The reference arm
 (the fp64 oracle on host cores) runs here on CPU; the CUDA arm runs its small profiling case on
 the GPU (the same code path as the full line, T = 4096)."""
 import json
