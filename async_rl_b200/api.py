@@ -30,12 +30,26 @@ def _stream(device: torch.device) -> int:
 
 
 def _check_cuda(t: torch.Tensor, name: str, dtype: torch.dtype, device: torch.device):
+    # the library dereferences every pointer on the GPU: host memory must never reach it
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor, got {t.device}")
     if t.device != device:
         raise ValueError(f"{name} must be on {device}, got {t.device}")
     if t.dtype != dtype:
         raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
+
+
+def _check_buffers(dev: torch.device, **named):
+    """Caller-supplied outputs, workspace and status words: CUDA tensors on `dev`, contiguous."""
+    for name, t in named.items():
+        if t is None:
+            continue
+        if t.device.type != "cuda" or t.device != dev:
+            raise ValueError(f"{name} must be a CUDA tensor on {dev}, got {t.device}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
 
 
 def workspace_bytes(T: int, H: int, V: int, R: int = 0, minimal: bool = False) -> int:
@@ -75,6 +89,9 @@ def logprob_fwd(hidden: torch.Tensor, w: torch.Tensor, targets: torch.Tensor, wa
     lib = _lib.load()
     if ws is None:
         ws = make_workspace(T, H, V, 0, dev)
+    _check_buffers(dev, ws=ws, out=out, status=status)
+    if out is not None and (out.dtype != torch.float32 or out.numel() < T):
+        raise ValueError("out must be float32 with at least T elements")
     logprob = out if out is not None else torch.empty(T, dtype=torch.float32, device=dev)
     lse = torch.empty(T, dtype=torch.float32, device=dev) if want_lse else None
     st = status if status is not None else torch.empty(1, dtype=torch.int32, device=dev)
@@ -132,6 +149,8 @@ def is_loss_fwd_bwd(hidden, w, targets, rollout_logprob, rewards, resp_offsets, 
     if ws is None:
         ws = make_workspace(T, H, V, R, dev)
     o = out if out is not None else LossOutputs.allocate(T, H, V, dev)
+    _check_buffers(dev, ws=ws, loss=o.loss, logprob=o.logprob, is_weight=o.is_weight, token_loss=o.token_loss,
+                   d3_raw=o.d3_raw, grad_hidden=o.grad_hidden, grad_w=o.grad_w, status=o.status)
     if variant not in _lib.LOSS_VARIANTS:
         raise ValueError(f"unknown loss variant {variant!r}")
     cfg = _lib.LossCfg(_lib.LOSS_VARIANTS[variant], float(eps_low), float(eps_high), float(gate))
@@ -156,6 +175,7 @@ def d3_stats(learner_logprob, rollout_logprob, mask=None, ws=None):
     lib = _lib.load()
     if ws is None:
         ws = make_workspace(T, 64, 1, 0, dev)  # the R = 0 layout covers the block partials
+    _check_buffers(dev, ws=ws)
     raw = torch.empty(D3_DTYPE_BYTES, dtype=torch.uint8, device=dev)
     st = torch.empty(1, dtype=torch.int32, device=dev)
     code = lib.bi_d3_stats(_ptr(learner_logprob), _ptr(rollout_logprob), _ptr(mask), T, _ptr(raw), _ptr(st),
@@ -189,6 +209,7 @@ def gemm_bf16(x: torch.Tensor, w: torch.Tensor, out: Optional[torch.Tensor] = No
     _check_cuda(y, "out", torch.bfloat16, dev)
     if tuple(y.shape) != (M, N):
         raise ValueError(f"out must be [{M}, {N}]")
+    _check_buffers(dev, status=status)
     st = status if status is not None else torch.empty(1, dtype=torch.int32, device=dev)
     code = _lib.load().bi_gemm_bf16(_ptr(x), _ptr(w), _ptr(y), M, N, K, _ptr(st), _stream(dev))
     _raise_host(code, "bi_gemm_bf16")
@@ -206,6 +227,9 @@ def rmsnorm(x: torch.Tensor, g: torch.Tensor, eps: float, out: Optional[torch.Te
         raise ValueError(f"g must be [{H}]")
     y = out if out is not None else torch.empty(M, H, dtype=torch.bfloat16, device=dev)
     _check_cuda(y, "out", torch.bfloat16, dev)
+    _check_buffers(dev, status=status)
+    if y.shape != x.shape:
+        raise ValueError(f"out must be [{M}, {H}]")
     st = status if status is not None else torch.empty(1, dtype=torch.int32, device=dev)
     code = _lib.load().bi_rmsnorm(_ptr(x), _ptr(g), float(eps), _ptr(y), M, H, _ptr(st), _stream(dev))
     _raise_host(code, "bi_rmsnorm")
