@@ -218,6 +218,7 @@ def run_ours(args):
     rank, world, local = dist_env()
     import async_rl_b200 as bi
     from async_rl_b200.build import build
+    from async_rl_b200.dp import allreduce_step
     from workloads import make_batch, spec_for
 
     if rank == 0:
@@ -249,8 +250,7 @@ def run_ours(args):
         bi.is_loss_fwd_bwd(b.hidden, b.w, b.targets, logmu, b.rewards, b.resp_offsets, b.group_offsets,
                            None, rnorm, ws=ws, out=out)
         if pg is not None:
-            pg.all_reduce(out.grad_w)
-            pg.all_reduce(out.loss)
+            allreduce_step(pg, out.grad_w, out.loss)
 
     for _ in range(args.warmup):
         step()
@@ -330,8 +330,7 @@ def run_ours(args):
                                    d["group_offsets"], None, rnorm, ws=ws, out=out)
                 used[i % 2].record(main_s)
                 if pg is not None:
-                    pg.all_reduce(out.grad_w)
-                    pg.all_reduce(out.loss)
+                    allreduce_step(pg, out.grad_w, out.loss)
                 loss_h.copy_(out.loss, non_blocking=True)
                 d3_h.copy_(out.d3_raw, non_blocking=True)
 

@@ -44,10 +44,11 @@ def _worker(rank, world, port, q):
 
 def test_shard_covers_all_groups_contiguously():
     b, _ = _batch()
-    for world in (1, 2, 3, 4):
+    for world in (1, 2, 3, 4, 6, 8):   # more ranks than groups leaves some ranks empty
         sh = shard_by_groups(b.resp_offsets, b.group_offsets, b.prompt_lens, world)
-        assert sh[0][0] == 0 and sh[-1][1] == b.G
+        assert len(sh) == world and sh[0][0] == 0 and sh[-1][1] == b.G
         assert all(sh[k][1] == sh[k + 1][0] for k in range(world - 1))
+        assert all(g0 <= g1 for g0, g1 in sh)
 
 
 def test_dp_two_ranks_matches_single_process():
