@@ -331,6 +331,26 @@ def grad_rows(hidden, w, targets, g_rows, rows) -> np.ndarray:
     return out
 
 
+def grad_w_rows(hidden, w, targets, g_rows, lse_rows, vocab_ids) -> np.ndarray:
+    """dW rows for the given vocabulary ids: dW_v = sum_t dZ_tv h_t over every row t, with
+    dZ_tv = g_t (1[v = y_t] - exp(z_tv - lse_t)) (g_t = 0 on unscored rows).  Needs only the
+    logits of the selected ids, so any T fits; ``lse_rows`` comes from ``token_logprob``."""
+    Hm = _f64(hidden)
+    Wm = _f64(w)
+    y = _i64(targets)
+    v = np.asarray(vocab_ids, dtype=np.int64)
+    g = np.asarray(g_rows, dtype=np.float64)
+    lse = np.asarray(lse_rows, dtype=np.float64)
+    out = np.zeros((v.shape[0], Wm.shape[1]))
+    for s in range(0, Hm.shape[0], 4096):
+        z = Hm[s:s + 4096] @ Wm[v].T
+        dZ = -np.exp(z - lse[s:s + 4096, None])
+        dZ += (y[s:s + 4096, None] == v[None, :])
+        dZ *= g[s:s + 4096, None]
+        out += dZ.T @ Hm[s:s + 4096]
+    return out
+
+
 def kl_estimators(learner_logprob, rollout_logprob, mask=None) -> dict:
     """Sampled estimators of KL(mu || pi) from rollout samples, r = w = pi/mu:
     k1 = -log r, k2 = (log r)^2 / 2, k3 = r - 1 - log r (the D3 term); means over tokens."""

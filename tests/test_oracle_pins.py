@@ -272,6 +272,25 @@ def test_grad_rows_matches_full():
     assert np.allclose(dh, out["grad_hidden"][rows], rtol=0, atol=1e-15)
 
 
+def test_grad_w_rows_matches_full_and_worked_example():
+    """dW rows of selected vocabulary ids (any T): the hand-worked two-row example's closed-form
+    rows, and the full gradient's rows on a prompt-masked batch with a tail id and a target id."""
+    ex = _worked_example()
+    out = orc.is_loss_fwd_bwd(**ex)
+    dz0 = np.array([-1 / 4, 1 / 12, 1 / 12, 1 / 12])
+    dz1 = np.array([-1 / 24, 1 / 8, -1 / 24, -1 / 24])
+    rows = orc.grad_w_rows(ex["hidden"], ex["w"], ex["targets"], out["token_loss"], out["lse"], [3, 0, 1])
+    ref = np.outer(dz0, [LN3, 0.0]) + np.outer(dz1, [0.0, LN3])
+    assert np.allclose(rows, ref[[3, 0, 1]], rtol=0, atol=1e-15)
+    b = make_batch(spec_for("tiny", prompt_len=3))
+    lp, _ = orc.token_logprob(b.hidden, b.w_roll, b.targets)
+    full = orc.is_loss_fwd_bwd(b.hidden, b.w, b.targets, lp, b.rewards, b.resp_offsets, b.group_offsets,
+                               b.prompt_lens)
+    ids = np.array([0, int(b.targets[7]), 200, 511])
+    got = orc.grad_w_rows(b.hidden, b.w, b.targets, full["token_loss"], full["lse"], ids)
+    assert np.allclose(got, full["grad_w"][ids], rtol=1e-12, atol=1e-17)
+
+
 def test_kl_estimators_small_delta():
     """k3 equals the D3 term; for small delta k1 ~ -mean(delta), k2 ~ k3 ~ delta^2/2."""
     rng = np.random.default_rng(4)
