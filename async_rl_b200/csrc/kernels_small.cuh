@@ -27,13 +27,14 @@ struct RedPart {
   int64_t count;
   int64_t nonfinite;
   int64_t nclip;       // tokens whose gradient the clip removed
+  int64_t nrej;        // responses the sequence gate rejected
 };
-__device__ __forceinline__ RedPart red_zero() { return RedPart{0.0, 0.0, 0.0, 0.0, -INFINITY, 0, 0, 0, 0}; }
+__device__ __forceinline__ RedPart red_zero() { return RedPart{0.0, 0.0, 0.0, 0.0, -INFINITY, 0, 0, 0, 0, 0}; }
 
 struct Ctrl {          // small device-side control block at the start of the workspace
   int64_t n_scored;    // number of scored (compact) rows
   int32_t valid;       // offsets passed validation
-  int32_t n_rejected;  // responses rejected by the sequence gate
+  int32_t pad;
 };
 
 // Largest i in [0, R) with off[i] <= r (off[R] > r is guaranteed by validation).
@@ -71,7 +72,6 @@ __global__ void k_prep(const float* __restrict__ rewards, const int64_t* __restr
       raise_status(status, 8 /* BI_ERR_BAD_OFFSETS */);
       ctrl->n_scored = 0;
       ctrl->valid = 0;
-      ctrl->n_rejected = 0;
     }
     return;
   }
@@ -96,7 +96,6 @@ __global__ void k_prep(const float* __restrict__ rewards, const int64_t* __restr
     cprefix[R] = acc;
     ctrl->n_scored = acc;
     ctrl->valid = 1;
-    ctrl->n_rejected = 0;
   }
 }
 
@@ -172,6 +171,7 @@ __device__ __forceinline__ RedPart block_reduce(RedPart v) {
     v.count += __shfl_xor_sync(0xffffffffu, v.count, o);
     v.nonfinite += __shfl_xor_sync(0xffffffffu, v.nonfinite, o);
     v.nclip += __shfl_xor_sync(0xffffffffu, v.nclip, o);
+    v.nrej += __shfl_xor_sync(0xffffffffu, v.nrej, o);
   }
   __shared__ RedPart wp[32];
   const int w = threadIdx.x >> 5, nw = blockDim.x >> 5;
@@ -188,6 +188,7 @@ __device__ __forceinline__ RedPart block_reduce(RedPart v) {
       out.count += wp[i].count;
       out.nonfinite += wp[i].nonfinite;
       out.nclip += wp[i].nclip;
+      out.nrej += wp[i].nrej;
     }
   }
   return out;
@@ -238,15 +239,23 @@ __global__ void k_d3_partial(const float* __restrict__ lp, const float* __restri
 // One block per response (sequence-gate variant).  rho_i = mean of delta over the response's
 // scored rows, summed in a fixed order in float64; a response with |rho_i| > gate (or a
 // non-finite rho_i) is rejected: its rows get no loss and no gradient (token loss, g and the dH
-// rows set to 0).  Runs after the forward and before the reductions and dW.
+// rows set to 0).  The decision is written to rej[i] (0 or 1) for every response, and the
+// rejections are counted by k_reduce_parts in a fixed order.  Runs after the forward and before
+// the reductions and dW.
 __global__ void k_seq_gate(const int64_t* __restrict__ cprefix, const float* __restrict__ delta_c,
-                           const int32_t* __restrict__ rowmap, float gate, int H, Ctrl* ctrl,
+                           const int32_t* __restrict__ rowmap, float gate, int H, const Ctrl* ctrl,
                            float* __restrict__ g_c, float* __restrict__ tl_c, float* __restrict__ token_loss,
-                           uint16_t* __restrict__ grad_hidden) {
-  if (!ctrl->valid) return;
+                           uint16_t* __restrict__ grad_hidden, uint8_t* __restrict__ rej) {
   const int i = blockIdx.x;
+  if (!ctrl->valid) {
+    if (threadIdx.x == 0) rej[i] = 0;
+    return;
+  }
   const int64_t k0 = cprefix[i], k1 = cprefix[i + 1];
-  if (k1 <= k0) return;
+  if (k1 <= k0) {
+    if (threadIdx.x == 0) rej[i] = 0;
+    return;
+  }
   double part = 0.0;
   for (int64_t k = k0 + threadIdx.x; k < k1; k += blockDim.x) part += static_cast<double>(delta_c[k]);
   for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
@@ -259,7 +268,7 @@ __global__ void k_seq_gate(const int64_t* __restrict__ cprefix, const float* __r
     for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) tot += wsum[w];
     const double rho = tot / static_cast<double>(k1 - k0);
     reject = !(fabs(rho) <= static_cast<double>(gate));
-    if (reject) atomicAdd(&ctrl->n_rejected, 1);
+    rej[i] = reject ? 1 : 0;
   }
   __syncthreads();
   if (!reject) return;
@@ -287,9 +296,12 @@ struct D3Out {  // layout of bi_d3
   int32_t n_rejected;
 };
 
-__global__ void k_reduce_parts(const RedPart* __restrict__ parts, int nparts, float* loss, D3Out* d3,
-                               const Ctrl* ctrl, int32_t* status) {
+// `rej` (may be NULL): the sequence gate's per-response decisions, R of them.
+__global__ void k_reduce_parts(const RedPart* __restrict__ parts, int nparts, const uint8_t* __restrict__ rej, int R,
+                               float* loss, D3Out* d3, int32_t* status) {
   RedPart v = red_zero();
+  if (rej != nullptr)
+    for (int i = threadIdx.x; i < R; i += blockDim.x) v.nrej += rej[i];
   for (int i = threadIdx.x; i < nparts; i += blockDim.x) {
     const RedPart p = parts[i];
     v.loss += p.loss;
@@ -315,7 +327,7 @@ __global__ void k_reduce_parts(const RedPart* __restrict__ parts, int nparts, fl
       o.k1_mean = any ? static_cast<float>(b.k1sum / n) : 0.f;
       o.k2_mean = any ? static_cast<float>(b.k2sum / n) : 0.f;
       o.n_clipped = static_cast<int32_t>(b.nclip);
-      o.n_rejected = ctrl ? ctrl->n_rejected : 0;
+      o.n_rejected = static_cast<int32_t>(b.nrej);
       *d3 = o;
     }
     if (b.nonfinite > 0 || (loss && !isfinite(b.loss))) raise_status(status, 7 /* BI_ERR_NONFINITE */);
