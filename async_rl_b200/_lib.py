@@ -9,7 +9,7 @@ import os
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libbi_isloss.so")
 
-EXPORTED = ("bi_workspace_bytes", "bi_workspace_bytes_min", "bi_logprob_fwd", "bi_logprob_fwd_noalloc", "bi_is_loss_fwd_bwd", "bi_d3_stats",
+EXPORTED = ("bi_workspace_bytes", "bi_workspace_bytes_min", "bi_workspace_bytes_pstore", "bi_logprob_fwd", "bi_logprob_fwd_noalloc", "bi_is_loss_fwd_bwd", "bi_d3_stats",
             "bi_status_string", "bi_version", "bi_debug_force_timeout_once", "bi_profile_enable",
             "bi_profile_reset", "bi_profile_read", "bi_gemm_bf16", "bi_rmsnorm")
 
@@ -23,7 +23,10 @@ _lib = None
 class LossCfg(ctypes.Structure):
     """bi_loss_cfg"""
     _fields_ = [("variant", ctypes.c_int32), ("eps_low", ctypes.c_float), ("eps_high", ctypes.c_float),
-                ("gate", ctypes.c_float)]
+                ("gate", ctypes.c_float), ("flags", ctypes.c_int32)]
+
+
+LOSS_STORE_P = 1  # bi_loss_cfg.flags: BI_LOSS_STORE_P
 
 
 LOSS_VARIANTS = {"unclipped": 0, "ppo_clip": 1, "seq_gate": 2}
@@ -48,6 +51,8 @@ def load() -> ctypes.CDLL:
     lib.bi_workspace_bytes.restype = _sz
     lib.bi_workspace_bytes_min.argtypes = [_i64, _i32, _i32, _i32]
     lib.bi_workspace_bytes_min.restype = _sz
+    lib.bi_workspace_bytes_pstore.argtypes = [_i64, _i32, _i32, _i32]
+    lib.bi_workspace_bytes_pstore.restype = _sz
     lib.bi_logprob_fwd.argtypes = [_p, _p, _p, _i64, _i32, _i32, _p, _p, _p, _p, _sz, _p]
     lib.bi_logprob_fwd.restype = ctypes.c_int
     lib.bi_logprob_fwd_noalloc.argtypes = [_p, _p, _p, _i64, _i32, _i32, _p, _p, _p, _p]

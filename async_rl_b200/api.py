@@ -52,16 +52,20 @@ def _check_buffers(dev: torch.device, **named):
             raise ValueError(f"{name} must be contiguous")
 
 
-def workspace_bytes(T: int, H: int, V: int, R: int = 0, minimal: bool = False) -> int:
-    """Workspace of the fastest path, or (minimal=True) the smallest accepted one, whose dW
-    recomputes the logits instead of reading the stored probability tiles."""
+def workspace_bytes(T: int, H: int, V: int, R: int = 0, minimal: bool = False, pstore: bool = False) -> int:
+    """Workspace of the default path (nothing of size T x V), the smallest accepted one
+    (minimal=True), or the one of the opt-in P store (pstore=True, loss calls only), which keeps
+    every exponentiated logit tile of the forward in device memory."""
     lib = _lib.load()
+    if pstore:
+        return int(lib.bi_workspace_bytes_pstore(T, H, V, R))
     fn = lib.bi_workspace_bytes_min if minimal else lib.bi_workspace_bytes
     return int(fn(T, H, V, R))
 
 
-def make_workspace(T: int, H: int, V: int, R: int = 0, device="cuda", minimal: bool = False) -> torch.Tensor:
-    n = workspace_bytes(T, H, V, R, minimal)
+def make_workspace(T: int, H: int, V: int, R: int = 0, device="cuda", minimal: bool = False,
+                   pstore: bool = False) -> torch.Tensor:
+    n = workspace_bytes(T, H, V, R, minimal, pstore)
     return torch.empty(max(n, 256), dtype=torch.uint8, device=device)
 
 
@@ -107,7 +111,7 @@ class LossOutputs:
     logprob: torch.Tensor      # [T] f32
     is_weight: torch.Tensor    # [T] f32
     token_loss: torch.Tensor   # [T] f32
-    d3_raw: torch.Tensor       # [24] u8 (bi_d3)
+    d3_raw: torch.Tensor       # [40] u8 (bi_d3)
     grad_hidden: torch.Tensor  # [T, H] bf16
     grad_w: torch.Tensor       # [V, H] f32
     status: torch.Tensor       # [1] i32
@@ -125,12 +129,14 @@ class LossOutputs:
 def is_loss_fwd_bwd(hidden, w, targets, rollout_logprob, rewards, resp_offsets, group_offsets,
                     prompt_lens=None, resp_normalizer: float = 0.0, ws: Optional[torch.Tensor] = None,
                     out: Optional[LossOutputs] = None, variant: str = "unclipped", eps_low: float = 0.2,
-                    eps_high: float = 0.2, gate: float = float("inf")) -> LossOutputs:
+                    eps_high: float = 0.2, gate: float = float("inf"), pstore: bool = False) -> LossOutputs:
     """Fused forward + backward of the token-level IS REINFORCE loss (see the C header).
 
     ``variant`` is "unclipped" (the method), or one of the comparison baselines "ppo_clip"
     (clip range [1 - eps_low, 1 + eps_high]) and "seq_gate" (rejects responses whose mean token
-    log-ratio exceeds ``gate`` in absolute value)."""
+    log-ratio exceeds ``gate`` in absolute value).  ``pstore`` opts in to the P store (dW as a
+    GEMM over the stored exponentiated logit tiles; needs a ``workspace_bytes(..., pstore=True)``
+    workspace); by default nothing of size T x V is written to device memory."""
     dev = hidden.device
     T, H = hidden.shape
     V = w.shape[0]
@@ -147,13 +153,14 @@ def is_loss_fwd_bwd(hidden, w, targets, rollout_logprob, rewards, resp_offsets, 
         _check_cuda(prompt_lens, "prompt_lens", torch.int32, dev)
     lib = _lib.load()
     if ws is None:
-        ws = make_workspace(T, H, V, R, dev)
+        ws = make_workspace(T, H, V, R, dev, pstore=pstore)
     o = out if out is not None else LossOutputs.allocate(T, H, V, dev)
     _check_buffers(dev, ws=ws, loss=o.loss, logprob=o.logprob, is_weight=o.is_weight, token_loss=o.token_loss,
                    d3_raw=o.d3_raw, grad_hidden=o.grad_hidden, grad_w=o.grad_w, status=o.status)
     if variant not in _lib.LOSS_VARIANTS:
         raise ValueError(f"unknown loss variant {variant!r}")
-    cfg = _lib.LossCfg(_lib.LOSS_VARIANTS[variant], float(eps_low), float(eps_high), float(gate))
+    cfg = _lib.LossCfg(_lib.LOSS_VARIANTS[variant], float(eps_low), float(eps_high), float(gate),
+                       _lib.LOSS_STORE_P if pstore else 0)
     import ctypes
     code = lib.bi_is_loss_fwd_bwd(_ptr(hidden), _ptr(w), _ptr(targets), _ptr(rollout_logprob), _ptr(rewards),
                                   _ptr(resp_offsets), _ptr(group_offsets), _ptr(prompt_lens), R, G,

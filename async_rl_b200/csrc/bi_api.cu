@@ -25,7 +25,6 @@ using bi::Ctrl;
 using bi::RedPart;
 
 constexpr uint64_t kWaitLimitNs = 4000000000ull;  // 4 s for any single in-kernel wait
-constexpr size_t kZscanSmemMax = 160 * 1024;      // per-row scan of decode-style scoring
 constexpr int kMaxSms = 160;                      // upper bound used to size the dZ scratch
 constexpr int kDzSlotsMax = 2 * kMaxSms;          // clusters * C * slots-per-CTA <= 2 * SMs
 
@@ -35,11 +34,12 @@ thread_local uint64_t g_force_timeout_ns = 0;
 // optional per-kernel timing (events around each launch; measurement tools only)
 // ---------------------------------------------------------------------------------------------
 enum KernelKind : int { kKPrep, kKRowmap, kKZeroRows, kKGather, kKLmFwd, kKLmFwdDH, kKLmDW, kKDwRows,
-                        kKDwStream, kKSeqGate, kKRowParts, kKReduce, kKD3Partial, kKGemm, kKRmsNorm, kKLmZtiles, kKLmZscan, kNumKinds };
+                        kKDwStream, kKSeqGate, kKRowParts, kKReduce, kKD3Partial, kKGemm, kKRmsNorm, kKLmZtiles,
+                        kKLmZchain, kKLmZscan, kNumKinds };
 const char* const kKindNames[kNumKinds] = {"k_prep", "k_rowmap", "k_zero_prompt_rows", "k_gather_rows",
                                            "k_lm_fwd", "k_lm_fwd_dh", "k_lm_dw", "k_dw_rows", "k_dw_stream",
                                            "k_seq_gate", "k_row_parts", "k_reduce_parts", "k_d3_partial",
-                                           "k_gemm_pair", "k_rmsnorm", "k_lm_ztiles", "k_lm_zscan"};
+                                           "k_gemm_pair", "k_rmsnorm", "k_lm_ztiles", "k_lm_zchain", "k_lm_zscan"};
 static_assert(sizeof(bi::D3Out) == sizeof(bi_d3), "device-written diagnostics match the ABI struct");
 struct Pending {
   int kind;
@@ -89,10 +89,10 @@ struct ProfScope {  // records an event pair around one launch when profiling is
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct WsLayout {
-  size_t ctrl, lse_c, g_c, tl_c, d3_c, delta_c, clip_c, y_c, logmu_c, rowmap, respof, coef, cprefix, red, hc, dz,
-      alpha, fin;
+  size_t ctrl, lse_c, g_c, tl_c, d3_c, delta_c, clip_c, y_c, logmu_c, rowmap, respof, coef, cprefix, rej, red, hc,
+      dz, alpha, fin;
   size_t sxr_c, mhist, hs, pbuf;  // the P store (loss layout with the store only)
-  size_t zbuf, zmax;              // decode-style scoring (logprob layout, T <= 128 rows)
+  size_t ztmax, zmref, zcsum, zy; // decode-style scoring (logprob layout, T <= 128 rows)
   bool decode;
   size_t total;
   int nred;
@@ -105,8 +105,10 @@ constexpr size_t kFinBytes = static_cast<size_t>(kMaxSms) * 2 * 384 * sizeof(flo
 // `store`, followed by the P store of the fused forward ([Tpad][V + 256] bf16, enough for any
 // logit-tile width NZ <= 256), the per-step reference history ([ceil(V / 128)][Tpad] float) and
 // the scaled hidden states of the dW GEMM ([Tpad][H] bf16).
-// R == 0 with `decode` and 0 < T <= 128: followed by the logits of the few rows ([T][V + 256]
-// fp32) and their per-tile maxima ([T][ceil(V / 128)] fp32) for the all-SM scoring path.
+// R == 0 with `decode` and 0 < T <= 128: followed by what the all-SM scoring path keeps between
+// its two passes over W: per-tile row maxima and references ([ceil(V / 128)][T] fp32 each, enough
+// for any tile width NZ >= 128), 32-column partial sums ([T][V / 32 + 8] fp32 at most) and the
+// target logits ([T] fp32).  Nothing of size T x V.
 WsLayout ws_layout(int64_t T, int32_t H, int32_t V, int32_t R, bool store, bool decode = false) {
   WsLayout L{};
   const size_t t = static_cast<size_t>(T > 0 ? T : 1);
@@ -135,6 +137,7 @@ WsLayout ws_layout(int64_t T, int32_t H, int32_t V, int32_t R, bool store, bool 
     L.respof = take(t * 4);
     L.coef = take(static_cast<size_t>(R) * 8);
     L.cprefix = take(static_cast<size_t>(R + 1) * 8);
+    L.rej = take(static_cast<size_t>(R));
     L.nred = static_cast<int>(nred);
     L.red = take(static_cast<size_t>(L.nred) * sizeof(RedPart));
     L.hc = take(t * static_cast<size_t>(H) * 2);
@@ -151,8 +154,11 @@ WsLayout ws_layout(int64_t T, int32_t H, int32_t V, int32_t R, bool store, bool 
   }
   if (R == 0 && decode && T > 0 && T <= bi::kDecodeRows) {
     L.decode = true;
-    L.zbuf = take(t * (static_cast<size_t>(V) + 256) * 4);
-    L.zmax = take(t * static_cast<size_t>((V + 127) / 128) * 4);
+    const size_t ntile = static_cast<size_t>((V + 127) / 128);
+    L.ztmax = take(t * ntile * 4);
+    L.zmref = take(t * ntile * 4);
+    L.zcsum = take(t * (static_cast<size_t>(V + 31) / 32 + 8) * 4);
+    L.zy = take(t * 4);
   }
   L.total = o;
   return L;
@@ -285,18 +291,15 @@ bool set_lm_attributes() {
 #undef BI_SET_DW_ATTR
   ok = ok && cudaFuncSetAttribute(bi::k_gemm_pair, cudaFuncAttributeMaxDynamicSharedMemorySize, bi::kGemmSmem) ==
                  cudaSuccess;
-  ok = ok && cudaFuncSetAttribute(bi::k_lm_ztiles<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  bi::ZtTile<256>::smem) == cudaSuccess;
-  ok = ok && cudaFuncSetAttribute(bi::k_lm_ztiles<192>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  bi::ZtTile<192>::smem) == cudaSuccess;
-  ok = ok && cudaFuncSetAttribute(bi::k_lm_ztiles<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  bi::ZtTile<128>::smem) == cudaSuccess;
-  ok = ok && cudaFuncSetAttribute(bi::k_lm_zscan<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  static_cast<int>(kZscanSmemMax)) == cudaSuccess;
-  ok = ok && cudaFuncSetAttribute(bi::k_lm_zscan<192>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  static_cast<int>(kZscanSmemMax)) == cudaSuccess;
-  ok = ok && cudaFuncSetAttribute(bi::k_lm_zscan<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  static_cast<int>(kZscanSmemMax)) == cudaSuccess;
+#define BI_SET_ZT_ATTR(NZ_)                                                                                   \
+  ok = ok && cudaFuncSetAttribute(bi::k_lm_ztiles<NZ_, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,  \
+                                  bi::ZtTile<NZ_>::smem) == cudaSuccess;                                     \
+  ok = ok && cudaFuncSetAttribute(bi::k_lm_ztiles<NZ_, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,   \
+                                  bi::ZtTile<NZ_>::smem) == cudaSuccess;
+  BI_SET_ZT_ATTR(256)
+  BI_SET_ZT_ATTR(192)
+  BI_SET_ZT_ATTR(128)
+#undef BI_SET_ZT_ATTR
   return ok;
 }
 
@@ -447,13 +450,11 @@ bi_status logprob_forward(const uint16_t* hidden, const uint16_t* w_lm, const in
 constexpr int kDecodeUnsupported = -1;
 
 int logprob_decode(const uint16_t* hidden, const uint16_t* w_lm, const int32_t* targets, int64_t T, int32_t H,
-                   int32_t V, float* logprob, float* lse, int32_t* dev_status, float* zbuf, float* zmax,
+                   int32_t V, float* logprob, float* lse, int32_t* dev_status, uint8_t* ws, const WsLayout& L,
                    const DevInfo* di, cudaStream_t s) {
   const LmPlan pl = plan_lm(H, di);
   if (pl.C == 0 || pl.C > 8) return kDecodeUnsupported;
   const int nvz = (V + pl.NZ - 1) / pl.NZ;
-  const size_t zsm = bi::zscan_smem(nvz, pl.NZ);
-  if (zsm > kZscanSmemMax) return kDecodeUnsupported;
   CUtensorMap tm_h, tm_w;
   if (!make_map(&tm_h, hidden, T, H, 128) || !make_map(&tm_w, w_lm, V, H, pl.NZ)) return BI_ERR_CUDA;
   bi::ZtArgs a{};
@@ -461,28 +462,39 @@ int logprob_decode(const uint16_t* hidden, const uint16_t* w_lm, const int32_t* 
   a.V = V;
   a.nvz = nvz;
   a.KB = H / 64;
-  a.z = zbuf;
-  a.z_ld = static_cast<int64_t>(nvz) * pl.NZ;
-  a.tmax = zmax;
+  a.tmax = reinterpret_cast<float*>(ws + L.ztmax);
+  a.mref = reinterpret_cast<const float*>(ws + L.zmref);
+  a.csum = reinterpret_cast<float*>(ws + L.zcsum);
+  a.zy = reinterpret_cast<float*>(ws + L.zy);
+  a.y = targets;
   a.status = dev_status;
   a.limit_ns = kWaitLimitNs;
   const unsigned grid = static_cast<unsigned>(nvz < di->sms ? nvz : di->sms);
-  {
+  // pass 1 (tile maxima), the chain, pass 2 (chunk sums and target logits), the combine
+#define BI_ZT(NZ_, SUMS_) \
+  bi::k_lm_ztiles<NZ_, SUMS_><<<grid, bi::kZtThreads, bi::ZtTile<NZ_>::smem, s>>>(tm_h, tm_w, a)
+  for (int pass = 0; pass < 2; ++pass) {
+    if (pass == 1) {
+      ProfScope ps(kKLmZchain, s);
+      bi::k_lm_zchain<<<blocks_for(T, 128), 128, 0, s>>>(a.tmax, T, nvz, reinterpret_cast<float*>(ws + L.zmref));
+      if (cudaGetLastError() != cudaSuccess) return BI_ERR_CUDA;
+    }
     ProfScope ps(kKLmZtiles, s);
     switch (pl.NZ) {
-      case 256: bi::k_lm_ztiles<256><<<grid, bi::kZtThreads, bi::ZtTile<256>::smem, s>>>(tm_h, tm_w, a); break;
-      case 192: bi::k_lm_ztiles<192><<<grid, bi::kZtThreads, bi::ZtTile<192>::smem, s>>>(tm_h, tm_w, a); break;
-      case 128: bi::k_lm_ztiles<128><<<grid, bi::kZtThreads, bi::ZtTile<128>::smem, s>>>(tm_h, tm_w, a); break;
+      case 256: if (pass == 0) BI_ZT(256, false); else BI_ZT(256, true); break;
+      case 192: if (pass == 0) BI_ZT(192, false); else BI_ZT(192, true); break;
+      case 128: if (pass == 0) BI_ZT(128, false); else BI_ZT(128, true); break;
       default: return kDecodeUnsupported;
     }
     if (cudaGetLastError() != cudaSuccess) return BI_ERR_CUDA;
   }
+#undef BI_ZT
   ProfScope ps(kKLmZscan, s);
   const unsigned rows = static_cast<unsigned>(T);
   switch (pl.NZ) {
-    case 256: bi::k_lm_zscan<256><<<rows, bi::kZsThreads, zsm, s>>>(zbuf, a.z_ld, zmax, targets, T, V, nvz, pl.C, logprob, lse, dev_status); break;
-    case 192: bi::k_lm_zscan<192><<<rows, bi::kZsThreads, zsm, s>>>(zbuf, a.z_ld, zmax, targets, T, V, nvz, pl.C, logprob, lse, dev_status); break;
-    default:  bi::k_lm_zscan<128><<<rows, bi::kZsThreads, zsm, s>>>(zbuf, a.z_ld, zmax, targets, T, V, nvz, pl.C, logprob, lse, dev_status); break;
+    case 256: bi::k_lm_zscan<256><<<rows, bi::kZsThreads, 0, s>>>(a.csum, a.mref, a.zy, targets, T, V, nvz, pl.C, logprob, lse, dev_status); break;
+    case 192: bi::k_lm_zscan<192><<<rows, bi::kZsThreads, 0, s>>>(a.csum, a.mref, a.zy, targets, T, V, nvz, pl.C, logprob, lse, dev_status); break;
+    default:  bi::k_lm_zscan<128><<<rows, bi::kZsThreads, 0, s>>>(a.csum, a.mref, a.zy, targets, T, V, nvz, pl.C, logprob, lse, dev_status); break;
   }
   return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
 }
@@ -576,12 +588,17 @@ int32_t bi_profile_read(const char** names_out, double* ms_out, int64_t* launche
 
 size_t bi_workspace_bytes(int64_t T, int32_t H, int32_t V, int32_t R) {
   if (T < 0 || H <= 0 || V <= 0 || R < 0) return 0;
-  return ws_layout(T, H, V, R, R > 0, true).total;
+  return ws_layout(T, H, V, R, false, true).total;
 }
 
 size_t bi_workspace_bytes_min(int64_t T, int32_t H, int32_t V, int32_t R) {
   if (T < 0 || H <= 0 || V <= 0 || R < 0) return 0;
   return ws_layout(T, H, V, R, false).total;
+}
+
+size_t bi_workspace_bytes_pstore(int64_t T, int32_t H, int32_t V, int32_t R) {
+  if (T < 0 || H <= 0 || V <= 0 || R < 1) return 0;
+  return ws_layout(T, H, V, R, true).total;
 }
 
 bi_status bi_logprob_fwd(const uint16_t* hidden, const uint16_t* w_lm, const int32_t* targets, int64_t T, int32_t H,
@@ -603,9 +620,8 @@ bi_status bi_logprob_fwd(const uint16_t* hidden, const uint16_t* w_lm, const int
   // a few rows: the same bits from every SM when the workspace holds their logits
   const WsLayout Ld = ws_layout(T, H, V, 0, false, true);
   if (Ld.decode && ws_bytes >= Ld.total && force == 0) {
-    uint8_t* w8 = static_cast<uint8_t*>(ws);
-    const int r = logprob_decode(hidden, w_lm, targets, T, H, V, logprob, lse, dev_status,
-                                 reinterpret_cast<float*>(w8 + Ld.zbuf), reinterpret_cast<float*>(w8 + Ld.zmax), di, s);
+    const int r = logprob_decode(hidden, w_lm, targets, T, H, V, logprob, lse, dev_status, static_cast<uint8_t*>(ws),
+                                 Ld, di, s);
     if (r != kDecodeUnsupported) return static_cast<bi_status>(r);
   }
   float* fin = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + L.fin);
@@ -641,8 +657,9 @@ bi_status bi_is_loss_fwd_bwd(const uint16_t* hidden, const uint16_t* w_lm, const
                              int32_t* dev_status, void* ws, size_t ws_bytes, void* stream) {
   if (T < 0 || T >= (int64_t(1) << 31) || H <= 0 || V <= 0 || R < 1 || G < 1 || G > R) return BI_ERR_INVALID_ARG;
   if (!(resp_normalizer >= 0.0)) return BI_ERR_INVALID_ARG;
-  const bi_loss_cfg lc = cfg ? *cfg : bi_loss_cfg{BI_LOSS_UNCLIPPED, 0.f, 0.f, 0.f};
+  const bi_loss_cfg lc = cfg ? *cfg : bi_loss_cfg{BI_LOSS_UNCLIPPED, 0.f, 0.f, 0.f, 0};
   if (lc.variant < BI_LOSS_UNCLIPPED || lc.variant > BI_LOSS_SEQ_GATE) return BI_ERR_INVALID_ARG;
+  if ((lc.flags & ~BI_LOSS_STORE_P) != 0) return BI_ERR_INVALID_ARG;
   if (lc.variant == BI_LOSS_PPO_CLIP &&
       !(lc.eps_low >= 0.f && lc.eps_high >= 0.f && std::isfinite(lc.eps_low) && std::isfinite(lc.eps_high)))
     return BI_ERR_INVALID_ARG;
@@ -653,10 +670,11 @@ bi_status bi_is_loss_fwd_bwd(const uint16_t* hidden, const uint16_t* w_lm, const
   if (!aligned16(w_lm) || !aligned16(grad_w) || (T > 0 && (!aligned16(hidden) || !aligned16(grad_hidden))))
     return BI_ERR_INVALID_ARG;
   if (H % 64 != 0 || cluster_split(H) == 0) return BI_ERR_UNSUPPORTED_SHAPE;
-  // the full workspace keeps the P tiles for dW; the minimum one makes dW recompute the logits
-  const WsLayout Lfull = ws_layout(T, H, V, R, true);
-  const bool store = ws_bytes >= Lfull.total && dw_split(H) != 0;
-  const WsLayout L = store ? Lfull : ws_layout(T, H, V, R, false);
+  // dW recomputes the logits tile by tile unless the caller opted in to the P store, which keeps
+  // every exponentiated logit tile of the forward in the workspace for a GEMM-only dW
+  const bool store = (lc.flags & BI_LOSS_STORE_P) != 0;
+  if (store && dw_split(H) == 0) return BI_ERR_UNSUPPORTED_SHAPE;
+  const WsLayout L = ws_layout(T, H, V, R, store);
   if (!ws || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) return BI_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const DevInfo* di = device_info();
@@ -784,7 +802,7 @@ bi_status bi_is_loss_fwd_bwd(const uint16_t* hidden, const uint16_t* w_lm, const
         ProfScope ps(kKSeqGate, s);                                                                        \
         bi::k_seq_gate<<<R, 256, 0, s>>>(reinterpret_cast<const int64_t*>(w8 + L.cprefix), F(L.delta_c),  \
                                          I(L.rowmap), lc.gate, H, ctrl, F(L.g_c), F(L.tl_c), token_loss,  \
-                                         grad_hidden);                                                     \
+                                         grad_hidden, reinterpret_cast<uint8_t*>(w8 + L.rej));            \
       }                                                                                                    \
       {                                                                                                    \
         ProfScope ps(kKRowParts, s);                                                                       \
@@ -794,7 +812,9 @@ bi_status bi_is_loss_fwd_bwd(const uint16_t* hidden, const uint16_t* w_lm, const
       }                                                                                                    \
       {                                                                                                    \
         ProfScope ps(kKReduce, s);                                                                         \
-        bi::k_reduce_parts<<<1, 1024, 0, s>>>(parts, L.nred, loss, reinterpret_cast<bi::D3Out*>(d3), ctrl, \
+        const uint8_t* rej = (lc.variant == BI_LOSS_SEQ_GATE && T > 0)                                     \
+                                 ? reinterpret_cast<const uint8_t*>(w8 + L.rej) : nullptr;                 \
+        bi::k_reduce_parts<<<1, 1024, 0, s>>>(parts, L.nred, rej, R, loss, reinterpret_cast<bi::D3Out*>(d3), \
                                               dev_status);                                                 \
       }                                                                                                    \
       if (cudaGetLastError() != cudaSuccess) st = BI_ERR_CUDA;                                             \
@@ -836,8 +856,8 @@ bi_status bi_d3_stats(const float* learner_logprob, const float* rollout_logprob
                                                                            parts);
   }
   ProfScope ps(kKReduce, s);
-  bi::k_reduce_parts<<<1, 1024, 0, s>>>(parts, static_cast<int>(nred), nullptr, reinterpret_cast<bi::D3Out*>(out),
-                                        nullptr, dev_status);
+  bi::k_reduce_parts<<<1, 1024, 0, s>>>(parts, static_cast<int>(nred), nullptr, 0, nullptr,
+                                        reinterpret_cast<bi::D3Out*>(out), dev_status);
   return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
 }
 

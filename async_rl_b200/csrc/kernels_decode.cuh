@@ -1,21 +1,27 @@
 // kernels_decode.cuh -- log pi for a few rows (decode-style scoring, T <= 128) on every SM, with
-// the same bits as the cluster kernel (kernels_lm.cuh, kModeFwd).
+// the same bits as the cluster kernel (kernels_lm.cuh, kModeFwd), and nothing of size T x V in
+// memory.
 //
 // "Zero Mismatch, Simple Async RL", section "Alignment permits a simpler learning path": rollout
 // and learner logprobs bit-identical for the same weights and tokens, whether a row is scored
 // alone or packed.  The cluster kernel gives a one-row call the same bits as a packed one, but it
-// sweeps the whole vocabulary on one cluster.  Here the same arithmetic is spread over the GPU:
+// sweeps the whole vocabulary on one cluster.  Here the same arithmetic is spread over the GPU in
+// two passes over W; between them only per-tile maxima, references and 32-column partial sums
+// (1/32 of the logits) are kept:
 //
-// Phase 1 (k_lm_ztiles): one CTA per vocabulary tile j at a time computes z_j = H W_j^T for the
-//   128-row tile with the cluster kernel's instruction sequence (tcgen05 M = 128, N = NZ, K = H in
-//   64-column chunks of four K = 16 instructions, first without accumulate), and writes z (fp32)
-//   and the tile's row maximum M_j over the valid columns for the T real rows.
-// Phase 2 (k_lm_zscan, one block per row): the lazy reference chain m_j = (M_j > m_{j-1} + tau) ?
-//   M_j : m_{j-1}; every 32-column chunk sum cs = sum_q e^{z - m_j} (target column and columns
-//   past V excluded, q in order); per class k (steps j = k mod C) the partial sum with its rescale
-//   at each change of reference and the chunk sums added in order; the combine of the C classes
-//   in class order.  Each of these is the cluster kernel's epilogue expression for expression;
-//   only the chunk sums run in parallel, and they are independent there too.
+// Pass 1 (k_lm_ztiles<NZ, false>): one CTA per vocabulary tile j at a time computes z_j = H W_j^T
+//   for the 128-row tile with the cluster kernel's instruction sequence (tcgen05 M = 128, N = NZ,
+//   K = H in 64-column chunks of four K = 16 instructions, first without accumulate) and writes
+//   the tile's row maximum M_j over the valid columns for the T real rows.
+// Chain (k_lm_zchain, one thread per row): the lazy reference chain m_j = (M_j > m_{j-1} + tau) ?
+//   M_j : m_{j-1}, as the producers of consecutive steps pass it on.
+// Pass 2 (k_lm_ztiles<NZ, true>): the same tiles again; every 32-column chunk sum
+//   cs = sum_q e^{z - m_j} (target column and columns past V excluded, q in order) and the target
+//   logit, exactly as the cluster kernel's producer epilogue forms them.
+// Combine (k_lm_zscan, one block per row): per class k (steps j = k mod C) the partial sum with its
+//   rescale at each change of reference and the chunk sums added in order; then the combine of
+//   the C classes in class order.  Each of these is the cluster kernel's epilogue expression for
+//   expression.
 #pragma once
 
 #include "kernels_lm.cuh"
@@ -44,14 +50,16 @@ struct ZtShared {
 struct ZtArgs {
   int64_t T;        // real rows (<= 128)
   int32_t V, nvz, KB;
-  float* z;         // [T][z_ld] fp32 logits, z_ld = nvz * NZ
-  int64_t z_ld;
-  float* tmax;      // [T][nvz] row maximum of each tile over its valid columns
+  float* tmax;      // [nvz][T] row maximum of each tile over its valid columns (pass 1 writes)
+  const float* mref;  // [nvz][T] reference of each row at each step (pass 2 reads)
+  float* csum;      // [T][nvz][NZ / 32] 32-column chunk sums of e^{z - m_j} (pass 2 writes)
+  float* zy;        // [T] target logit (pass 2 writes, from the tile holding the target)
+  const int32_t* y; // [T] targets
   int32_t* status;
   uint64_t limit_ns;
 };
 
-template <int kNZ>
+template <int kNZ, bool kSums>
 __global__ void __launch_bounds__(kZtThreads, 1)
     k_lm_ztiles(const __grid_constant__ CUtensorMap tm_h, const __grid_constant__ CUtensorMap tm_w, ZtArgs a) {
   // tm_h: hidden [T][H], box {64, 128}; tm_w: W [V][H], box {64, NZ}; both 128-byte swizzled
@@ -156,30 +164,51 @@ __global__ void __launch_bounds__(kZtThreads, 1)
     const uint32_t tl = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     const bool warp_rows = static_cast<int64_t>(quarter * 32) < a.T;  // warp-uniform
     uint32_t tc = 0;
+    const bool real = row < a.T;
+    const int32_t yt = real ? a.y[row] : -1;
     for (int j = blockIdx.x; j < ntiles; j += gridDim.x, ++tc) {
       const uint32_t b = tc & 1u;
       if (!__all_sync(0xffffffffu, mbar_wait<false>(&sh.z_full[b], (tc >> 1) & 1u, wc))) break;
       tc_fence_after();
       if (warp_rows) {
-        const bool real = row < a.T;
-        float* zr = a.z + (real ? row : 0) * a.z_ld + static_cast<int64_t>(j) * kNZ;
-        float M = -INFINITY;
+        if (!kSums) {
+          // pass 1: the tile's row maximum over the valid columns (the producer's first pass)
+          float M = -INFINITY;
 #pragma unroll 1
-        for (int c = 0; c < kNZ / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld32(tl + b * 256u + c * 32, v);
-          tmem_ld_wait();
-          const int vb = j * kNZ + c * 32;
+          for (int c = 0; c < kNZ / 32; ++c) {
+            uint32_t v[32];
+            tmem_ld32(tl + b * 256u + c * 32, v);
+            tmem_ld_wait();
+            const int vb = j * kNZ + c * 32;
 #pragma unroll
-          for (int q = 0; q < 32; ++q)
-            if (vb + q < a.V) M = fmaxf(M, __uint_as_float(v[q]));
-          if (real) {
-            uint4* d4 = reinterpret_cast<uint4*>(zr + c * 32);
+            for (int q = 0; q < 32; ++q)
+              if (vb + q < a.V) M = fmaxf(M, __uint_as_float(v[q]));
+          }
+          if (real) a.tmax[static_cast<int64_t>(j) * a.T + row] = M;
+        } else {
+          // pass 2: chunk sums against the step's reference, and the target logit (the
+          // producer's second pass)
+          const float mn2 = (real ? a.mref[static_cast<int64_t>(j) * a.T + row] : 0.f) * kLog2e;
+          float* cs_out = a.csum + (static_cast<int64_t>(real ? row : 0) * a.nvz + j) * (kNZ / 32);
+#pragma unroll 1
+          for (int c = 0; c < kNZ / 32; ++c) {
+            uint32_t v[32];
+            tmem_ld32(tl + b * 256u + c * 32, v);
+            tmem_ld_wait();
+            const int vb = j * kNZ + c * 32;
+            float cs = 0.f;
 #pragma unroll
-            for (int q = 0; q < 8; ++q) d4[q] = make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+            for (int q = 0; q < 32; ++q) {
+              const float z = __uint_as_float(v[q]);
+              const bool tgt = (vb + q == yt);
+              const bool in = (vb + q < a.V) && !tgt;
+              const float pr = in ? ex2_approx(fmaf(z, kLog2e, -mn2)) : 0.f;
+              cs += pr;
+              if (tgt && real) a.zy[row] = z;
+            }
+            if (real) cs_out[c] = cs;
           }
         }
-        if (real) a.tmax[static_cast<int64_t>(row) * a.nvz + j] = M;
       }
       tc_fence_before();
       mbar_arrive(&sh.z_empty[b]);
@@ -199,87 +228,54 @@ __global__ void __launch_bounds__(kZtThreads, 1)
   }
 }
 
-constexpr int kZsThreads = 1024;
-
-// Dynamic shared memory of k_lm_zscan: the references and the chunk sums of one row.
-__host__ __device__ constexpr size_t zscan_smem(int nvz, int nz) {
-  return static_cast<size_t>(nvz) * 4 + static_cast<size_t>(nvz) * (nz / 32) * 4 + 2 * 8 * 4;
+// One thread per row: the reference chain from the tile maxima, in step order.
+__global__ void k_lm_zchain(const float* __restrict__ tmax, int64_t T, int nvz, float* __restrict__ mref) {
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (t >= T) return;
+  float mprev = -INFINITY;
+#pragma unroll 4
+  for (int j = 0; j < nvz; ++j) {
+    const float M = tmax[static_cast<int64_t>(j) * T + t];
+    const float mnew = (M > mprev + kTau) ? M : mprev;
+    mref[static_cast<int64_t>(j) * T + t] = mnew;
+    mprev = mnew;
+  }
 }
 
+constexpr int kZsThreads = 32;
+
+// One block (one warp) per row: the class partial sums and their combine.
 template <int kNZ>
 __global__ void __launch_bounds__(kZsThreads)
-    k_lm_zscan(const float* __restrict__ z, int64_t z_ld, const float* __restrict__ tmax, const int32_t* __restrict__ y,
-               int64_t T, int V, int nvz, int C, float* __restrict__ logprob, float* __restrict__ lse_out,
-               int32_t* status) {
+    k_lm_zscan(const float* __restrict__ csum, const float* __restrict__ mref, const float* __restrict__ zyb,
+               const int32_t* __restrict__ y, int64_t T, int V, int nvz, int C, float* __restrict__ logprob,
+               float* __restrict__ lse_out, int32_t* status) {
   constexpr int kChunks = kNZ / 32;
-  extern __shared__ float zs[];
-  float* mref = zs;                                     // [nvz] reference after each step
-  float* csum = zs + nvz;                               // [nvz][kChunks] chunk sums
-  float* cls = csum + static_cast<int64_t>(nvz) * kChunks;  // [8] class reference, [8] class sum
+  __shared__ float cls[2 * 8];  // [8] class reference, [8] class sum
   const int64_t t = blockIdx.x;
   if (t >= T) return;
-  const float* zrow = z + t * z_ld;
-  const int32_t yt = y[t];
-  // the chain (as the producers of consecutive steps pass it on), from the tile maxima staged in
-  // shared memory
-  for (int j = threadIdx.x; j < nvz; j += kZsThreads) mref[j] = tmax[t * nvz + j];
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float mprev = -INFINITY;
-#pragma unroll 8
-    for (int j = 0; j < nvz; ++j) {
-      const float M = mref[j];
-      const float mnew = (M > mprev + kTau) ? M : mprev;
-      mref[j] = mnew;
-      mprev = mnew;
-    }
-  }
-  __syncthreads();
-  // every 32-column chunk: e^{z - m_j} summed in column order, the target column excluded
-  for (int idx = threadIdx.x; idx < nvz * kChunks; idx += kZsThreads) {
-    const int j = idx / kChunks;
-    const int c = idx - j * kChunks;
-    const float mn2 = mref[j] * kLog2e;
-    const int vb = j * kNZ + c * 32;
-    float zv[32];
-    const float4* z4 = reinterpret_cast<const float4*>(zrow + vb);
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const float4 f = __ldg(z4 + q);
-      zv[4 * q] = f.x;
-      zv[4 * q + 1] = f.y;
-      zv[4 * q + 2] = f.z;
-      zv[4 * q + 3] = f.w;
-    }
-    float cs = 0.f;
-#pragma unroll
-    for (int q = 0; q < 32; ++q) {
-      const bool tgt = (vb + q == yt);
-      const bool in = (vb + q < V) && !tgt;
-      const float pr = in ? ex2_approx(fmaf(zv[q], kLog2e, -mn2)) : 0.f;
-      cs += pr;
-    }
-    csum[idx] = cs;
-  }
-  __syncthreads();
+  const float* crow = csum + t * static_cast<int64_t>(nvz) * kChunks;
   // class k: its steps in order, rescaled at each change of reference
-  if (threadIdx.x < C) {
+  if (static_cast<int>(threadIdx.x) < C) {
     const int k = threadIdx.x;
     float mp = -INFINITY, sp = 0.f;
-#pragma unroll 4
+#pragma unroll 2
     for (int j = k; j < nvz; j += C) {
-      const float mnew = mref[j];
+      const float mnew = mref[static_cast<int64_t>(j) * T + t];
       if (mnew != mp) {
         sp = (mp == -INFINITY) ? 0.f : sp * ex2_approx((mp - mnew) * kLog2e);
         mp = mnew;
       }
+      float cv[kChunks];
 #pragma unroll
-      for (int c = 0; c < kChunks; ++c) sp += csum[j * kChunks + c];
+      for (int c = 0; c < kChunks; ++c) cv[c] = crow[j * kChunks + c];
+#pragma unroll
+      for (int c = 0; c < kChunks; ++c) sp += cv[c];
     }
     cls[k] = mp;
     cls[8 + k] = sp;
   }
-  __syncthreads();
+  __syncwarp();
   if (threadIdx.x == 0) {
     float mstar = -INFINITY;
     for (int k = 0; k < C; ++k) mstar = fmaxf(mstar, cls[k]);
@@ -288,10 +284,11 @@ __global__ void __launch_bounds__(kZsThreads)
       const float mq = cls[k];
       if (mq != -INFINITY) s_ex = fmaf(cls[8 + k], ex2_approx((mq - mstar) * kLog2e), s_ex);
     }
+    const int32_t yt = y[t];
     const bool ybad = yt < 0 || yt >= V;
     float lp = __int_as_float(0x7fc00000), lse = __int_as_float(0x7fc00000);
     if (!ybad) {
-      const float zy = zrow[yt];
+      const float zy = zyb[t];
       const float s = s_ex + ex2_approx(fmaf(zy, kLog2e, -mstar * kLog2e));
       lse = mstar + logf(s);
       lp = zy - lse;

@@ -13,7 +13,8 @@
  *       kernel mismatch comes from batch composition, prefill/decode paths and float ordering.
  *
  * Definitions computed by the library (T rows, hidden size H, vocabulary V):
- *   z_t     = W h_t                          (LM-head logits; never written to memory)
+ *   z_t     = W h_t                          (LM-head logits; never written to memory unless the
+ *                                            caller opts in to the P store, BI_LOSS_STORE_P)
  *   lse_t   = log sum_v exp(z_tv)
  *   logpi_t = z_{t,y_t} - lse_t
  *   w_t     = exp(logpi_t - logmu_t)         (no clipping)
@@ -66,7 +67,7 @@ typedef enum {
   BI_OK = 0,
   BI_ERR_INVALID_ARG = 1,       /* NULL pointer, negative size, misaligned pointer */
   BI_ERR_UNSUPPORTED_SHAPE = 2, /* H not supported (see above) */
-  BI_ERR_WORKSPACE = 3,         /* ws == NULL or ws_bytes < bi_workspace_bytes_min(...) */
+  BI_ERR_WORKSPACE = 3,         /* ws == NULL or ws_bytes below the size the call needs */
   BI_ERR_CUDA = 4,              /* a CUDA runtime call or launch failed */
   BI_ERR_TIMEOUT = 5,           /* device: a bounded wait ran out */
   BI_ERR_BAD_TARGET = 6,        /* device: a target id outside [0, V) */
@@ -108,32 +109,45 @@ typedef struct {
  *                      gradient) when its mean token log-ratio rho_i = mean_t (log pi_t - log mu_t)
  *                      has |rho_i| > gate or is not finite; it still counts in R*. */
 typedef enum { BI_LOSS_UNCLIPPED = 0, BI_LOSS_PPO_CLIP = 1, BI_LOSS_SEQ_GATE = 2 } bi_loss_variant;
+
+/* bi_loss_cfg.flags.  BI_LOSS_STORE_P opts in to the P store: the forward writes every bf16 tile
+ * e^{z - m} of the exponentiated logits to the workspace (about 2 T (V + 384) bytes, 23 GB for
+ * T = 76,000 rows of a 151,936-token vocabulary; size from bi_workspace_bytes_pstore) and dW is
+ * one GEMM over those tiles instead of a second pass over the logits.  This MATERIALISES THE
+ * T x V LOGITS (as probabilities) IN DEVICE MEMORY; without the flag nothing of size T x V is
+ * ever written.  Both paths give the same bits for every output except grad_w, where they differ
+ * by rounding only. */
+#define BI_LOSS_STORE_P 1
+
 typedef struct {
   int32_t variant;  /* bi_loss_variant */
   float eps_low;    /* PPO_CLIP: >= 0 */
   float eps_high;   /* PPO_CLIP: >= 0 */
   float gate;       /* SEQ_GATE: >= 0 (may be +inf) */
+  int32_t flags;    /* 0 or BI_LOSS_STORE_P; other bits: BI_ERR_INVALID_ARG */
 } bi_loss_cfg;
 
 /* Size in bytes of the scratch workspace for these sizes (R = number of responses; pass 0 for
  * bi_logprob_fwd / bi_d3_stats).  Deterministic and free of side effects; the caller allocates
  * the workspace (256-byte aligned) and may reuse it across calls on the same stream.
- * For bi_is_loss_fwd_bwd this is the workspace of the fastest path: besides O(T) per-row arrays
- * it holds every bf16 probability tile of the forward (about 2 T (V + 384) bytes, 23 GB for
- * T = 76,000 rows of a 151,936-token vocabulary), so that dW is one GEMM over stored tiles instead
- * of a second pass over the logits.
- * For bi_logprob_fwd with 1 <= T <= 128 rows (decode-style scoring) it also holds the rows' fp32
- * logits (about 4 T (V + 256) bytes), so that the call runs on every SM instead of one cluster;
- * the bits are the same either way. */
+ * Nothing in it has T x V entries.  For bi_is_loss_fwd_bwd it holds O(T) per-row arrays, a compact
+ * copy of the scored hidden rows (T H bf16), per-response coefficients and a fixed-size scratch for
+ * the tiles the cluster passes between its CTAs; dW recomputes the logits tile by tile.
+ * For bi_logprob_fwd with 1 <= T <= 128 rows (decode-style scoring) it also holds what the all-SM
+ * path keeps between its two passes over W: per-tile row maxima and references and 32-column
+ * partial sums of e^{z - m} (about 4 T V / 32 bytes at most), so that the call runs on every SM
+ * instead of one cluster; the bits are the same either way. */
 BI_API size_t bi_workspace_bytes(int64_t T, int32_t H, int32_t V, int32_t R);
 
-/* Smallest workspace bi_is_loss_fwd_bwd accepts (O(T H) bytes).  Any ws_bytes from this size up
- * to just below bi_workspace_bytes(...) selects the low-memory path, whose dW kernel recomputes
- * the logits (about a third more tensor work per step).  Both paths produce the same bits for
- * every output except grad_w, where they differ by rounding only.  For R = 0 it is the per-CTA
- * partials only; bi_logprob_fwd accepts it for any T (with T <= 128 it then scores the rows on one
- * cluster, with the same bits). */
+/* Smallest workspace accepted.  For bi_is_loss_fwd_bwd it equals bi_workspace_bytes.  For R = 0 it
+ * is the per-CTA partials only: bi_logprob_fwd accepts it for any T (with T <= 128 it then scores
+ * the rows on one cluster, with the same bits). */
 BI_API size_t bi_workspace_bytes_min(int64_t T, int32_t H, int32_t V, int32_t R);
+
+/* Workspace of bi_is_loss_fwd_bwd with BI_LOSS_STORE_P in cfg->flags (R >= 1; 0 otherwise): the
+ * default workspace plus the P store, the per-step reference history ([ceil(V / 128)][T'] float)
+ * and the scaled hidden states of the dW GEMM ([T'][H] bf16), T' = T rounded up to 128. */
+BI_API size_t bi_workspace_bytes_pstore(int64_t T, int32_t H, int32_t V, int32_t R);
 
 /* Token log-probabilities log pi(y_t | h_t) under the LM head W (definition above).
  *   hidden   [T, H] bf16      rows to score (row-major, 16-byte aligned)
@@ -144,10 +158,11 @@ BI_API size_t bi_workspace_bytes_min(int64_t T, int32_t H, int32_t V, int32_t R)
  * A row gets identical bits whether it is scored alone (T = 1, decode style) or packed.  Packed
  * batches run on the cluster kernel (one cluster sweeps the vocabulary for each 128-row tile).
  * With 1 <= T <= 128 and a workspace of bi_workspace_bytes(T, H, V, 0) bytes the rows are scored
- * on every SM instead: the logit tiles with the cluster kernel's instruction sequence, then the
- * reference chain, the class partial sums and their combine in the cluster kernel's order, which
- * reproduces its bits ("Zero Mismatch, Simple Async RL", section "Alignment permits a simpler
- * learning path"). */
+ * on every SM instead, in two passes over W: the logit tiles with the cluster kernel's
+ * instruction sequence give the per-tile row maxima, then the reference chain, then the same
+ * tiles again give the 32-column partial sums against each step's reference, and the class sums
+ * and their combine follow the cluster kernel's order, which reproduces its bits ("Zero Mismatch,
+ * Simple Async RL", section "Alignment permits a simpler learning path"). */
 BI_API bi_status bi_logprob_fwd(const uint16_t* hidden, const uint16_t* w_lm, const int32_t* targets,
                          int64_t T, int32_t H, int32_t V, float* logprob, float* lse,
                          int32_t* dev_status, void* ws, size_t ws_bytes, void* stream);
@@ -186,7 +201,9 @@ BI_API bi_status bi_logprob_fwd_noalloc(const uint16_t* hidden, const uint16_t* 
  *                               scored (0 <= prompt_lens[i] <= its length)
  *   resp_normalizer  R* in c_i = A_i / (R* n_i); 0 means R.  Data-parallel callers pass the
  *                               global number of responses.
- *   cfg              (may be NULL: BI_LOSS_UNCLIPPED) host pointer, read during the call
+ *   cfg              (may be NULL: BI_LOSS_UNCLIPPED, no flags) host pointer, read during the
+ *                               call; with BI_LOSS_STORE_P in cfg->flags ws_bytes must be at least
+ *                               bi_workspace_bytes_pstore(T, H, V, R), else BI_ERR_WORKSPACE
  * Outputs (device):
  *   loss        [1]    float   L (sum over scored tokens in a fixed order, float64 accumulation)
  *   logprob     [T]    float   log pi_t on scored rows, 0 on prompt rows

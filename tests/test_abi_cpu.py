@@ -62,13 +62,18 @@ def test_workspace_bytes(lib):
     assert lib.bi_workspace_bytes(-1, 128, 512, 0) == 0
     # the compact copy of the hidden states is part of the loss workspace
     assert d - c >= 1000 * 1536 * 2
-    # the full loss workspace stores the bf16 probability tiles (T x (V + 256) rounded to 128 rows);
-    # the minimum one does not, and the logprob-only one is its own minimum
+    # the default loss workspace is O(T H + R): nothing of size T x V; it is also the minimum
     lo = lib.bi_workspace_bytes_min(2000, 1536, 151936, 64)
-    assert d - lo >= 2048 * 151936 * 2 and lo < 2000 * 1536 * 2 * 4 + (64 << 20)
+    assert lo == d and d < 2000 * 1536 * 2 * 4 + (64 << 20)
+    # the opt-in P store holds the bf16 probability tiles (T x (V + 256) rounded to 128 rows)
+    ps = lib.bi_workspace_bytes_pstore(2000, 1536, 151936, 64)
+    assert ps - d >= 2048 * 151936 * 2
+    assert lib.bi_workspace_bytes_pstore(2000, 1536, 151936, 0) == 0
     assert lib.bi_workspace_bytes_min(2000, 1536, 151936, 0) == b
-    # up to 128 rows the logprob workspace also holds the rows' logits for the all-SM path
-    assert lib.bi_workspace_bytes(128, 1536, 151936, 0) >= 128 * (151936 + 256) * 4
+    # up to 128 rows the logprob workspace also holds the all-SM path's per-tile maxima, references
+    # and 32-column partial sums: about 1/32 of the rows' logits, never the logits themselves
+    dec = lib.bi_workspace_bytes(128, 1536, 151936, 0)
+    assert b < dec < b + 128 * 151936 * 4 // 16
     assert lib.bi_workspace_bytes_min(128, 1536, 151936, 0) == b
 
 
@@ -125,8 +130,14 @@ def test_is_loss_argument_checks(lib):
     bad_gate = _lib.LossCfg(2, 0.2, 0.2, float("nan"))
     assert call(cfg=ctypes.addressof(bad_gate)) == 1
     ws_min = lib.bi_workspace_bytes_min(T, H, V, R)
-    assert 0 < ws_min < ws_bytes
+    assert 0 < ws_min == ws_bytes
     assert call(ws_bytes=ws_min - 1) == 3
+    # the opt-in P store with a default-size workspace, and unknown flag bits
+    store = _lib.LossCfg(0, 0.0, 0.0, 0.0, _lib.LOSS_STORE_P)
+    assert call(cfg=ctypes.addressof(store)) == 3
+    assert lib.bi_workspace_bytes_pstore(T, H, V, R) > ws_bytes
+    bad_flags = _lib.LossCfg(0, 0.0, 0.0, 0.0, 4)
+    assert call(cfg=ctypes.addressof(bad_flags)) == 1
 
 
 def test_d3_argument_checks(lib):

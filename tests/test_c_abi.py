@@ -20,9 +20,9 @@ C_SOURCE = r"""
 int main(void) {
   if (bi_version() <= 0) return 1;
   if (strcmp(bi_status_string(BI_ERR_BAD_OFFSETS), "BI_ERR_BAD_OFFSETS") != 0) return 2;
-  size_t full = bi_workspace_bytes(2000, 1536, 151936, 64);
-  size_t small = bi_workspace_bytes_min(2000, 1536, 151936, 64);
-  if (!(full > small && small > 0)) return 3;
+  size_t full = bi_workspace_bytes_pstore(2000, 1536, 151936, 64);
+  size_t small = bi_workspace_bytes(2000, 1536, 151936, 64);
+  if (!(full > small && small > 0 && small == bi_workspace_bytes_min(2000, 1536, 151936, 64))) return 3;
   if (bi_workspace_bytes(-1, 128, 512, 0) != 0) return 4;
   /* argument checks return before any CUDA call */
   const uint16_t* fake = (const uint16_t*)(uintptr_t)(1u << 20);
@@ -31,7 +31,7 @@ int main(void) {
   if (bi_rmsnorm(fake, fake, -1.0f, (uint16_t*)(uintptr_t)(1u << 22), 4, 64, st, NULL) != BI_ERR_INVALID_ARG) return 6;
   if (bi_logprob_fwd(NULL, fake, (const int32_t*)fake, 10, 128, 512, (float*)fake, NULL, st, (void*)fake, 1u << 20,
                      NULL) != BI_ERR_INVALID_ARG) return 7;
-  bi_loss_cfg cfg = {BI_LOSS_PPO_CLIP, 0.2f, 0.2f, 0.0f};
+  bi_loss_cfg cfg = {BI_LOSS_PPO_CLIP, 0.2f, 0.2f, 0.0f, BI_LOSS_STORE_P};
   (void)cfg;
   printf("ok %zu %zu\n", full, small);
   return 0;

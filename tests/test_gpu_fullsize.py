@@ -1,4 +1,5 @@
-"""Parity at the full sizes of the three loss workloads, in the launch configuration bench.py times:
+"""Parity at the full sizes of the three loss workloads, in the launch configuration bench.py times
+(the default path; the 1.5B shape also on the opt-in P store):
 
 * 1.5B shape: H = 1536, V = 151936, 8 x 8 responses of U[256, 2048] rows (T = 76,239);
 * 8K reasoning budget: H = 1536, 4 x 8 responses of U[1024, 8192] rows (about 147K rows);
@@ -22,22 +23,25 @@ from .util import GRAD_TOL, LOGPROB_TOL, assert_close, assert_grad_close, f64
 
 pytestmark = pytest.mark.gpu
 
-FULL_CONFIGS = ["qwen1.5b", "reason8k", "qwen4b_lag64"]
+# every workload on the default path (nothing of size T x V in memory; dW recomputes the logits),
+# and the 1.5B shape once more on the opt-in P store
+FULL_CASES = [("qwen1.5b", False), ("reason8k", False), ("qwen4b_lag64", False), ("qwen1.5b", True)]
 
 
-@pytest.fixture(scope="module", params=FULL_CONFIGS)
+@pytest.fixture(scope="module", params=FULL_CASES, ids=lambda c: c[0] + ("-pstore" if c[1] else ""))
 def full(request, cuda_device):
     from async_rl_b200.build import build
     build()
-    b = make_batch(spec_for(request.param), with_w_roll=False)
+    name, pstore = request.param
+    b = make_batch(spec_for(name), with_w_roll=False)
     gen = torch.Generator().manual_seed(4242)
     mu = (torch.randn(b.n_rows, generator=gen) * 0.3 - 12.0).to(torch.float32)
     d = b.to(cuda_device)
     out = bi.is_loss_fwd_bwd(d.hidden, d.w, d.targets, mu.to(cuda_device), d.rewards, d.resp_offsets,
-                             d.group_offsets, d.prompt_lens)
+                             d.group_offsets, d.prompt_lens, pstore=pstore)
     torch.cuda.synchronize()
     bi.check_status(out.status)
-    state = {"name": request.param, "b": b, "mu": mu, "d": d, "out": out}
+    state = {"name": name, "pstore": pstore, "b": b, "mu": mu, "d": d, "out": out}
     yield state
     state.clear()
     del d, out
@@ -95,7 +99,7 @@ def test_fullsize_diff_zero(full, cuda_device):
     b, d = full["b"], full["d"]
     lp, _, st = bi.logprob_fwd(d.hidden, d.w, d.targets)
     out = bi.is_loss_fwd_bwd(d.hidden, d.w, d.targets, lp, d.rewards, d.resp_offsets, d.group_offsets,
-                             d.prompt_lens)
+                             d.prompt_lens, pstore=full["pstore"])
     torch.cuda.synchronize()
     bi.check_status(st)
     bi.check_status(out.status)

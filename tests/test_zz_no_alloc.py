@@ -56,6 +56,26 @@ def test_noalloc_matches_workspace_entry_point_on_consecutive_calls(cuda_device)
         assert torch.isfinite(lp).all()
 
 
+def test_noalloc_matches_decode_sized_calls_and_null_lse(cuda_device):
+    """Decode-sized calls (T = 1 and T = 128): bi_logprob_fwd with its default workspace scores them
+    on every SM in two passes, the no-allocation entry point on the cluster kernel; the header
+    promises the same bits.  Then a call with lse = NULL must give the same logprob bits."""
+    lib = _lib.load()
+    for (T, seed) in [(1, 41), (128, 42)]:
+        h, w, y = random_inputs(T, 1536, 151936, seed)
+        h, w, y = h.to(cuda_device), w.to(cuda_device), y.to(cuda_device)
+        code, lp, lse, st = _call_noalloc(lib, h, w, y)
+        assert code == 0, _lib.STATUS_NAMES.get(code, code)
+        rcode, rlp, rlse, rst = _call_with_workspace(lib, h, w, y)
+        assert rcode == 0
+        code2, lp2, lse2, st2 = _call_noalloc(lib, h, w, y, want_lse=False)
+        assert code2 == 0 and lse2 is None
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0 and int(rst.item()) == 0 and int(st2.item()) == 0
+        assert torch.equal(lp, rlp) and torch.equal(lse, rlse)
+        assert torch.equal(lp2, lp)
+
+
 def test_noalloc_refuses_unsupported_shape_without_launching(cuda_device):
     lib = _lib.load()
     T, H = 16, 704  # no column split of H = 704 over <= 8 CTAs has 64-multiple slices

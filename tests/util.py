@@ -38,6 +38,35 @@ def assert_grad_close(name, got, ref, tol=GRAD_TOL):
                              f"first {i.tolist()} got {got.ravel()[i].tolist()} ref {ref.ravel()[i].tolist()}")
 
 
+def diag_bounds(lp_gpu, lp_ref, logmu, mask) -> dict:
+    """Absolute error bounds of the D3 mean and the k1 / k2 means of one call, propagated from the
+    measured per-row log-probability errors through the arithmetic the kernels use.
+
+    Per scored row the device forms delta = fl32(lp - log mu) (log mu is the same fp32 value on
+    both sides), so |delta_gpu - delta| <= e_t + 2^-24 |delta|, e_t = |lp_gpu - lp_ref|.  Then
+      * d3 = expm1f(delta) - delta: first order |expm1(delta)| |d delta|, plus expm1f's error
+        (<= 2 ulp of expm1) and the rounding of the subtraction, <= 2^-21 (|expm1 delta| + |delta|);
+        the cancellation in expm1(delta) - delta is why the bound is absolute, not relative;
+      * k1 = -delta: |d delta|;
+      * k2 = delta^2 / 2 (formed in fp64 from the fp32 delta): |delta| |d delta| + |d delta|^2 / 2.
+    The means are summed in fp64 and rounded to fp32 once (2^-24 of the result).  The factor 2 in
+    front of the first-order terms covers the second-order terms of the expansion."""
+    m = np.asarray(mask, dtype=bool)
+    e = np.abs(np.asarray(lp_gpu, np.float64)[m] - np.asarray(lp_ref, np.float64)[m])
+    delta = np.asarray(lp_ref, np.float64)[m] - np.asarray(logmu, np.float64)[m]
+    dd = e + 2.0 ** -24 * np.abs(delta)
+    em1 = np.abs(np.expm1(delta))
+    n = max(1, int(m.sum()))
+    d3 = np.expm1(delta) - delta
+    k2 = 0.5 * delta * delta
+    return {
+        "d3": 2.0 * float(np.sum(em1 * dd)) / n + 2.0 ** -21 * float(np.sum(em1 + np.abs(delta))) / n
+              + 2.0 ** -24 * abs(float(np.mean(d3))) + 1e-30,
+        "k1": 2.0 * float(np.sum(dd)) / n + 2.0 ** -24 * abs(float(np.mean(delta))) + 1e-30,
+        "k2": 2.0 * float(np.sum(np.abs(delta) * dd + 0.5 * dd * dd)) / n + 2.0 ** -24 * float(np.mean(k2)) + 1e-30,
+    }
+
+
 def to_dev(batch, device):
     b = batch.to(device)
     return b
