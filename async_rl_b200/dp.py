@@ -53,6 +53,24 @@ def local_slices(resp_offsets, group_offsets, g0: int, g1: int):
     return row0, row1, r0, r1, loff, lgoff
 
 
+def shard_of(resp_offsets, group_offsets, prompt_lens, world: int, rank: int):
+    """This rank's whole-group shard of a global batch: (row0, row1, r0, r1, local_resp_offsets,
+    local_group_offsets), from ``shard_by_groups`` then ``local_slices``."""
+    g0, g1 = shard_by_groups(resp_offsets, group_offsets, prompt_lens, world)[rank]
+    return local_slices(resp_offsets, group_offsets, g0, g1)
+
+
+def pin_collectives(env=None) -> dict:
+    """Fix NCCL's all-reduce algorithm and protocol (unless the caller already chose them), so that
+    the dW sum over ranks takes the same reduction order on every step and every run.  Must run
+    before the first NCCL communicator is created.  Returns the settings in force."""
+    import os
+    env = os.environ if env is None else env
+    env.setdefault("NCCL_ALGO", "Ring")
+    env.setdefault("NCCL_PROTO", "Simple")
+    return {"NCCL_ALGO": env["NCCL_ALGO"], "NCCL_PROTO": env["NCCL_PROTO"]}
+
+
 def allreduce_step(dist, grad_w, loss, group=None) -> None:
     """Sum dW and the loss over the ranks (the one exchange step of data parallelism)."""
     dist.all_reduce(grad_w, group=group)

@@ -9,8 +9,18 @@ steps.  Prints one JSON line (rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload loss|dense]
 
-N > 1 runs one process per GPU (torchrun): each rank scores its own batch (weak scaling) and the
-ranks sum dW and the three loss/D3 scalars with NCCL, the one exchange step of data parallelism.
+The default line runs the path that never writes anything of size T x V to device memory: the
+fused forward + dH kernel, then the dW kernel that recomputes the logits tile by tile.  The opt-in
+P store (every exponentiated logit tile kept in a 23 GB workspace, dW as one GEMM over it) is
+timed beside it as the extra key "pstore_opt_in" at N = 1.
+
+N > 1 runs one process per GPU (bench.py re-launches itself under torchrun when WORLD_SIZE is not
+set).  One global batch of N sub-batches of the workload is drawn on every rank; each rank scores
+its whole-group shard (dp.shard_by_groups) with R* = the global number of responses (weak scaling:
+about one sub-batch per rank), and the ranks sum dW and the loss with NCCL (algorithm and protocol
+pinned), the one exchange step of data parallelism.
+
+--dry-run checks that plumbing on CPU (gloo ranks, the tiny workload, no kernels).
 
 --workload dense times the batch-invariant dense layers instead (not the default line): one step is
 RMSNorm of the 1.5B-shape hidden states [76239, 1536] followed by the gate/up projection
@@ -51,11 +61,34 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--small", action="store_true",
-                    help="profiling case: same head, 4 responses of 1024 rows (T=4096); not a bench line")
+                    help="profiling case: same head, 4 responses of 1408 rows (T=5632: two full rounds of "
+                         "22 clusters); not a bench line")
     ap.add_argument("--workload", choices=["loss", "dense", "decode"], default="loss",
                     help="loss: the fused LM-head step (default line); dense: RMSNorm + linear layer; "
                          "decode: one-row logprob scoring latency")
+    ap.add_argument("--dry-run", action="store_true",
+                    help="CPU check of the multi-rank plumbing (gloo, tiny workload, no GPU kernels)")
+    ap.add_argument("--no-pstore", action="store_true", help="skip the opt-in P-store comparison key")
     return ap.parse_args()
+
+
+def relaunch_if_needed(args):
+    """--gpus N > 1 without a torchrun environment: run this script again as N ranks (torchrun on
+    127.0.0.1, bounded by `timeout`).  Under torchrun, refuse a world size other than --gpus."""
+    if "WORLD_SIZE" not in os.environ:
+        if args.gpus > 1:
+            import socket
+            with socket.socket() as sk:
+                sk.bind(("127.0.0.1", 0))
+                port = sk.getsockname()[1]
+            cmd = ["timeout", "-k", "60", "3600", sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+                   f"--nproc-per-node={args.gpus}", "--master-addr", "127.0.0.1", "--master-port", str(port),
+                   os.path.abspath(__file__)] + sys.argv[1:]
+            os.execvp(cmd[0], cmd)
+        return
+    world = int(os.environ["WORLD_SIZE"])
+    if world != args.gpus:
+        raise SystemExit(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world}")
 
 
 def dist_env():
@@ -74,25 +107,35 @@ def measured_peaks():
     return {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}, "fallback"
 
 
-TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "dram_traffic_qwen1.5b_step.md")
+TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "dram_traffic_small_T5632.md")
 CSRC_HASHED = ("sm100.cuh", "kernels_lm.cuh", "kernels_dw.cuh", "kernels_small.cuh", "bi_api.cu")
 
 
-def recorded_traffic(kernel: str):
-    """DRAM bytes per launch of `kernel` from the committed full-size ncu record, or None when the
-    CUDA sources changed since that capture (the record carries their sha256)."""
+def sources_hash() -> str:
     import hashlib
-    if not os.path.exists(TRAFFIC_RECORD):
-        return None
     h = hashlib.sha256()
     for f in CSRC_HASHED:
         with open(os.path.join(ROOT, "async_rl_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(kernel: str, T: int, H: int):
+    """DRAM bytes per launch of `kernel` at T rows, scaled from the committed small-case ncu record
+    (`traffic <kernel> <bytes per launch> <T_small> <sha256 of the CUDA sources>`), or None when the
+    sources changed since that capture.  The forward + dH kernel reads W once per round of
+    clusters and the hidden rows once, and writes dH once: the bytes beyond 4 T H (hidden in, dH
+    out) are scaled by T (the number of 128-row units, hence of rounds), the 4 T H part is exact."""
+    if not os.path.exists(TRAFFIC_RECORD) or kernel != "k_lm_fwd_dh":
+        return None
+    digest = sources_hash()
     with open(TRAFFIC_RECORD) as fh:
         for ln in fh:
             parts = ln.split()
-            if len(parts) == 4 and parts[0] == "traffic" and parts[1] == kernel and parts[3] == h.hexdigest():
-                return int(parts[2])
+            if len(parts) == 5 and parts[0] == "traffic" and parts[1] == kernel and parts[4] == digest:
+                small, t_small = int(parts[2]), int(parts[3])
+                per_row_fixed = 4.0 * H
+                return int((small - per_row_fixed * t_small) * T / t_small + per_row_fixed * T)
     return None
 
 
@@ -214,28 +257,75 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def local_shard(gb, world, rank):
+    """This rank's whole-group shard of the global batch (a Batch of its own rows and responses)
+    and the global number of responses R*."""
+    from async_rl_b200.dp import shard_of
+    from workloads import Batch
+    pl = None if gb.prompt_lens is None else gb.prompt_lens.cpu()
+    row0, row1, r0, r1, loff, lgoff = shard_of(gb.resp_offsets.cpu(), gb.group_offsets.cpu(), pl, world, rank)
+    dev = gb.hidden.device
+    b = Batch(gb.spec, gb.hidden[row0:row1].contiguous(), gb.w, gb.w_roll, gb.targets[row0:row1].contiguous(),
+              gb.rewards[r0:r1].contiguous(), torch.as_tensor(loff, device=dev), torch.as_tensor(lgoff, device=dev),
+              None if gb.prompt_lens is None else gb.prompt_lens[r0:r1].contiguous(),
+              gb.logmu_noise[row0:row1].contiguous())
+    return b, gb.R, (row0, row1)
+
+
+def run_dry(args):
+    """--dry-run: the multi-rank plumbing on CPU with gloo: the global tiny batch, each rank's
+    whole-group shard, R*, the pinned collective settings and one all-reduce; no GPU kernels."""
+    import datetime
+    import torch.distributed as dist
+    from async_rl_b200.dp import pin_collectives
+    from workloads import make_global_batch, spec_for
+    rank, world, _ = dist_env()
+    pinned = pin_collectives()
+    if world > 1:
+        dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+    gb = make_global_batch(spec_for("tiny"), world)
+    b, rstar, rows = local_shard(gb, world, rank)
+    tok = torch.tensor([float(b.n_rows)], dtype=torch.float64)
+    shards = [rows]
+    if world > 1:
+        dist.all_reduce(tok)
+        shards = [None] * world
+        dist.all_gather_object(shards, rows)
+    if rank == 0:
+        print(json.dumps({"dry_run": True, "metric": METRIC, "n_gpus": world, "global_rows": gb.n_rows,
+                          "rows_all_ranks": int(tok.item()), "resp_normalizer": rstar, "shards": shards,
+                          "collectives": pinned}), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def run_ours(args):
     rank, world, local = dist_env()
     import async_rl_b200 as bi
     from async_rl_b200.build import build
-    from async_rl_b200.dp import allreduce_step
-    from workloads import make_batch, spec_for
+    from async_rl_b200.dp import allreduce_step, pin_collectives
+    from workloads import make_global_batch, spec_for
 
     if rank == 0:
         build()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     pg = None
+    pinned = None
     if world > 1:
         import datetime
         import torch.distributed as dist
+        pinned = pin_collectives()
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
         dist.barrier()
         pg = dist
     spec = spec_for(CONFIG)
     if args.small:
-        spec = spec_for(CONFIG, groups=1, per_group=4, len_lo=1024, len_hi=1024)
-    b = make_batch(spec, seed=1234 + spec.index + 1000 * rank, device=dev)
+        spec = spec_for(CONFIG, groups=1, per_group=4, len_lo=1408, len_hi=1408)
+    gb = make_global_batch(spec, world, device=dev)
+    b, rstar, _ = local_shard(gb, world, rank)
+    del gb
     T, H, V, R = b.n_rows, spec.H, spec.V, b.R
     # rollout log-probabilities from the lagged head (the rollout engine's role), plus noise rows
     logmu, _, st = bi.logprob_fwd(b.hidden, b.w_roll, b.targets)
@@ -244,7 +334,7 @@ def run_ours(args):
     b.w_roll = None
     ws = bi.make_workspace(T, H, V, R, dev)
     out = bi.LossOutputs.allocate(T, H, V, dev)
-    rnorm = float(R * world)
+    rnorm = float(rstar)
 
     def step():
         bi.is_loss_fwd_bwd(b.hidden, b.w, b.targets, logmu, b.rewards, b.resp_offsets, b.group_offsets,
@@ -347,6 +437,35 @@ def run_ours(args):
         e2e = {"value": total_tokens / (float(ems.item()) * 1e-3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h), "h2d": "pinned host buffers, prefetched one step ahead on a copy stream"}
 
+    # the opt-in P store beside it (N = 1 only): same batch, its own 23 GB workspace
+    pstore = None
+    if world == 1 and not args.no_pstore:
+        ws_p = bi.make_workspace(T, H, V, R, dev, pstore=True)
+        out_p = bi.LossOutputs.allocate(T, H, V, dev)
+
+        def pstep():
+            bi.is_loss_fwd_bwd(b.hidden, b.w, b.targets, logmu, b.rewards, b.resp_offsets, b.group_offsets,
+                               None, rnorm, ws=ws_p, out=out_p, pstore=True)
+
+        for _ in range(args.warmup):
+            pstep()
+        torch.cuda.synchronize()
+        n_p = min(args.steps, 5)
+        p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        p0.record()
+        for _ in range(n_p):
+            pstep()
+        p1.record()
+        torch.cuda.synchronize()
+        bi.check_status(out_p.status)
+        pms = p0.elapsed_time(p1) / n_p
+        pstore = {"ms_per_step": pms, "tokens_per_s": T / (pms * 1e-3), "steps": n_p,
+                  "workspace_gb": ws_p.numel() / 1e9,
+                  "note": "opt-in BI_LOSS_STORE_P: every exponentiated logit tile kept in device memory "
+                          "(materialises T x V), dW as one GEMM over it; not the headline"}
+        del ws_p, out_p
+        torch.cuda.empty_cache()
+
     peaks, peak_src = measured_peaks()
     peak_tf = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
     flops_tvh = 2.0 * T * V * H  # one LM-head contraction over the batch
@@ -369,17 +488,26 @@ def run_ours(args):
             "config": {"workload": f"{CONFIG}: H={H} V={V}, {spec.groups}x{spec.per_group} responses "
                                    f"U[{spec.len_lo},{spec.len_hi}] rows, T={T} scored rows per rank",
                        "global_batch_tokens": int(total_tokens), "parallelism": f"dp{world}",
+                       "path": "default: no T x V array in device memory (dW recomputes the logits)",
+                       "workspace_gb": ws.numel() / 1e9,
+                       "sharding": "whole groups of one global batch (shard_by_groups), R* = global responses",
+                       "collectives": pinned,
                        "l2": "inputs larger than L2 (hidden 0.23 GB, W 0.47 GB); no flush"},
             "pct_bf16_peak": 100.0 * step_tflops / peak_tf,
             "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak_tf,
                          "unit": "TFLOP/s", "frac": achieved / peak_tf,
-                         "traffic": recorded_traffic(dom) if (CONFIG == "qwen1.5b" and not args.small) else None,
+                         "traffic": recorded_traffic(dom, T, H) if (CONFIG == "qwen1.5b" and not args.small) else None,
+                         "traffic_source": "ncu small case (T=5632) scaled to this launch by T; null when the "
+                                           "CUDA sources changed since the capture",
                          "peak_source": f"{peak_src} bf16_tflops_sustained",
                          "algorithmic_flops_per_launch": alg[dom],
                          "executed_frac": executed[dom] / (davg * 1e-3) / 1e12 / peak_tf},
             "step_roofline": {"achieved": step_tflops, "frac": step_tflops / peak_tf,
                               "algorithmic_flops": 6.0 * T * V * H, "unit": "TFLOP/s"},
             "kernels": kernels, "gpu_launches": launches, "clocks": clk, "e2e": e2e}
+    if pstore is not None:
+        pstore["pct_bf16_peak"] = 100.0 * 6.0 * T * V * H / (pstore["ms_per_step"] * 1e-3) / 1e12 / peak_tf
+        line["pstore_opt_in"] = pstore
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_oracle_sample(b, logmu.cpu().double().numpy(), CPU_SAMPLE_ROWS)
     if rank == 0:
@@ -681,6 +809,10 @@ def run_decode(args):
 
 def main():
     args = parse()
+    relaunch_if_needed(args)
+    if args.dry_run:
+        run_dry(args)
+        return
     if args.workload == "decode":
         if args.impl == "reference":
             run_decode_reference(args)

@@ -24,18 +24,22 @@ def bench():
     return m
 
 
-def test_traffic_record_needs_matching_sources(bench, tmp_path, monkeypatch):
-    import hashlib
-    h = hashlib.sha256()
-    for f in bench.CSRC_HASHED:
-        with open(os.path.join(ROOT, "async_rl_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+def test_traffic_record_needs_matching_sources_and_scales_by_rows(bench, tmp_path, monkeypatch):
+    digest = bench.sources_hash()
     rec = tmp_path / "rec.md"
-    rec.write_text(f"    traffic k_lm_fwd_dh 123456 {h.hexdigest()}\n    traffic k_dw_stream 99 {'0' * 64}\n")
+    H = 1536
+    small_T = 5632
+    small = 1_000_000_000 + 4 * H * small_T   # W part + hidden in / dH out
+    rec.write_text(f"    traffic k_lm_fwd_dh {small} {small_T} {digest}\n"
+                   f"    traffic k_lm_dw 99 {small_T} {'0' * 64}\n")
     monkeypatch.setattr(bench, "TRAFFIC_RECORD", str(rec))
-    assert bench.recorded_traffic("k_lm_fwd_dh") == 123456
-    assert bench.recorded_traffic("k_dw_stream") is None      # captured on other sources
-    assert bench.recorded_traffic("k_gemm_pair") is None      # never captured
+    # the per-row part is exact, the rest scales with the rows (rounds of clusters)
+    assert bench.recorded_traffic("k_lm_fwd_dh", small_T, H) == small
+    assert bench.recorded_traffic("k_lm_fwd_dh", 2 * small_T, H) == 2_000_000_000 + 4 * H * 2 * small_T
+    assert bench.recorded_traffic("k_lm_dw", small_T, H) is None      # not modelled (and other sources)
+    assert bench.recorded_traffic("k_gemm_pair", small_T, H) is None  # never captured
+    rec.write_text(f"    traffic k_lm_fwd_dh {small} {small_T} {'1' * 64}\n")
+    assert bench.recorded_traffic("k_lm_fwd_dh", small_T, H) is None  # captured on other sources
 
 
 def test_sub_batch_covers_whole_groups_of_the_first_rows(bench):

@@ -168,6 +168,32 @@ def make_batch(spec: ConfigSpec, seed: Optional[int] = None, device="cpu",
                  None if prompt_lens is None else prompt_lens.to(device), noise)
 
 
+def make_global_batch(spec: ConfigSpec, world: int, seed: Optional[int] = None, device="cpu") -> Batch:
+    """The batch of a data-parallel step on ``world`` ranks: ``world`` sub-batches of ``spec``
+    (sub-batch k drawn by ``make_batch`` with seed + 1000 k) packed one after another, sharing the
+    LM heads of sub-batch 0.  With world = 1 it is ``make_batch(spec, seed)`` itself, so the
+    per-GPU workload stays the same as the number of ranks grows."""
+    seed = 1234 + spec.index if seed is None else seed
+    subs = []
+    for k in range(world):
+        b = make_batch(spec, seed=seed + 1000 * k, device=device, with_w_roll=(k == 0))
+        subs.append(b if k == 0 else dataclasses.replace(b, w=None, w_roll=None))
+    if world == 1:
+        return subs[0]
+    row_base, resp_base = 0, 0
+    offs, goffs, plens = [torch.zeros(1, dtype=torch.int64, device=device)], [torch.zeros(1, dtype=torch.int32, device=device)], []
+    for b in subs:
+        offs.append(b.resp_offsets[1:] + row_base)
+        goffs.append(b.group_offsets[1:] + resp_base)
+        if b.prompt_lens is not None:
+            plens.append(b.prompt_lens)
+        row_base += b.n_rows
+        resp_base += b.R
+    cat = lambda name: torch.cat([getattr(b, name) for b in subs])
+    return Batch(spec, cat("hidden"), subs[0].w, subs[0].w_roll, cat("targets"), cat("rewards"),
+                 torch.cat(offs), torch.cat(goffs), torch.cat(plens) if plens else None, cat("logmu_noise"))
+
+
 def random_inputs(T: int, H: int, V: int, seed: int, w_std: float = 0.02, device="cpu"):
     """Plain (hidden, W, targets) triple for shape sweeps: h ~ N(0,1), W ~ N(0,w_std)."""
     gen = torch.Generator(device=device)
