@@ -25,6 +25,7 @@ using bi::Ctrl;
 using bi::RedPart;
 
 constexpr uint64_t kWaitLimitNs = 4000000000ull;  // 4 s for any single in-kernel wait
+constexpr size_t kZscanSmemMax = 200 * 1024;      // one row's partial sums in the decode combine
 constexpr int kMaxSms = 160;                      // upper bound used to size the dZ scratch
 constexpr int kDzSlotsMax = 2 * kMaxSms;          // clusters * C * slots-per-CTA <= 2 * SMs
 
@@ -34,12 +35,12 @@ thread_local uint64_t g_force_timeout_ns = 0;
 // optional per-kernel timing (events around each launch; measurement tools only)
 // ---------------------------------------------------------------------------------------------
 enum KernelKind : int { kKPrep, kKRowmap, kKZeroRows, kKGather, kKLmFwd, kKLmFwdDH, kKLmDW, kKDwRows,
-                        kKDwStream, kKSeqGate, kKRowParts, kKReduce, kKD3Partial, kKGemm, kKRmsNorm, kKLmZtiles,
-                        kKLmZchain, kKLmZscan, kNumKinds };
+                        kKDwStream, kKSeqGate, kKRowParts, kKReduce, kKD3Partial, kKGemm, kKRmsNorm, kKLmZscan,
+                        kKLmDecode1, kNumKinds };
 const char* const kKindNames[kNumKinds] = {"k_prep", "k_rowmap", "k_zero_prompt_rows", "k_gather_rows",
                                            "k_lm_fwd", "k_lm_fwd_dh", "k_lm_dw", "k_dw_rows", "k_dw_stream",
                                            "k_seq_gate", "k_row_parts", "k_reduce_parts", "k_d3_partial",
-                                           "k_gemm_pair", "k_rmsnorm", "k_lm_ztiles", "k_lm_zchain", "k_lm_zscan"};
+                                           "k_gemm_pair", "k_rmsnorm", "k_lm_zscan", "k_lm_decode1"};
 static_assert(sizeof(bi::D3Out) == sizeof(bi_d3), "device-written diagnostics match the ABI struct");
 struct Pending {
   int kind;
@@ -92,7 +93,7 @@ struct WsLayout {
   size_t ctrl, lse_c, g_c, tl_c, d3_c, delta_c, clip_c, y_c, logmu_c, rowmap, respof, coef, cprefix, rej, red, hc,
       dz, alpha, fin;
   size_t sxr_c, mhist, hs, pbuf;  // the P store (loss layout with the store only)
-  size_t ztmax, zmref, zcsum, zy; // decode-style scoring (logprob layout, T <= 128 rows)
+  size_t zmref, zcsum, zy, zsmax, zprog;  // decode-style scoring (logprob layout, T <= 128)
   bool decode;
   size_t total;
   int nred;
@@ -105,10 +106,10 @@ constexpr size_t kFinBytes = static_cast<size_t>(kMaxSms) * 2 * 384 * sizeof(flo
 // `store`, followed by the P store of the fused forward ([Tpad][V + 256] bf16, enough for any
 // logit-tile width NZ <= 256), the per-step reference history ([ceil(V / 128)][Tpad] float) and
 // the scaled hidden states of the dW GEMM ([Tpad][H] bf16).
-// R == 0 with `decode` and 0 < T <= 128: followed by what the all-SM scoring path keeps between
-// its two passes over W: per-tile row maxima and references ([ceil(V / 128)][T] fp32 each, enough
-// for any tile width NZ >= 128), 32-column partial sums ([T][V / 32 + 8] fp32 at most) and the
-// target logits ([T] fp32).  Nothing of size T x V.
+// R == 0 with `decode` and 0 < T <= 128: followed by what the all-SM scoring path keeps: per-tile
+// references ([ceil(V / 128)][T] fp32, enough for any tile width NZ >= 128), 32-column partial
+// sums ([T][V / 32 + 8] fp32 at most), the target logits ([T] fp32), the row maxima of 64-column
+// sub-tiles ([T][V / 64 + 4] fp32 at most) and one progress flag per SM.  Nothing of size T x V.
 WsLayout ws_layout(int64_t T, int32_t H, int32_t V, int32_t R, bool store, bool decode = false) {
   WsLayout L{};
   const size_t t = static_cast<size_t>(T > 0 ? T : 1);
@@ -155,10 +156,11 @@ WsLayout ws_layout(int64_t T, int32_t H, int32_t V, int32_t R, bool store, bool 
   if (R == 0 && decode && T > 0 && T <= bi::kDecodeRows) {
     L.decode = true;
     const size_t ntile = static_cast<size_t>((V + 127) / 128);
-    L.ztmax = take(t * ntile * 4);
     L.zmref = take(t * ntile * 4);
     L.zcsum = take(t * (static_cast<size_t>(V + 31) / 32 + 8) * 4);
     L.zy = take(t * 4);
+    L.zsmax = take(t * (static_cast<size_t>(V + 63) / 64 + 4) * 4);
+    L.zprog = take(static_cast<size_t>(kMaxSms) * 4);
   }
   L.total = o;
   return L;
@@ -232,6 +234,7 @@ struct DevInfo {
   bool ready = false;
   bool ok = false;
   int sms = 0;
+  bool coop = false;                                // one k_lm_decode1 CTA fits on every SM, cooperatively
   int max_clusters[3][bi::kMaxCluster + 1] = {};  // [mode][C]
   int gemm_clusters = 0;                            // resident CTA pairs of the GEMM kernel
 };
@@ -291,15 +294,18 @@ bool set_lm_attributes() {
 #undef BI_SET_DW_ATTR
   ok = ok && cudaFuncSetAttribute(bi::k_gemm_pair, cudaFuncAttributeMaxDynamicSharedMemorySize, bi::kGemmSmem) ==
                  cudaSuccess;
-#define BI_SET_ZT_ATTR(NZ_)                                                                                   \
-  ok = ok && cudaFuncSetAttribute(bi::k_lm_ztiles<NZ_, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,  \
-                                  bi::ZtTile<NZ_>::smem) == cudaSuccess;                                     \
-  ok = ok && cudaFuncSetAttribute(bi::k_lm_ztiles<NZ_, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,   \
-                                  bi::ZtTile<NZ_>::smem) == cudaSuccess;
-  BI_SET_ZT_ATTR(256)
-  BI_SET_ZT_ATTR(192)
-  BI_SET_ZT_ATTR(128)
-#undef BI_SET_ZT_ATTR
+  ok = ok && cudaFuncSetAttribute(bi::k_lm_decode1<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  bi::kD1Smem) == cudaSuccess;
+  ok = ok && cudaFuncSetAttribute(bi::k_lm_decode1<192>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  bi::kD1Smem) == cudaSuccess;
+  ok = ok && cudaFuncSetAttribute(bi::k_lm_decode1<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  bi::kD1Smem) == cudaSuccess;
+  ok = ok && cudaFuncSetAttribute(bi::k_lm_zscan<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(kZscanSmemMax)) == cudaSuccess;
+  ok = ok && cudaFuncSetAttribute(bi::k_lm_zscan<192>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(kZscanSmemMax)) == cudaSuccess;
+  ok = ok && cudaFuncSetAttribute(bi::k_lm_zscan<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(kZscanSmemMax)) == cudaSuccess;
   return ok;
 }
 
@@ -335,6 +341,11 @@ const DevInfo* device_info() {
     d.max_clusters[bi::kModeDW][c] = query_clusters<bi::kModeDW>(c);
   }
   d.gemm_clusters = query_gemm_clusters();
+  int coop_attr = 0, per_sm = 0;
+  d.coop = cudaDeviceGetAttribute(&coop_attr, cudaDevAttrCooperativeLaunch, dev) == cudaSuccess && coop_attr != 0 &&
+           cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, bi::k_lm_decode1<256>, bi::kZtThreads,
+                                                         bi::kD1Smem) == cudaSuccess &&
+           per_sm >= 1;
   cudaGetLastError();
   d.ok = d.sms > 0 && d.sms <= kMaxSms;
   return d.ok ? &d : nullptr;
@@ -443,58 +454,68 @@ bi_status logprob_forward(const uint16_t* hidden, const uint16_t* w_lm, const in
   return st;
 }
 
-// Decode-style scoring (T <= 128 rows) on every SM: the logit tiles of the rows with the cluster
-// kernel's instruction sequence, then the chain, the class sums and the combine of its epilogue,
-// expression for expression (kernels_decode.cuh).  The same plan (C, NZ) as the cluster kernel,
-// so the same bits.  Returns kDecodeUnsupported when the shape needs the cluster kernel.
+// Decode-style scoring (T <= 128 rows) on every SM (kernels_decode.cuh): one cooperative pass over
+// W that leaves per-sub-tile row maxima, each step's reference and 32-column partial sums, then the
+// per-row combine in the cluster kernel's order.  The same plan (C, NZ) as the cluster kernel, so
+// the same bits.  Returns kDecodeUnsupported when the rows should go to the cluster kernel (no
+// cooperative launch on this device, or a shape the combine does not hold in shared memory).
 constexpr int kDecodeUnsupported = -1;
 
 int logprob_decode(const uint16_t* hidden, const uint16_t* w_lm, const int32_t* targets, int64_t T, int32_t H,
                    int32_t V, float* logprob, float* lse, int32_t* dev_status, uint8_t* ws, const WsLayout& L,
                    const DevInfo* di, cudaStream_t s) {
   const LmPlan pl = plan_lm(H, di);
-  if (pl.C == 0 || pl.C > 8) return kDecodeUnsupported;
+  if (pl.C == 0 || pl.C > 8 || !di->coop || pl.NZ % bi::kD1Sub != 0) return kDecodeUnsupported;
   const int nvz = (V + pl.NZ - 1) / pl.NZ;
-  CUtensorMap tm_h, tm_w;
-  if (!make_map(&tm_h, hidden, T, H, 128) || !make_map(&tm_w, w_lm, V, H, pl.NZ)) return BI_ERR_CUDA;
-  bi::ZtArgs a{};
-  a.T = T;
-  a.V = V;
-  a.nvz = nvz;
-  a.KB = H / 64;
-  a.tmax = reinterpret_cast<float*>(ws + L.ztmax);
-  a.mref = reinterpret_cast<const float*>(ws + L.zmref);
-  a.csum = reinterpret_cast<float*>(ws + L.zcsum);
-  a.zy = reinterpret_cast<float*>(ws + L.zy);
-  a.y = targets;
-  a.status = dev_status;
-  a.limit_ns = kWaitLimitNs;
-  const unsigned grid = static_cast<unsigned>(nvz < di->sms ? nvz : di->sms);
-  // pass 1 (tile maxima), the chain, pass 2 (chunk sums and target logits), the combine
-#define BI_ZT(NZ_, SUMS_) \
-  bi::k_lm_ztiles<NZ_, SUMS_><<<grid, bi::kZtThreads, bi::ZtTile<NZ_>::smem, s>>>(tm_h, tm_w, a)
-  for (int pass = 0; pass < 2; ++pass) {
-    if (pass == 1) {
-      ProfScope ps(kKLmZchain, s);
-      bi::k_lm_zchain<<<blocks_for(T, 128), 128, 0, s>>>(a.tmax, T, nvz, reinterpret_cast<float*>(ws + L.zmref));
-      if (cudaGetLastError() != cudaSuccess) return BI_ERR_CUDA;
-    }
-    ProfScope ps(kKLmZtiles, s);
+  const size_t zsm = bi::zscan_smem(nvz, pl.NZ);
+  if (zsm > kZscanSmemMax) return kDecodeUnsupported;
+  CUtensorMap tm_h, tm_w64;
+  if (!make_map(&tm_h, hidden, T, H, 128) || !make_map(&tm_w64, w_lm, V, H, bi::kD1Sub)) return BI_ERR_CUDA;
+  const int nsub = nvz * (pl.NZ / bi::kD1Sub);
+  const int G = nsub < di->sms ? nsub : di->sms;  // >= NZ / 64 sub-tiles: every wait has a finite target
+  bi::D1Args d{};
+  d.T = T;
+  d.V = V;
+  d.nvz = nvz;
+  d.KB = H / 64;
+  d.nsub = nsub;
+  d.rounds = (nsub + G - 1) / G;
+  d.smax = reinterpret_cast<float*>(ws + L.zsmax);
+  d.mref = reinterpret_cast<float*>(ws + L.zmref);
+  d.csum = reinterpret_cast<float*>(ws + L.zcsum);
+  d.zy = reinterpret_cast<float*>(ws + L.zy);
+  d.y = targets;
+  d.progress = reinterpret_cast<uint32_t*>(ws + L.zprog);
+  d.status = dev_status;
+  d.limit_ns = kWaitLimitNs;
+  if (cudaMemsetAsync(d.progress, 0, static_cast<size_t>(G) * 4, s) != cudaSuccess) return BI_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(G), 1, 1);
+  cfg.blockDim = dim3(bi::kZtThreads, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(bi::kD1Smem);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaErrorInvalidValue;
+  {
+    ProfScope ps(kKLmDecode1, s);
     switch (pl.NZ) {
-      case 256: if (pass == 0) BI_ZT(256, false); else BI_ZT(256, true); break;
-      case 192: if (pass == 0) BI_ZT(192, false); else BI_ZT(192, true); break;
-      case 128: if (pass == 0) BI_ZT(128, false); else BI_ZT(128, true); break;
-      default: return kDecodeUnsupported;
+      case 256: e = cudaLaunchKernelEx(&cfg, bi::k_lm_decode1<256>, tm_h, tm_w64, d); break;
+      case 192: e = cudaLaunchKernelEx(&cfg, bi::k_lm_decode1<192>, tm_h, tm_w64, d); break;
+      case 128: e = cudaLaunchKernelEx(&cfg, bi::k_lm_decode1<128>, tm_h, tm_w64, d); break;
+      default: break;
     }
-    if (cudaGetLastError() != cudaSuccess) return BI_ERR_CUDA;
   }
-#undef BI_ZT
+  if (e != cudaSuccess) return BI_ERR_CUDA;
   ProfScope ps(kKLmZscan, s);
   const unsigned rows = static_cast<unsigned>(T);
   switch (pl.NZ) {
-    case 256: bi::k_lm_zscan<256><<<rows, bi::kZsThreads, 0, s>>>(a.csum, a.mref, a.zy, targets, T, V, nvz, pl.C, logprob, lse, dev_status); break;
-    case 192: bi::k_lm_zscan<192><<<rows, bi::kZsThreads, 0, s>>>(a.csum, a.mref, a.zy, targets, T, V, nvz, pl.C, logprob, lse, dev_status); break;
-    default:  bi::k_lm_zscan<128><<<rows, bi::kZsThreads, 0, s>>>(a.csum, a.mref, a.zy, targets, T, V, nvz, pl.C, logprob, lse, dev_status); break;
+    case 256: bi::k_lm_zscan<256><<<rows, bi::kZsThreads, zsm, s>>>(d.csum, d.mref, d.zy, targets, T, V, nvz, pl.C, logprob, lse, dev_status); break;
+    case 192: bi::k_lm_zscan<192><<<rows, bi::kZsThreads, zsm, s>>>(d.csum, d.mref, d.zy, targets, T, V, nvz, pl.C, logprob, lse, dev_status); break;
+    default:  bi::k_lm_zscan<128><<<rows, bi::kZsThreads, zsm, s>>>(d.csum, d.mref, d.zy, targets, T, V, nvz, pl.C, logprob, lse, dev_status); break;
   }
   return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
 }
@@ -717,14 +738,15 @@ bi_status bi_is_loss_fwd_bwd(const uint16_t* hidden, const uint16_t* w_lm, const
   }
   if (cudaGetLastError() != cudaSuccess) return BI_ERR_CUDA;
 
-  CUtensorMap tm_h128, tm_hz, tm_h64, tm_w128, tm_wz, tm_w64, tm_dz, tm_p64, tm_hblk;
+  CUtensorMap tm_h128, tm_hz, tm_hsl, tm_w128, tm_wz, tm_wsl, tm_dz, tm_p64, tm_hblk;
   const int64_t trows = T > 0 ? T : 1;
   const int nvz = (V + pl.NZ - 1) / pl.NZ;
   const int64_t p_ld = static_cast<int64_t>(nvz) * pl.NZ;  // <= L.pcols
   const void* hsrc = hc ? static_cast<const void*>(hc) : static_cast<const void*>(w8 + L.hc);
+  // slice operands: the Hs / 64 column blocks of a CTA's slice, 64 rows, in one load
   if (!make_map(&tm_h128, hsrc, trows, H, 128) || !make_map(&tm_hz, hsrc, trows, H, pl.NZ) ||
-      !make_map(&tm_h64, hsrc, trows, H, 64) || !make_map(&tm_w128, w_lm, V, H, 128) ||
-      !make_map(&tm_wz, w_lm, V, H, pl.NZ) || !make_map(&tm_w64, w_lm, V, H, 64))
+      !make_map_blocks(&tm_hsl, hsrc, trows, H, 64, pl.Hs / 64) || !make_map(&tm_w128, w_lm, V, H, 128) ||
+      !make_map(&tm_wz, w_lm, V, H, pl.NZ) || !make_map_blocks(&tm_wsl, w_lm, V, H, 64, pl.Hs / 64))
     return BI_ERR_CUDA;
   const int dw_hs = dw_split(H);
   if (store ? !(make_map(&tm_dz, w8 + L.pbuf, L.tpad, p_ld, 128) &&
@@ -796,7 +818,7 @@ bi_status bi_is_loss_fwd_bwd(const uint16_t* hidden, const uint16_t* w_lm, const
 #define BI_LAUNCH(NZ_, HS_)                                                                                  \
   if (pl.NZ == NZ_ && pl.Hs == HS_) {                                                                        \
     st = BI_OK;                                                                                            \
-    if (T > 0) st = launch_lm<bi::kModeFwdDH, NZ_, HS_>(tm_h128, tm_wz, tm_w64, tm_dz, a, (T + 127) / 128, di, s); \
+    if (T > 0) st = launch_lm<bi::kModeFwdDH, NZ_, HS_>(tm_h128, tm_wz, tm_wsl, tm_dz, a, (T + 127) / 128, di, s); \
     if (st == BI_OK) {                                                                                     \
       if (lc.variant == BI_LOSS_SEQ_GATE && T > 0) {                                                      \
         ProfScope ps(kKSeqGate, s);                                                                        \
@@ -819,7 +841,7 @@ bi_status bi_is_loss_fwd_bwd(const uint16_t* hidden, const uint16_t* w_lm, const
       }                                                                                                    \
       if (cudaGetLastError() != cudaSuccess) st = BI_ERR_CUDA;                                             \
     }                                                                                                      \
-    if (st == BI_OK && !store) st = launch_lm<bi::kModeDW, NZ_, HS_>(tm_w128, tm_hz, tm_h64, tm_dz, a, a.nv128, di, s); \
+    if (st == BI_OK && !store) st = launch_lm<bi::kModeDW, NZ_, HS_>(tm_w128, tm_hz, tm_hsl, tm_dz, a, a.nv128, di, s); \
   }
   BI_LM_CONFIGS(BI_LAUNCH)
 #undef BI_LAUNCH

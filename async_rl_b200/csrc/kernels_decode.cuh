@@ -5,23 +5,10 @@
 // "Zero Mismatch, Simple Async RL", section "Alignment permits a simpler learning path": rollout
 // and learner logprobs bit-identical for the same weights and tokens, whether a row is scored
 // alone or packed.  The cluster kernel gives a one-row call the same bits as a packed one, but it
-// sweeps the whole vocabulary on one cluster.  Here the same arithmetic is spread over the GPU in
-// two passes over W; between them only per-tile maxima, references and 32-column partial sums
-// (1/32 of the logits) are kept:
-//
-// Pass 1 (k_lm_ztiles<NZ, false>): one CTA per vocabulary tile j at a time computes z_j = H W_j^T
-//   for the 128-row tile with the cluster kernel's instruction sequence (tcgen05 M = 128, N = NZ,
-//   K = H in 64-column chunks of four K = 16 instructions, first without accumulate) and writes
-//   the tile's row maximum M_j over the valid columns for the T real rows.
-// Chain (k_lm_zchain, one thread per row): the lazy reference chain m_j = (M_j > m_{j-1} + tau) ?
-//   M_j : m_{j-1}, as the producers of consecutive steps pass it on.
-// Pass 2 (k_lm_ztiles<NZ, true>): the same tiles again; every 32-column chunk sum
-//   cs = sum_q e^{z - m_j} (target column and columns past V excluded, q in order) and the target
-//   logit, exactly as the cluster kernel's producer epilogue forms them.
-// Combine (k_lm_zscan, one block per row): per class k (steps j = k mod C) the partial sum with its
-//   rescale at each change of reference and the chunk sums added in order; then the combine of
-//   the C classes in class order.  Each of these is the cluster kernel's epilogue expression for
-//   expression.
+// sweeps the whole vocabulary on one cluster.  Here the same arithmetic is spread over the GPU:
+// k_lm_decode1 reads W once on every SM and leaves per-sub-tile row maxima, each step's reference
+// and 32-column partial sums (about 1/20 of the logits); k_lm_zscan combines them per row in the
+// cluster kernel's order.
 #pragma once
 
 #include "kernels_lm.cuh"
@@ -31,56 +18,92 @@ namespace bi {
 constexpr int kDecodeRows = 128;  // rows one tile holds: the largest T this path serves
 constexpr int kZtThreads = 192;   // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 
-template <int kNZ>
-struct ZtTile {
-  static constexpr int stage_bytes = kAUnitBytes + kNZ * 128;  // hidden [128 x 64] + W rows [NZ x 64]
-  static constexpr int nstages = 4;
-  static constexpr int smem = nstages * stage_bytes + 1024;
-  static_assert(smem <= kLmSmemLimit, "stages do not fit");
-};
+// ---------------------------------------------------------------------------------------------
+// Single pass (k_lm_decode1): one cooperative launch, one CTA per SM, W read once.
+//
+// The vocabulary is cut into 64-column sub-tiles (an NZ-wide tile of the cluster kernel is NZ / 64
+// of them; a logit column's value does not depend on the N of the instruction that computes it,
+// only on its row of A, its row of B and the K order, which are the cluster kernel's).  Sub-tile
+// s is handled by CTA s mod G in round s div G, which spreads the vocabulary evenly over the SMs.
+// Per round a CTA computes its sub-tile's logits into one of four TMEM buffers, takes the row
+// maxima over the valid columns, writes them and publishes its progress (a release store of the
+// number of rounds done).  Two rounds later it forms the sub-tile's 32-column chunk sums: by then
+// every CTA has published the maxima of every sub-tile of the tiles up to this one (an acquire
+// poll of the progress flags, bounded), so each row's reference chain can be advanced up to this
+// tile, as the cluster kernel's producers pass it on.  Every CTA advances the chain of every row
+// itself (the same arithmetic everywhere); the CTAs of a tile write its references for the
+// combine.  Co-residency of all CTAs, on which the polls rely, is what the cooperative launch
+// guarantees.
+// ---------------------------------------------------------------------------------------------
+__device__ __forceinline__ void st_release_gpu_u32(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t ld_relaxed_gpu_u32(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 
-struct ZtShared {
-  uint64_t full[4], empty[4];
-  uint64_t z_full[2], z_empty[2];
-  uint64_t mma_done;
+constexpr int kD1Sub = 64;     // columns of a sub-tile (one MMA of N = 64)
+constexpr int kD1Stages = 8;
+constexpr int kD1Buf = 4;      // logit buffers in TMEM
+constexpr int kD1Lag = 2;      // rounds between a sub-tile's maxima and its chunk sums
+constexpr int kD1StageBytes = kAUnitBytes + kD1Sub * 128;  // hidden [128 x 64] + W rows [64 x 64]
+constexpr int kD1Smem = kD1Stages * kD1StageBytes + 1024;
+static_assert(kD1Smem <= kLmSmemLimit, "stages do not fit");
+
+struct D1Shared {
+  uint64_t full[kD1Stages], empty[kD1Stages];
+  uint64_t z_full[kD1Buf], z_empty[kD1Buf];
+  uint64_t mma_done, ep_bar;
+  float mcs[kDecodeRows];  // each row's reference after tile jc - 1
   uint32_t tmem_base;
   volatile uint32_t abort_flag;
 };
 
-struct ZtArgs {
-  int64_t T;        // real rows (<= 128)
+struct D1Args {
+  int64_t T;          // real rows (<= 128)
   int32_t V, nvz, KB;
-  float* tmax;      // [nvz][T] row maximum of each tile over its valid columns (pass 1 writes)
-  const float* mref;  // [nvz][T] reference of each row at each step (pass 2 reads)
-  float* csum;      // [T][nvz][NZ / 32] 32-column chunk sums of e^{z - m_j} (pass 2 writes)
-  float* zy;        // [T] target logit (pass 2 writes, from the tile holding the target)
-  const int32_t* y; // [T] targets
+  int32_t nsub;       // sub-tiles: nvz * NZ / 64
+  int32_t rounds;     // ceil(nsub / gridDim.x)
+  float* smax;        // [T][nsub] row maxima of each sub-tile over its valid columns
+  float* mref;        // [nvz][T] reference of each row at each step
+  float* csum;        // [T][nvz][NZ / 32] chunk sums
+  float* zy;          // [T] target logits
+  const int32_t* y;   // [T]
+  uint32_t* progress; // [gridDim.x] rounds whose maxima each CTA has published (zero at launch)
   int32_t* status;
   uint64_t limit_ns;
 };
 
-template <int kNZ, bool kSums>
+template <int kNZ>
 __global__ void __launch_bounds__(kZtThreads, 1)
-    k_lm_ztiles(const __grid_constant__ CUtensorMap tm_h, const __grid_constant__ CUtensorMap tm_w, ZtArgs a) {
-  // tm_h: hidden [T][H], box {64, 128}; tm_w: W [V][H], box {64, NZ}; both 128-byte swizzled
-  using ZT = ZtTile<kNZ>;
+    k_lm_decode1(const __grid_constant__ CUtensorMap tm_h, const __grid_constant__ CUtensorMap tm_w, D1Args a) {
+  // tm_h: hidden [T][H], box {64, 128}; tm_w: W [V][H], box {64, 64}; both 128-byte swizzled
+  constexpr int kSubPerTile = kNZ / kD1Sub;
+  constexpr int kChunks = kNZ / 32;
   extern __shared__ __align__(1024) uint8_t dsmem[];
-  ZtShared& sh = *reinterpret_cast<ZtShared*>(dsmem + ZT::nstages * ZT::stage_bytes);
+  D1Shared& sh = *reinterpret_cast<D1Shared*>(dsmem + kD1Stages * kD1StageBytes);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const int G = static_cast<int>(gridDim.x);
+  const int b = static_cast<int>(blockIdx.x);
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < kD1Stages; ++i) {
       mbar_init(&sh.full[i], 1);
       mbar_init(&sh.empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kD1Buf; ++i) {
       mbar_init(&sh.z_full[i], 1);
       mbar_init(&sh.z_empty[i], 128);
     }
     mbar_init(&sh.mma_done, 1);
+    mbar_init(&sh.ep_bar, 128);
     sh.abort_flag = 0u;
     fence_mbar_init_cluster();
   }
+  if (threadIdx.x < kDecodeRows) sh.mcs[threadIdx.x] = -INFINITY;
   if (warp == 1) {
     tmem_alloc(&sh.tmem_base, 512);
     tmem_relinquish();
@@ -92,9 +115,9 @@ __global__ void __launch_bounds__(kZtThreads, 1)
   const uint32_t ring = smem_u32(dsmem);
   const bool misaligned = (ring & 1023u) != 0;
   if (misaligned && threadIdx.x == 0) raise_status(a.status, 4 /* BI_ERR_CUDA */);
-  const int ntiles = misaligned ? 0 : a.nvz;
+  const int rounds = misaligned ? 0 : a.rounds;
   const WaitCtl wc{&sh.abort_flag, a.status, a.limit_ns};
-  constexpr uint32_t nst = static_cast<uint32_t>(ZT::nstages);
+  constexpr uint32_t nst = static_cast<uint32_t>(kD1Stages);
 
   if (warp == 0) {
     if (lane == 0) {
@@ -102,18 +125,19 @@ __global__ void __launch_bounds__(kZtThreads, 1)
       tma_prefetch_desc(&tm_w);
       uint32_t stage = 0, phase = 0;
       bool ok = true;
-      for (int j = blockIdx.x; ok && j < ntiles; j += gridDim.x) {
+      for (int r = 0; ok && r < rounds; ++r) {
+        const int sub = r * G + b;
+        if (sub >= a.nsub) continue;
 #pragma unroll 1
         for (int kb = 0; kb < a.KB; ++kb) {
           if (!mbar_wait<false>(&sh.empty[stage], phase ^ 1u, wc)) { ok = false; break; }
-          mbar_arrive_expect_tx(&sh.full[stage], static_cast<uint32_t>(ZT::stage_bytes));
-          const uint32_t dst = ring + stage * ZT::stage_bytes;
+          mbar_arrive_expect_tx(&sh.full[stage], static_cast<uint32_t>(kD1StageBytes));
+          const uint32_t dst = ring + stage * kD1StageBytes;
           tma_load_2d(dst, &tm_h, &sh.full[stage], kb * 64, 0);
-          tma_load_2d(dst + kAUnitBytes, &tm_w, &sh.full[stage], kb * 64, j * kNZ);
+          tma_load_2d(dst + kAUnitBytes, &tm_w, &sh.full[stage], kb * 64, sub * kD1Sub);
           ring_advance(stage, phase, nst);
         }
       }
-      // copies still in flight land before the CTA may exit
       for (uint32_t i = 0; i < nst; ++i) {
         const uint32_t ph = (i < stage) ? phase : (phase ^ 1u);
         const uint64_t t0 = globaltimer_ns();
@@ -124,95 +148,174 @@ __global__ void __launch_bounds__(kZtThreads, 1)
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
-      // the logit tile of kernels_lm.cuh: the same descriptors and the same instruction sequence
-      constexpr uint32_t idesc_z = idesc_bf16(128, kNZ, false, false);
-      constexpr uint64_t sb = static_cast<uint64_t>(ZT::stage_bytes >> 4);
+      // the cluster kernel's instruction sequence per 64-column chunk of K, with N = 64
+      constexpr uint32_t idesc = idesc_bf16(128, kD1Sub, false, false);
+      constexpr uint64_t sb = static_cast<uint64_t>(kD1StageBytes >> 4);
       const uint64_t dk0 = sdesc_k_sw128(ring);
       const uint64_t dkb0 = sdesc_k_sw128(ring + kAUnitBytes);
-      uint32_t stage = 0, phase = 0, tc = 0;
+      uint32_t stage = 0, phase = 0;
       bool ok = true;
-      for (int j = blockIdx.x; ok && j < ntiles; j += gridDim.x, ++tc) {
-        const uint32_t b = tc & 1u;
-        if (!mbar_wait<false>(&sh.z_empty[b], ((tc >> 1) & 1u) ^ 1u, wc)) break;
+      for (int r = 0; ok && r < rounds; ++r) {
+        const int sub = r * G + b;
+        if (sub >= a.nsub) continue;
+        const uint32_t bb = static_cast<uint32_t>(r % kD1Buf);
+        if (!mbar_wait<false>(&sh.z_empty[bb], ((r / kD1Buf) & 1u) ^ 1u, wc)) break;
         tc_fence_after();
-        const uint32_t zt = tmem + b * 256u;
+        const uint32_t zt = tmem + bb * kD1Sub;
 #pragma unroll 1
         for (int kb = 0; kb < a.KB; ++kb) {
           if (!mbar_wait<false>(&sh.full[stage], phase, wc)) { ok = false; break; }
           tc_fence_after();
           const uint64_t da = dk0 + stage * sb;
           const uint64_t db = dkb0 + stage * sb;
-          umma_bf16(zt, da, db, idesc_z, kb != 0 ? 1u : 0u);
-          umma_bf16(zt, da + 2, db + 2, idesc_z, 1u);
-          umma_bf16(zt, da + 4, db + 4, idesc_z, 1u);
-          umma_bf16(zt, da + 6, db + 6, idesc_z, 1u);
+          umma_bf16(zt, da, db, idesc, kb != 0 ? 1u : 0u);
+          umma_bf16(zt, da + 2, db + 2, idesc, 1u);
+          umma_bf16(zt, da + 4, db + 4, idesc, 1u);
+          umma_bf16(zt, da + 6, db + 6, idesc, 1u);
           umma_commit(&sh.empty[stage]);
           ring_advance(stage, phase, nst);
         }
         if (!ok) break;
-        umma_commit(&sh.z_full[b]);
+        umma_commit(&sh.z_full[bb]);
       }
-      // every MMA (and its commits) completes before the CTA may release its memory
       umma_commit(&sh.mma_done);
       mbar_wait<false>(&sh.mma_done, 0u, wc);
     }
     __syncwarp();
   } else {
-    // epilogue: warp w reads TMEM lanes 32 (w mod 4) ..; one row per thread
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
+    const int et = threadIdx.x - 64;  // 0..127
     const uint32_t tl = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     const bool warp_rows = static_cast<int64_t>(quarter * 32) < a.T;  // warp-uniform
-    uint32_t tc = 0;
     const bool real = row < a.T;
     const int32_t yt = real ? a.y[row] : -1;
-    for (int j = blockIdx.x; j < ntiles; j += gridDim.x, ++tc) {
-      const uint32_t b = tc & 1u;
-      if (!__all_sync(0xffffffffu, mbar_wait<false>(&sh.z_full[b], (tc >> 1) & 1u, wc))) break;
-      tc_fence_after();
-      if (warp_rows) {
-        if (!kSums) {
-          // pass 1: the tile's row maximum over the valid columns (the producer's first pass)
-          float M = -INFINITY;
+    uint32_t epc = 0;
+    int jc = 0;              // next tile of the rows' chains (the same for every row)
+    bool ok = true;
+    for (int r = 0; ok && r < rounds + kD1Lag; ++r) {
+      if (r < rounds) {
+        const int sub = r * G + b;
+        if (sub < a.nsub) {
+          const uint32_t bb = static_cast<uint32_t>(r % kD1Buf);
+          if (!__all_sync(0xffffffffu, mbar_wait<false>(&sh.z_full[bb], (r / kD1Buf) & 1u, wc))) { ok = false; break; }
+          tc_fence_after();
+          if (warp_rows) {
+            float M = -INFINITY;
 #pragma unroll 1
-          for (int c = 0; c < kNZ / 32; ++c) {
-            uint32_t v[32];
-            tmem_ld32(tl + b * 256u + c * 32, v);
-            tmem_ld_wait();
-            const int vb = j * kNZ + c * 32;
+            for (int c = 0; c < kD1Sub / 32; ++c) {
+              uint32_t v[32];
+              tmem_ld32(tl + bb * kD1Sub + c * 32, v);
+              tmem_ld_wait();
+              const int vb = sub * kD1Sub + c * 32;
 #pragma unroll
-            for (int q = 0; q < 32; ++q)
-              if (vb + q < a.V) M = fmaxf(M, __uint_as_float(v[q]));
-          }
-          if (real) a.tmax[static_cast<int64_t>(j) * a.T + row] = M;
-        } else {
-          // pass 2: chunk sums against the step's reference, and the target logit (the
-          // producer's second pass)
-          const float mn2 = (real ? a.mref[static_cast<int64_t>(j) * a.T + row] : 0.f) * kLog2e;
-          float* cs_out = a.csum + (static_cast<int64_t>(real ? row : 0) * a.nvz + j) * (kNZ / 32);
-#pragma unroll 1
-          for (int c = 0; c < kNZ / 32; ++c) {
-            uint32_t v[32];
-            tmem_ld32(tl + b * 256u + c * 32, v);
-            tmem_ld_wait();
-            const int vb = j * kNZ + c * 32;
-            float cs = 0.f;
-#pragma unroll
-            for (int q = 0; q < 32; ++q) {
-              const float z = __uint_as_float(v[q]);
-              const bool tgt = (vb + q == yt);
-              const bool in = (vb + q < a.V) && !tgt;
-              const float pr = in ? ex2_approx(fmaf(z, kLog2e, -mn2)) : 0.f;
-              cs += pr;
-              if (tgt && real) a.zy[row] = z;
+              for (int q = 0; q < 32; ++q)
+                if (vb + q < a.V) M = fmaxf(M, __uint_as_float(v[q]));
             }
-            if (real) cs_out[c] = cs;
+            if (real) a.smax[static_cast<int64_t>(row) * a.nsub + sub] = M;
           }
+        }
+        // this round's maxima are written by every epilogue thread: publish the progress
+        __threadfence();
+        mbar_arrive(&sh.ep_bar);
+        if (!__all_sync(0xffffffffu, mbar_wait<false>(&sh.ep_bar, (epc++) & 1u, wc))) { ok = false; break; }
+        if (et == 0) st_release_gpu_u32(a.progress + b, static_cast<uint32_t>(r + 1));
+      }
+      const int qr = r - kD1Lag;
+      if (qr < 0 || qr >= rounds) continue;
+      const int sub = qr * G + b;
+      if (sub >= a.nsub) continue;
+      const int j = sub / kSubPerTile;
+      // every CTA has published the maxima of the rounds holding tiles 0 .. j: the first epilogue
+      // warp reads the G flags 32 at a time (relaxed), and once all are there an acquire fence
+      // orders the maxima reads after them; the CTA barrier below passes that on
+      const uint32_t need = static_cast<uint32_t>(((j + 1) * kSubPerTile - 1) / G + 1);
+      if (et < 32) {
+        const uint64_t t0 = globaltimer_ns();
+        uint32_t spins = 0;
+        while (true) {
+          bool mine = true;
+          for (int c = et; c < G; c += 32) mine = mine && (ld_relaxed_gpu_u32(a.progress + c) >= need);
+          if (__all_sync(0xffffffffu, mine)) break;
+          if ((++spins & 15u) == 0) {
+            const bool stop = sh.abort_flag != 0u || globaltimer_ns() - t0 > a.limit_ns;
+            if (__any_sync(0xffffffffu, stop)) {
+              if (et == 0 && sh.abort_flag == 0u) {
+                raise_status(a.status, 5 /* BI_ERR_TIMEOUT */);
+                sh.abort_flag = 1u;
+              }
+              ok = false;
+              break;
+            }
+          }
+        }
+        fence_acq_rel_gpu();
+      }
+      mbar_arrive(&sh.ep_bar);
+      if (!__all_sync(0xffffffffu, mbar_wait<false>(&sh.ep_bar, (epc++) & 1u, wc))) { ok = false; break; }
+      if (sh.abort_flag) { ok = false; break; }
+      const uint32_t bb = static_cast<uint32_t>(qr % kD1Buf);
+      if (jc <= j) {
+        // advance every row's chain over tiles jc .. j, a warp per row: the range's largest
+        // sub-tile maximum first (coalesced loads); only when it could raise the reference are the
+        // tiles walked in order, 32 at a time (lane l takes tile base + l, the chain runs over
+        // the lanes by shuffles), as the cluster kernel's producers pass the reference on
+        const int ew = warp - 2;  // 0..3
+        for (int r = ew; r < static_cast<int>(a.T); r += 4) {
+          const float* rr = a.smax + static_cast<int64_t>(r) * a.nsub;
+          float m = sh.mcs[r];
+          float mx = -INFINITY;
+          for (int i = jc * kSubPerTile + lane; i < (j + 1) * kSubPerTile; i += 32) mx = fmaxf(mx, __ldcg(rr + i));
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+          if (mx > m + kTau) {
+            for (int base = jc; base <= j; base += 32) {
+              float Ml = -INFINITY;
+              if (base + lane <= j) {
+#pragma unroll
+                for (int i = 0; i < kSubPerTile; ++i) Ml = fmaxf(Ml, __ldcg(rr + (base + lane) * kSubPerTile + i));
+              }
+              const int nt = (j - base + 1) < 32 ? (j - base + 1) : 32;
+              for (int l = 0; l < nt; ++l) {
+                const float M = __shfl_sync(0xffffffffu, Ml, l);
+                m = (M > m + kTau) ? M : m;
+              }
+            }
+          }
+          if (lane == 0) sh.mcs[r] = m;
+        }
+        jc = j + 1;
+        mbar_arrive(&sh.ep_bar);
+        if (!__all_sync(0xffffffffu, mbar_wait<false>(&sh.ep_bar, (epc++) & 1u, wc))) { ok = false; break; }
+      }
+      const float mc = real ? sh.mcs[row] : 0.f;
+      if (warp_rows) {
+        if (real && sub % kSubPerTile == 0) a.mref[static_cast<int64_t>(j) * a.T + row] = mc;
+        const float mn2 = (real ? mc : 0.f) * kLog2e;
+        float* cs_out = a.csum + (static_cast<int64_t>(real ? row : 0) * a.nvz + j) * kChunks + (sub % kSubPerTile) * 2;
+#pragma unroll 1
+        for (int c = 0; c < kD1Sub / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tl + bb * kD1Sub + c * 32, v);
+          tmem_ld_wait();
+          const int vb = sub * kD1Sub + c * 32;
+          float cs = 0.f;
+#pragma unroll
+          for (int q = 0; q < 32; ++q) {
+            const float z = __uint_as_float(v[q]);
+            const bool tgt = (vb + q == yt);
+            const bool in = (vb + q < a.V) && !tgt;
+            const float pr = in ? ex2_approx(fmaf(z, kLog2e, -mn2)) : 0.f;
+            cs += pr;
+            if (tgt && real) a.zy[row] = z;
+          }
+          if (real) cs_out[c] = cs;
         }
       }
       tc_fence_before();
-      mbar_arrive(&sh.z_empty[b]);
+      mbar_arrive(&sh.z_empty[bb]);
     }
+    if (!ok && et == 0) sh.abort_flag = 1u;
   }
 
   tc_fence_before();
@@ -228,54 +331,50 @@ __global__ void __launch_bounds__(kZtThreads, 1)
   }
 }
 
-// One thread per row: the reference chain from the tile maxima, in step order.
-__global__ void k_lm_zchain(const float* __restrict__ tmax, int64_t T, int nvz, float* __restrict__ mref) {
-  const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (t >= T) return;
-  float mprev = -INFINITY;
-#pragma unroll 4
-  for (int j = 0; j < nvz; ++j) {
-    const float M = tmax[static_cast<int64_t>(j) * T + t];
-    const float mnew = (M > mprev + kTau) ? M : mprev;
-    mref[static_cast<int64_t>(j) * T + t] = mnew;
-    mprev = mnew;
-  }
+constexpr int kZsThreads = 256;
+
+// Dynamic shared memory of k_lm_zscan: one row's chunk sums and references.
+__host__ __device__ constexpr size_t zscan_smem(int nvz, int nz) {
+  return static_cast<size_t>(nvz) * (static_cast<size_t>(nz / 32) + 1) * 4;
 }
 
-constexpr int kZsThreads = 32;
-
-// One block (one warp) per row: the class partial sums and their combine.
+// One block per row: the row's chunk sums and references are staged in shared memory by the whole
+// block (coalesced), then C threads form the class partial sums (serial by definition) and one
+// thread combines them.
 template <int kNZ>
 __global__ void __launch_bounds__(kZsThreads)
     k_lm_zscan(const float* __restrict__ csum, const float* __restrict__ mref, const float* __restrict__ zyb,
                const int32_t* __restrict__ y, int64_t T, int V, int nvz, int C, float* __restrict__ logprob,
                float* __restrict__ lse_out, int32_t* status) {
   constexpr int kChunks = kNZ / 32;
+  extern __shared__ float zs[];
+  float* cs = zs;                                            // [nvz][kChunks]
+  float* mr = zs + static_cast<int64_t>(nvz) * kChunks;      // [nvz]
   __shared__ float cls[2 * 8];  // [8] class reference, [8] class sum
   const int64_t t = blockIdx.x;
   if (t >= T) return;
   const float* crow = csum + t * static_cast<int64_t>(nvz) * kChunks;
+  for (int i = threadIdx.x; i < nvz * kChunks; i += kZsThreads) cs[i] = crow[i];
+  for (int j = threadIdx.x; j < nvz; j += kZsThreads) mr[j] = mref[static_cast<int64_t>(j) * T + t];
+  __syncthreads();
   // class k: its steps in order, rescaled at each change of reference
   if (static_cast<int>(threadIdx.x) < C) {
     const int k = threadIdx.x;
     float mp = -INFINITY, sp = 0.f;
 #pragma unroll 2
     for (int j = k; j < nvz; j += C) {
-      const float mnew = mref[static_cast<int64_t>(j) * T + t];
+      const float mnew = mr[j];
       if (mnew != mp) {
         sp = (mp == -INFINITY) ? 0.f : sp * ex2_approx((mp - mnew) * kLog2e);
         mp = mnew;
       }
-      float cv[kChunks];
 #pragma unroll
-      for (int c = 0; c < kChunks; ++c) cv[c] = crow[j * kChunks + c];
-#pragma unroll
-      for (int c = 0; c < kChunks; ++c) sp += cv[c];
+      for (int c = 0; c < kChunks; ++c) sp += cs[j * kChunks + c];
     }
     cls[k] = mp;
     cls[8 + k] = sp;
   }
-  __syncwarp();
+  __syncthreads();
   if (threadIdx.x == 0) {
     float mstar = -INFINITY;
     for (int k = 0; k < C; ++k) mstar = fmaxf(mstar, cls[k]);

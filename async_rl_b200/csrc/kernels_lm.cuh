@@ -224,7 +224,7 @@ __device__ __forceinline__ void ring_advance(uint32_t& stage, uint32_t& phase, u
 struct TmaMaps {
   const CUtensorMap* stat;  // stationary operand, box {64, 128}
   const CUtensorMap* zb;    // streamed operand, box {64, NZ}  (logit phase B)
-  const CUtensorMap* sl;    // streamed operand, box {64, 64}  (slice units)
+  const CUtensorMap* sl;    // streamed operand seen as [cols / 64][rows][64], box {64, 64, Hs / 64}
   const CUtensorMap* dz;    // scratch tiles, box {64, 128}
 };
 
@@ -240,7 +240,6 @@ __device__ __forceinline__ void lm_tma_role(LmShared& sh, const LmArgs& a, const
   constexpr uint32_t sbytes = static_cast<uint32_t>(LmTile<kNZ, kHS>::stage_bytes);
   constexpr uint32_t zbytes = kAUnitBytes + kNZ * 128;
   constexpr uint32_t obytes = kAUnitBytes + kHS * 128;
-  constexpr int nsl = kHS / 64;
   constexpr int nkc = kNZ / 64;
   uint32_t stage = 0, phase = 0;
 
@@ -284,9 +283,8 @@ __device__ __forceinline__ void lm_tma_role(LmShared& sh, const LmArgs& a, const
         mbar_arrive_expect_tx(&sh.full[stage], obytes);
         const uint32_t dst = x.ring_base + stage * sbytes;
         const int yrow = p.j * kNZ + kc * 64;
-#pragma unroll
-        for (int u = 0; u < nsl; ++u)
-          tma_load_2d(dst + kAUnitBytes + u * kSlUnitBytes, m.sl, &sh.full[stage], x.slice0 + u * 64, yrow);
+        // the Hs / 64 blocks of this CTA's columns in one load (block-major view of the operand)
+        tma_load_3d(dst + kAUnitBytes, m.sl, &sh.full[stage], 0, yrow, x.slice0 / 64);
         if (!dz_ok) {
           if (!lm_wait<true>(sh, a, x.C, &sh.dz_ready[p.slot], p.round & 1u)) { ok = false; break; }
           dz_ok = true;

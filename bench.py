@@ -27,7 +27,8 @@ RMSNorm of the 1.5B-shape hidden states [76239, 1536] followed by the gate/up pr
 Y = X W^T with W [8960, 1536] (bi_rmsnorm + bi_gemm_bf16); ranks are independent replicas.
 
 --workload decode times decode-style scoring (not the default line): one bi_logprob_fwd call per
-step on one row of the 1.5B head (the all-SM path), with the cluster kernel's latency beside it.
+step on one row of the 1.5B head (the all-SM path: one pass over W on every SM, then the
+per-row combine), with the cluster kernel's latency beside it.
 """
 from __future__ import annotations
 
@@ -107,8 +108,8 @@ def measured_peaks():
     return {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}, "fallback"
 
 
-TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "dram_traffic_small_T5632.md")
-CSRC_HASHED = ("sm100.cuh", "kernels_lm.cuh", "kernels_dw.cuh", "kernels_small.cuh", "bi_api.cu")
+TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "k_lm_fwd_dh_k_lm_dw_T5632.md")
+CSRC_HASHED = ("sm100.cuh", "kernels_lm.cuh")  # the forward + dH kernel's sources
 
 
 def sources_hash() -> str:
@@ -787,7 +788,9 @@ def run_decode(args):
     ems = e0.elapsed_time(e1) / args.steps
     peaks, peak_src = measured_peaks()
     w_bytes = 2.0 * V * H
-    zt = prof.get("k_lm_ztiles", (float("nan"), 1))
+    # the kernel that streams W (the cluster kernel's launches when the device has no cooperative launch)
+    wk = "k_lm_decode1" if "k_lm_decode1" in prof else "k_lm_fwd"
+    zt = prof.get(wk, (float("nan"), 1))
     zt_ms = zt[0] / max(zt[1], 1)
     line = {"metric": DECODE_METRIC, "value": ms, "unit": "ms per call", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": False, "scaling": "weak",
@@ -795,7 +798,7 @@ def run_decode(args):
             "config": {"workload": f"decode: 1 row per bi_logprob_fwd call, H={H} V={V}, all-SM path",
                        "parallelism": f"replicas{world}", "l2": "W 0.47 GB exceeds L2; no flush"},
             "rows_128_ms": ms_128, "cluster_kernel_ms": ms_cluster,
-            "roofline": {"bound": "hbm", "kernel": "k_lm_ztiles", "achieved": w_bytes / (zt_ms * 1e-3) / 1e9,
+            "roofline": {"bound": "hbm", "kernel": wk, "achieved": w_bytes / (zt_ms * 1e-3) / 1e9,
                          "peak": float(peaks.get("hbm_gbs")), "unit": "GB/s",
                          "frac": w_bytes / (zt_ms * 1e-3) / 1e9 / float(peaks.get("hbm_gbs")), "traffic": None,
                          "peak_source": f"{peak_src} hbm_gbs", "algorithmic_bytes_per_launch": w_bytes},

@@ -134,9 +134,9 @@ typedef struct {
  * copy of the scored hidden rows (T H bf16), per-response coefficients and a fixed-size scratch for
  * the tiles the cluster passes between its CTAs; dW recomputes the logits tile by tile.
  * For bi_logprob_fwd with 1 <= T <= 128 rows (decode-style scoring) it also holds what the all-SM
- * path keeps between its two passes over W: per-tile row maxima and references and 32-column
- * partial sums of e^{z - m} (about 4 T V / 32 bytes at most), so that the call runs on every SM
- * instead of one cluster; the bits are the same either way. */
+ * path keeps: row maxima of 64-column sub-tiles, each step's reference and 32-column partial sums
+ * of e^{z - m} (about 4 T V / 18 bytes at most), so that the call runs on every SM instead of one
+ * cluster; the bits are the same either way. */
 BI_API size_t bi_workspace_bytes(int64_t T, int32_t H, int32_t V, int32_t R);
 
 /* Smallest workspace accepted.  For bi_is_loss_fwd_bwd it equals bi_workspace_bytes.  For R = 0 it
@@ -158,11 +158,13 @@ BI_API size_t bi_workspace_bytes_pstore(int64_t T, int32_t H, int32_t V, int32_t
  * A row gets identical bits whether it is scored alone (T = 1, decode style) or packed.  Packed
  * batches run on the cluster kernel (one cluster sweeps the vocabulary for each 128-row tile).
  * With 1 <= T <= 128 and a workspace of bi_workspace_bytes(T, H, V, 0) bytes the rows are scored
- * on every SM instead, in two passes over W: the logit tiles with the cluster kernel's
- * instruction sequence give the per-tile row maxima, then the reference chain, then the same
- * tiles again give the 32-column partial sums against each step's reference, and the class sums
- * and their combine follow the cluster kernel's order, which reproduces its bits ("Zero Mismatch,
- * Simple Async RL", section "Alignment permits a simpler learning path"). */
+ * on every SM instead, in one cooperative pass over W: the logits of 64-column sub-tiles with the
+ * cluster kernel's per-column instruction sequence give the row maxima, every CTA advances the
+ * reference chain once the maxima of the tiles it needs are published, forms the 32-column partial
+ * sums against each step's reference, and a per-row combine follows the cluster kernel's class
+ * order, which reproduces its bits ("Zero Mismatch, Simple Async RL", section "Alignment permits a
+ * simpler learning path").  Without cooperative launch support the rows go to the cluster kernel,
+ * with the same bits. */
 BI_API bi_status bi_logprob_fwd(const uint16_t* hidden, const uint16_t* w_lm, const int32_t* targets,
                          int64_t T, int32_t H, int32_t V, float* logprob, float* lse,
                          int32_t* dev_status, void* ws, size_t ws_bytes, void* stream);

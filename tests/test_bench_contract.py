@@ -102,6 +102,6 @@ def test_decode_workload_line():
     line = _run(["--workload", "decode", "--steps", "20", "--warmup", "3"], timeout=900)
     for k in REQUIRED + ("roofline", "clocks", "gpu_launches", "cluster_kernel_ms", "rows_128_ms"):
         assert k in line, k
-    # four launches per one-row call: tile maxima, the reference chain, chunk sums, the combine
-    assert line["gpu_launches"] == 4 * 20 and line["value"] < line["cluster_kernel_ms"]
+    # two launches per one-row call: the single pass over W on every SM, then the combine
+    assert line["gpu_launches"] == 2 * 20 and line["value"] < line["cluster_kernel_ms"]
     assert 0 < line["roofline"]["frac"] < 2 and line["e2e"]["h2d_bytes_per_step"] > 0

@@ -1,5 +1,5 @@
-"""Decode-style scoring (bi_logprob_fwd with T <= 128 rows, computed on every SM in two passes
-over W that keep only per-tile maxima, references and 32-column partial sums) gives the same bits
+"""Decode-style scoring (bi_logprob_fwd with T <= 128 rows, computed on every SM in one cooperative
+pass over W that keeps only sub-tile maxima, references and 32-column partial sums) gives the same bits
 as the cluster kernel that scores packed batches ("Zero Mismatch, Simple Async RL", section
 "Alignment permits a simpler learning path": rollout and learner logprobs bit-identical whether a
 row is scored alone or packed), for the tilings of several hidden sizes, and matches the oracle."""
@@ -51,7 +51,7 @@ def test_few_rows_bitwise_equal_to_packed_batch(H, V, cuda_device):
 def test_few_rows_with_moving_reference_bitwise_equal_to_packed_batch(cuda_device):
     """Logits growing along the vocabulary (W_v scaled by 1 + 60 (v/V)^2): each row's reference
     is raised on many tiles, so the chain, the per-class rescales and the class combine of the
-    two-pass path all take their rarely used branches."""
+    single-pass path all take their rarely used branches."""
     H, V = 1536, 40000
     h, w, y = random_inputs(300, H, V, seed=77)
     ramp = (1.0 + 60.0 * (torch.arange(V, dtype=torch.float32) / V) ** 2)[:, None]
@@ -65,7 +65,7 @@ def test_few_rows_with_moving_reference_bitwise_equal_to_packed_batch(cuda_devic
 
 
 def test_few_rows_with_minimum_workspace_take_the_cluster_kernel(cuda_device):
-    """A workspace without room for the two-pass path's partial sums is accepted (the cluster
+    """A workspace without room for the all-SM path's partial sums is accepted (the cluster
     kernel scores the rows); the bits are the same."""
     h, w, y = random_inputs(5, 1536, 8192, seed=3)
     h, w, y = h.to(cuda_device), w.to(cuda_device), y.to(cuda_device)

@@ -58,7 +58,7 @@ def test_noalloc_matches_workspace_entry_point_on_consecutive_calls(cuda_device)
 
 def test_noalloc_matches_decode_sized_calls_and_null_lse(cuda_device):
     """Decode-sized calls (T = 1 and T = 128): bi_logprob_fwd with its default workspace scores them
-    on every SM in two passes, the no-allocation entry point on the cluster kernel; the header
+    on every SM in one pass, the no-allocation entry point on the cluster kernel; the header
     promises the same bits.  Then a call with lse = NULL must give the same logprob bits."""
     lib = _lib.load()
     for (T, seed) in [(1, 41), (128, 42)]:
