@@ -93,7 +93,7 @@ struct WsLayout {
   size_t ctrl, lse_c, g_c, tl_c, d3_c, delta_c, clip_c, y_c, logmu_c, rowmap, respof, coef, cprefix, rej, red, hc,
       dz, alpha, fin;
   size_t sxr_c, mhist, hs, pbuf;  // the P store (loss layout with the store only)
-  size_t zmref, zcsum, zy, zsmax, zprog;  // decode-style scoring (logprob layout, T <= 128)
+  size_t zmref, zcsum, zy, zsmax;  // decode-style scoring (logprob layout, T <= 128)
   bool decode;
   size_t total;
   int nred;
@@ -108,8 +108,8 @@ constexpr size_t kFinBytes = static_cast<size_t>(kMaxSms) * 2 * 384 * sizeof(flo
 // the scaled hidden states of the dW GEMM ([Tpad][H] bf16).
 // R == 0 with `decode` and 0 < T <= 128: followed by what the all-SM scoring path keeps: per-tile
 // references ([ceil(V / 128)][T] fp32, enough for any tile width NZ >= 128), 32-column partial
-// sums ([T][V / 32 + 8] fp32 at most), the target logits ([T] fp32), the row maxima of 64-column
-// sub-tiles ([T][V / 64 + 4] fp32 at most) and one progress flag per SM.  Nothing of size T x V.
+// sums ([T][V / 32 + 8] fp32 at most), the target logits ([T] fp32) and the row maxima of
+// 64-column sub-tiles ([T][V / 64 + 4] tagged 64-bit words at most).  Nothing of size T x V.
 WsLayout ws_layout(int64_t T, int32_t H, int32_t V, int32_t R, bool store, bool decode = false) {
   WsLayout L{};
   const size_t t = static_cast<size_t>(T > 0 ? T : 1);
@@ -159,8 +159,7 @@ WsLayout ws_layout(int64_t T, int32_t H, int32_t V, int32_t R, bool store, bool 
     L.zmref = take(t * ntile * 4);
     L.zcsum = take(t * (static_cast<size_t>(V + 31) / 32 + 8) * 4);
     L.zy = take(t * 4);
-    L.zsmax = take(t * (static_cast<size_t>(V + 63) / 64 + 4) * 4);
-    L.zprog = take(static_cast<size_t>(kMaxSms) * 4);
+    L.zsmax = take(t * (static_cast<size_t>(V + 63) / 64 + 4) * 8);
   }
   L.total = o;
   return L;
@@ -294,12 +293,15 @@ bool set_lm_attributes() {
 #undef BI_SET_DW_ATTR
   ok = ok && cudaFuncSetAttribute(bi::k_gemm_pair, cudaFuncAttributeMaxDynamicSharedMemorySize, bi::kGemmSmem) ==
                  cudaSuccess;
-  ok = ok && cudaFuncSetAttribute(bi::k_lm_decode1<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+#define BI_SET_D1_ATTR(NZ_, AG_)                                                                            \
+  ok = ok && cudaFuncSetAttribute(bi::k_lm_decode1<NZ_, AG_>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
                                   bi::kD1Smem) == cudaSuccess;
-  ok = ok && cudaFuncSetAttribute(bi::k_lm_decode1<192>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  bi::kD1Smem) == cudaSuccess;
-  ok = ok && cudaFuncSetAttribute(bi::k_lm_decode1<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  bi::kD1Smem) == cudaSuccess;
+#define BI_SET_D1_ATTRS(NZ_) BI_SET_D1_ATTR(NZ_, 0) BI_SET_D1_ATTR(NZ_, 1) BI_SET_D1_ATTR(NZ_, 2) BI_SET_D1_ATTR(NZ_, 4)
+  BI_SET_D1_ATTRS(256)
+  BI_SET_D1_ATTRS(192)
+  BI_SET_D1_ATTRS(128)
+#undef BI_SET_D1_ATTRS
+#undef BI_SET_D1_ATTR
   ok = ok && cudaFuncSetAttribute(bi::k_lm_zscan<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   static_cast<int>(kZscanSmemMax)) == cudaSuccess;
   ok = ok && cudaFuncSetAttribute(bi::k_lm_zscan<192>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -343,7 +345,7 @@ const DevInfo* device_info() {
   d.gemm_clusters = query_gemm_clusters();
   int coop_attr = 0, per_sm = 0;
   d.coop = cudaDeviceGetAttribute(&coop_attr, cudaDevAttrCooperativeLaunch, dev) == cudaSuccess && coop_attr != 0 &&
-           cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, bi::k_lm_decode1<256>, bi::kZtThreads,
+           cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, bi::k_lm_decode1<256, 0>, bi::kZtThreads,
                                                          bi::kD1Smem) == cudaSuccess &&
            per_sm >= 1;
   cudaGetLastError();
@@ -469,8 +471,12 @@ int logprob_decode(const uint16_t* hidden, const uint16_t* w_lm, const int32_t* 
   const int nvz = (V + pl.NZ - 1) / pl.NZ;
   const size_t zsm = bi::zscan_smem(nvz, pl.NZ);
   if (zsm > kZscanSmemMax) return kDecodeUnsupported;
+  // hidden rows kept resident in 1 KB atoms of 8 rows when few (the ring then carries W only)
+  int ag = T <= 8 ? 1 : (T <= 16 ? 2 : (T <= 32 ? 4 : 0));
+  if (ag > 0 && bi::d1_a_bytes(ag, H / 64) + 4 * bi::kD1WBytes + 4096 > bi::kD1Smem) ag = 0;
   CUtensorMap tm_h, tm_w64;
-  if (!make_map(&tm_h, hidden, T, H, 128) || !make_map(&tm_w64, w_lm, V, H, bi::kD1Sub)) return BI_ERR_CUDA;
+  if (!make_map(&tm_h, hidden, T, H, ag > 0 ? 8 * ag : 128) || !make_map(&tm_w64, w_lm, V, H, bi::kD1Sub))
+    return BI_ERR_CUDA;
   const int nsub = nvz * (pl.NZ / bi::kD1Sub);
   const int G = nsub < di->sms ? nsub : di->sms;  // >= NZ / 64 sub-tiles: every wait has a finite target
   bi::D1Args d{};
@@ -480,15 +486,15 @@ int logprob_decode(const uint16_t* hidden, const uint16_t* w_lm, const int32_t* 
   d.KB = H / 64;
   d.nsub = nsub;
   d.rounds = (nsub + G - 1) / G;
-  d.smax = reinterpret_cast<float*>(ws + L.zsmax);
+  d.smax = reinterpret_cast<uint64_t*>(ws + L.zsmax);
   d.mref = reinterpret_cast<float*>(ws + L.zmref);
   d.csum = reinterpret_cast<float*>(ws + L.zcsum);
   d.zy = reinterpret_cast<float*>(ws + L.zy);
   d.y = targets;
-  d.progress = reinterpret_cast<uint32_t*>(ws + L.zprog);
   d.status = dev_status;
   d.limit_ns = kWaitLimitNs;
-  if (cudaMemsetAsync(d.progress, 0, static_cast<size_t>(G) * 4, s) != cudaSuccess) return BI_ERR_CUDA;
+  // the tagged maxima start untagged: a reader waits for its writer's tag
+  if (cudaMemsetAsync(d.smax, 0, static_cast<size_t>(T) * nsub * 8, s) != cudaSuccess) return BI_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(G), 1, 1);
   cfg.blockDim = dim3(bi::kZtThreads, 1, 1);
@@ -502,12 +508,14 @@ int logprob_decode(const uint16_t* hidden, const uint16_t* w_lm, const int32_t* 
   cudaError_t e = cudaErrorInvalidValue;
   {
     ProfScope ps(kKLmDecode1, s);
-    switch (pl.NZ) {
-      case 256: e = cudaLaunchKernelEx(&cfg, bi::k_lm_decode1<256>, tm_h, tm_w64, d); break;
-      case 192: e = cudaLaunchKernelEx(&cfg, bi::k_lm_decode1<192>, tm_h, tm_w64, d); break;
-      case 128: e = cudaLaunchKernelEx(&cfg, bi::k_lm_decode1<128>, tm_h, tm_w64, d); break;
-      default: break;
-    }
+#define BI_D1_LAUNCH(NZ_, AG_) \
+  if (pl.NZ == NZ_ && ag == AG_) e = cudaLaunchKernelEx(&cfg, bi::k_lm_decode1<NZ_, AG_>, tm_h, tm_w64, d);
+#define BI_D1_LAUNCHES(NZ_) BI_D1_LAUNCH(NZ_, 0) BI_D1_LAUNCH(NZ_, 1) BI_D1_LAUNCH(NZ_, 2) BI_D1_LAUNCH(NZ_, 4)
+    BI_D1_LAUNCHES(256)
+    BI_D1_LAUNCHES(192)
+    BI_D1_LAUNCHES(128)
+#undef BI_D1_LAUNCHES
+#undef BI_D1_LAUNCH
   }
   if (e != cudaSuccess) return BI_ERR_CUDA;
   ProfScope ps(kKLmZscan, s);

@@ -25,38 +25,81 @@ constexpr int kZtThreads = 192;   // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 // of them; a logit column's value does not depend on the N of the instruction that computes it,
 // only on its row of A, its row of B and the K order, which are the cluster kernel's).  Sub-tile
 // s is handled by CTA s mod G in round s div G, which spreads the vocabulary evenly over the SMs.
-// Per round a CTA computes its sub-tile's logits into one of four TMEM buffers, takes the row
-// maxima over the valid columns, writes them and publishes its progress (a release store of the
-// number of rounds done).  Two rounds later it forms the sub-tile's 32-column chunk sums: by then
-// every CTA has published the maxima of every sub-tile of the tiles up to this one (an acquire
-// poll of the progress flags, bounded), so each row's reference chain can be advanced up to this
-// tile, as the cluster kernel's producers pass it on.  Every CTA advances the chain of every row
-// itself (the same arithmetic everywhere); the CTAs of a tile write its references for the
-// combine.  Co-residency of all CTAs, on which the polls rely, is what the cooperative launch
-// guarantees.
+// Per round a CTA computes its sub-tile's logits into one of eight TMEM buffers, takes the row
+// maxima over the valid columns and stores each as a tagged 64-bit word.  Five rounds later it
+// forms the sub-tile's 32-column chunk sums: each row's reference chain is first advanced up to
+// this tile, as the cluster kernel's producers pass it on, from the maxima of every sub-tile of the
+// tiles up to this one, each read (and waited for, bounded, should its writer not have stored it
+// yet) by every CTA for itself.  The CTA of a tile's first sub-tile writes the tile's references
+// for the combine.  A round's sums need maxima of at most the next round, so by the schedule the
+// entries are nearly always there; that every CTA is resident, on which the waits rely, is what
+// the cooperative launch guarantees.
 // ---------------------------------------------------------------------------------------------
-__device__ __forceinline__ void st_release_gpu_u32(uint32_t* p, uint32_t v) {
-  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+// A sub-tile maximum travels between CTAs as one 64-bit word, the float's bits below a "written"
+// tag: an aligned 8-byte access is single-copy atomic, so a reader that sees the tag sees the
+// value, with no fence on either side (GPU-scope fences stall an SM whose TMA ring is in flight).
+// The words are zeroed before the launch.
+__device__ __forceinline__ void st_relaxed_gpu_u64(uint64_t* p, uint64_t v) {
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
-__device__ __forceinline__ uint32_t ld_relaxed_gpu_u32(const uint32_t* p) {
-  uint32_t v;
-  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+__device__ __forceinline__ uint64_t ld_relaxed_gpu_u64(const uint64_t* p) {
+  uint64_t v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
   return v;
 }
-__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+constexpr uint64_t kD1Tag = uint64_t{1} << 32;
+__device__ __forceinline__ float d1_value(uint64_t w) { return __uint_as_float(static_cast<uint32_t>(w)); }
+
+// The value of entry i of a row, waiting (bounded) until its writer has stored it.  Returns false
+// on a timeout or an abort.
+__device__ __forceinline__ bool d1_entry(const uint64_t* rr, int i, float& v, volatile uint32_t* abort_flag,
+                                         int32_t* status, uint64_t limit_ns) {
+  uint64_t w = ld_relaxed_gpu_u64(rr + i);
+  if (w & kD1Tag) {
+    v = d1_value(w);
+    return true;
+  }
+  const uint64_t t0 = globaltimer_ns();
+  uint32_t spins = 0;
+  while (true) {
+    w = ld_relaxed_gpu_u64(rr + i);
+    if (w & kD1Tag) {
+      v = d1_value(w);
+      return true;
+    }
+    if ((++spins & 15u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer_ns() - t0 > limit_ns) {
+        raise_status(status, 5 /* BI_ERR_TIMEOUT */);
+        *abort_flag = 1u;
+        return false;
+      }
+    }
+  }
+}
 
 constexpr int kD1Sub = 64;     // columns of a sub-tile (one MMA of N = 64)
-constexpr int kD1Stages = 8;
-constexpr int kD1Buf = 4;      // logit buffers in TMEM
-constexpr int kD1Lag = 2;      // rounds between a sub-tile's maxima and its chunk sums
-constexpr int kD1StageBytes = kAUnitBytes + kD1Sub * 128;  // hidden [128 x 64] + W rows [64 x 64]
-constexpr int kD1Smem = kD1Stages * kD1StageBytes + 1024;
-static_assert(kD1Smem <= kLmSmemLimit, "stages do not fit");
+constexpr int kD1MaxStages = 24;
+constexpr int kD1Buf = 8;      // logit buffers in TMEM (8 x 64 columns)
+constexpr int kD1Lag = 5;      // rounds between a sub-tile's maxima and its chunk sums: a round's sums
+                               // need every CTA's maxima of at most the next round, so the waits
+                               // have three rounds of slack
+constexpr int kD1WBytes = kD1Sub * 128;  // W rows [64 x 64]
+constexpr int kD1Smem = kLmSmemLimit;     // the ring takes what the resident rows leave
+
+// Hidden rows, the A operand of every sub-tile, are either streamed with each stage (kAG = 0: a
+// [128 x 64] box per stage) or, for T <= 8 kAG rows, loaded once and kept: the [128 x 64] A tile of
+// K chunk kb is a window starting at kb kAG KB, whose first 8 kAG rows are the real ones (one or
+// more 1 KB atoms of the 128-byte swizzle) and whose other rows are those of later chunks.  Those
+// rows give logits of rows past T, which nothing reads; the windows overlap, so the rows cost
+// (KB - 1) kAG KB + 16 KB instead of KB x 16 KB, and every stage of the ring carries W only.
+__host__ __device__ constexpr int d1_a_bytes(int kag, int kb) { return kag == 0 ? 0 : ((kb - 1) * kag + 16) * 1024; }
+__host__ __device__ constexpr int d1_stage_bytes(int kag) { return kag == 0 ? kAUnitBytes + kD1WBytes : kD1WBytes; }
 
 struct D1Shared {
-  uint64_t full[kD1Stages], empty[kD1Stages];
+  uint64_t full[kD1MaxStages], empty[kD1MaxStages];
   uint64_t z_full[kD1Buf], z_empty[kD1Buf];
-  uint64_t mma_done, ep_bar;
+  uint64_t a_full, mma_done, ep_bar;
   float mcs[kDecodeRows];  // each row's reference after tile jc - 1
   uint32_t tmem_base;
   volatile uint32_t abort_flag;
@@ -67,33 +110,39 @@ struct D1Args {
   int32_t V, nvz, KB;
   int32_t nsub;       // sub-tiles: nvz * NZ / 64
   int32_t rounds;     // ceil(nsub / gridDim.x)
-  float* smax;        // [T][nsub] row maxima of each sub-tile over its valid columns
+  uint64_t* smax;     // [T][nsub] row maxima of each sub-tile over its valid columns, tagged (zero at launch)
   float* mref;        // [nvz][T] reference of each row at each step
   float* csum;        // [T][nvz][NZ / 32] chunk sums
   float* zy;          // [T] target logits
   const int32_t* y;   // [T]
-  uint32_t* progress; // [gridDim.x] rounds whose maxima each CTA has published (zero at launch)
   int32_t* status;
   uint64_t limit_ns;
 };
 
-template <int kNZ>
+template <int kNZ, int kAG>
 __global__ void __launch_bounds__(kZtThreads, 1)
     k_lm_decode1(const __grid_constant__ CUtensorMap tm_h, const __grid_constant__ CUtensorMap tm_w, D1Args a) {
-  // tm_h: hidden [T][H], box {64, 128}; tm_w: W [V][H], box {64, 64}; both 128-byte swizzled
+  // tm_h: hidden [T][H], box {64, kAG ? 8 kAG : 128}; tm_w: W [V][H], box {64, 64}; both 128-byte
+  // swizzled
   constexpr int kSubPerTile = kNZ / kD1Sub;
   constexpr int kChunks = kNZ / 32;
+  constexpr int kStageBytes = d1_stage_bytes(kAG);
   extern __shared__ __align__(1024) uint8_t dsmem[];
-  D1Shared& sh = *reinterpret_cast<D1Shared*>(dsmem + kD1Stages * kD1StageBytes);
+  constexpr int kShBytes = static_cast<int>((sizeof(D1Shared) + 1023) / 1024 * 1024);
+  D1Shared& sh = *reinterpret_cast<D1Shared*>(dsmem + kD1Smem - kShBytes);
+  const int a_bytes = d1_a_bytes(kAG, a.KB);
+  const int nst_i = (kD1Smem - kShBytes - a_bytes) / kStageBytes;
+  const uint32_t nst = static_cast<uint32_t>(nst_i < kD1MaxStages ? nst_i : kD1MaxStages);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int G = static_cast<int>(gridDim.x);
   const int b = static_cast<int>(blockIdx.x);
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kD1Stages; ++i) {
+    for (int i = 0; i < kD1MaxStages; ++i) {
       mbar_init(&sh.full[i], 1);
       mbar_init(&sh.empty[i], 1);
     }
+    mbar_init(&sh.a_full, 1);
     for (int i = 0; i < kD1Buf; ++i) {
       mbar_init(&sh.z_full[i], 1);
       mbar_init(&sh.z_empty[i], 128);
@@ -112,12 +161,12 @@ __global__ void __launch_bounds__(kZtThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sh.tmem_base;
-  const uint32_t ring = smem_u32(dsmem);
-  const bool misaligned = (ring & 1023u) != 0;
+  const uint32_t abase = smem_u32(dsmem);            // resident hidden rows (kAG > 0)
+  const uint32_t ring = abase + static_cast<uint32_t>(a_bytes);
+  const bool misaligned = (abase & 1023u) != 0 || nst < 2;
   if (misaligned && threadIdx.x == 0) raise_status(a.status, 4 /* BI_ERR_CUDA */);
   const int rounds = misaligned ? 0 : a.rounds;
   const WaitCtl wc{&sh.abort_flag, a.status, a.limit_ns};
-  constexpr uint32_t nst = static_cast<uint32_t>(kD1Stages);
 
   if (warp == 0) {
     if (lane == 0) {
@@ -125,18 +174,32 @@ __global__ void __launch_bounds__(kZtThreads, 1)
       tma_prefetch_desc(&tm_w);
       uint32_t stage = 0, phase = 0;
       bool ok = true;
+      if (kAG > 0 && rounds > 0) {
+        // the real rows of every K chunk, once: chunk kb's 8 kAG rows at kb kAG KB
+        mbar_arrive_expect_tx(&sh.a_full, static_cast<uint32_t>(a.KB * kAG * 1024));
+        for (int kb = 0; kb < a.KB; ++kb) tma_load_2d(abase + kb * kAG * 1024, &tm_h, &sh.a_full, kb * 64, 0);
+      }
       for (int r = 0; ok && r < rounds; ++r) {
         const int sub = r * G + b;
         if (sub >= a.nsub) continue;
 #pragma unroll 1
         for (int kb = 0; kb < a.KB; ++kb) {
           if (!mbar_wait<false>(&sh.empty[stage], phase ^ 1u, wc)) { ok = false; break; }
-          mbar_arrive_expect_tx(&sh.full[stage], static_cast<uint32_t>(kD1StageBytes));
-          const uint32_t dst = ring + stage * kD1StageBytes;
-          tma_load_2d(dst, &tm_h, &sh.full[stage], kb * 64, 0);
-          tma_load_2d(dst + kAUnitBytes, &tm_w, &sh.full[stage], kb * 64, sub * kD1Sub);
+          mbar_arrive_expect_tx(&sh.full[stage], static_cast<uint32_t>(kStageBytes));
+          const uint32_t dst = ring + stage * kStageBytes;
+          if (kAG == 0) {
+            tma_load_2d(dst, &tm_h, &sh.full[stage], kb * 64, 0);
+            tma_load_2d(dst + kAUnitBytes, &tm_w, &sh.full[stage], kb * 64, sub * kD1Sub);
+          } else {
+            tma_load_2d(dst, &tm_w, &sh.full[stage], kb * 64, sub * kD1Sub);
+          }
           ring_advance(stage, phase, nst);
         }
+      }
+      if (kAG > 0 && rounds > 0) {
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_test(&sh.a_full, 0))
+          if (globaltimer_ns() - t0 > a.limit_ns) break;
       }
       for (uint32_t i = 0; i < nst; ++i) {
         const uint32_t ph = (i < stage) ? phase : (phase ^ 1u);
@@ -150,11 +213,12 @@ __global__ void __launch_bounds__(kZtThreads, 1)
     if (lane == 0) {
       // the cluster kernel's instruction sequence per 64-column chunk of K, with N = 64
       constexpr uint32_t idesc = idesc_bf16(128, kD1Sub, false, false);
-      constexpr uint64_t sb = static_cast<uint64_t>(kD1StageBytes >> 4);
-      const uint64_t dk0 = sdesc_k_sw128(ring);
-      const uint64_t dkb0 = sdesc_k_sw128(ring + kAUnitBytes);
+      constexpr uint64_t sb = static_cast<uint64_t>(kStageBytes >> 4);
+      const uint64_t dk0 = sdesc_k_sw128(kAG == 0 ? ring : abase);
+      const uint64_t dkb0 = sdesc_k_sw128(kAG == 0 ? ring + kAUnitBytes : ring);
       uint32_t stage = 0, phase = 0;
       bool ok = true;
+      if (kAG > 0 && rounds > 0 && !mbar_wait<false>(&sh.a_full, 0u, wc)) ok = false;
       for (int r = 0; ok && r < rounds; ++r) {
         const int sub = r * G + b;
         if (sub >= a.nsub) continue;
@@ -166,7 +230,7 @@ __global__ void __launch_bounds__(kZtThreads, 1)
         for (int kb = 0; kb < a.KB; ++kb) {
           if (!mbar_wait<false>(&sh.full[stage], phase, wc)) { ok = false; break; }
           tc_fence_after();
-          const uint64_t da = dk0 + stage * sb;
+          const uint64_t da = kAG == 0 ? dk0 + stage * sb : dk0 + static_cast<uint64_t>((kb * kAG * 1024) >> 4);
           const uint64_t db = dkb0 + stage * sb;
           umma_bf16(zt, da, db, idesc, kb != 0 ? 1u : 0u);
           umma_bf16(zt, da + 2, db + 2, idesc, 1u);
@@ -212,78 +276,87 @@ __global__ void __launch_bounds__(kZtThreads, 1)
               for (int q = 0; q < 32; ++q)
                 if (vb + q < a.V) M = fmaxf(M, __uint_as_float(v[q]));
             }
-            if (real) a.smax[static_cast<int64_t>(row) * a.nsub + sub] = M;
+            if (real) st_relaxed_gpu_u64(a.smax + static_cast<int64_t>(row) * a.nsub + sub, kD1Tag | __float_as_uint(M));
           }
         }
-        // this round's maxima are written by every epilogue thread: publish the progress
-        __threadfence();
-        mbar_arrive(&sh.ep_bar);
-        if (!__all_sync(0xffffffffu, mbar_wait<false>(&sh.ep_bar, (epc++) & 1u, wc))) { ok = false; break; }
-        if (et == 0) st_release_gpu_u32(a.progress + b, static_cast<uint32_t>(r + 1));
       }
       const int qr = r - kD1Lag;
       if (qr < 0 || qr >= rounds) continue;
       const int sub = qr * G + b;
       if (sub >= a.nsub) continue;
       const int j = sub / kSubPerTile;
-      // every CTA has published the maxima of the rounds holding tiles 0 .. j: the first epilogue
-      // warp reads the G flags 32 at a time (relaxed), and once all are there an acquire fence
-      // orders the maxima reads after them; the CTA barrier below passes that on
-      const uint32_t need = static_cast<uint32_t>(((j + 1) * kSubPerTile - 1) / G + 1);
-      if (et < 32) {
-        const uint64_t t0 = globaltimer_ns();
-        uint32_t spins = 0;
-        while (true) {
-          bool mine = true;
-          for (int c = et; c < G; c += 32) mine = mine && (ld_relaxed_gpu_u32(a.progress + c) >= need);
-          if (__all_sync(0xffffffffu, mine)) break;
-          if ((++spins & 15u) == 0) {
-            const bool stop = sh.abort_flag != 0u || globaltimer_ns() - t0 > a.limit_ns;
-            if (__any_sync(0xffffffffu, stop)) {
-              if (et == 0 && sh.abort_flag == 0u) {
-                raise_status(a.status, 5 /* BI_ERR_TIMEOUT */);
-                sh.abort_flag = 1u;
-              }
-              ok = false;
-              break;
-            }
-          }
-        }
-        fence_acq_rel_gpu();
-      }
-      mbar_arrive(&sh.ep_bar);
-      if (!__all_sync(0xffffffffu, mbar_wait<false>(&sh.ep_bar, (epc++) & 1u, wc))) { ok = false; break; }
-      if (sh.abort_flag) { ok = false; break; }
       const uint32_t bb = static_cast<uint32_t>(qr % kD1Buf);
       if (jc <= j) {
-        // advance every row's chain over tiles jc .. j, a warp per row: the range's largest
-        // sub-tile maximum first (coalesced loads); only when it could raise the reference are the
-        // tiles walked in order, 32 at a time (lane l takes tile base + l, the chain runs over
-        // the lanes by shuffles), as the cluster kernel's producers pass the reference on
-        const int ew = warp - 2;  // 0..3
-        for (int r = ew; r < static_cast<int>(a.T); r += 4) {
-          const float* rr = a.smax + static_cast<int64_t>(r) * a.nsub;
-          float m = sh.mcs[r];
-          float mx = -INFINITY;
-          for (int i = jc * kSubPerTile + lane; i < (j + 1) * kSubPerTile; i += 32) mx = fmaxf(mx, __ldcg(rr + i));
+        // advance every row's chain over tiles jc .. j, as the cluster kernel's producers pass the
+        // reference on.  The range's largest sub-tile maximum is checked first: only when it could
+        // raise the reference are the tiles walked in order.  Few rows: a warp per row (coalesced
+        // loads, the ordered walk 32 tiles at a time over the lanes by shuffles).  Many rows: each
+        // row's owner thread alone, its loads independent of one another.
+        // (each entry is waited for until its writer has stored it: by the schedule it nearly
+        // always has, the entries a round needs being at least two rounds old)
+        const int lo = jc * kSubPerTile, hi = (j + 1) * kSubPerTile;
+        bool good = true;
+        if (a.T <= 8) {
+          const int ew = warp - 2;  // 0..3
+          for (int r = ew; r < static_cast<int>(a.T); r += 4) {
+            const uint64_t* rr = a.smax + static_cast<int64_t>(r) * a.nsub;
+            float m = sh.mcs[r];
+            float mx = -INFINITY;
+            for (int i = lo + lane; i < hi; i += 32) {
+              float v;
+              good = good && d1_entry(rr, i, v, &sh.abort_flag, a.status, a.limit_ns);
+              mx = fmaxf(mx, v);
+            }
+            if (!__all_sync(0xffffffffu, good)) { good = false; break; }
 #pragma unroll
-          for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-          if (mx > m + kTau) {
-            for (int base = jc; base <= j; base += 32) {
-              float Ml = -INFINITY;
-              if (base + lane <= j) {
+            for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            if (mx > m + kTau) {
+              for (int base = jc; base <= j; base += 32) {
+                float Ml = -INFINITY;
+                if (base + lane <= j) {
 #pragma unroll
-                for (int i = 0; i < kSubPerTile; ++i) Ml = fmaxf(Ml, __ldcg(rr + (base + lane) * kSubPerTile + i));
-              }
-              const int nt = (j - base + 1) < 32 ? (j - base + 1) : 32;
-              for (int l = 0; l < nt; ++l) {
-                const float M = __shfl_sync(0xffffffffu, Ml, l);
-                m = (M > m + kTau) ? M : m;
+                  for (int i = 0; i < kSubPerTile; ++i) Ml = fmaxf(Ml, d1_value(ld_relaxed_gpu_u64(rr + (base + lane) * kSubPerTile + i)));
+                }
+                const int nt = (j - base + 1) < 32 ? (j - base + 1) : 32;
+                for (int l = 0; l < nt; ++l) {
+                  const float M = __shfl_sync(0xffffffffu, Ml, l);
+                  m = (M > m + kTau) ? M : m;
+                }
               }
             }
+            if (lane == 0) sh.mcs[r] = m;
           }
-          if (lane == 0) sh.mcs[r] = m;
+        } else if (real) {
+          const uint64_t* rr = a.smax + static_cast<int64_t>(row) * a.nsub;
+          float m = sh.mcs[row];
+          float mx = -INFINITY;
+          uint64_t tags = kD1Tag;
+#pragma unroll 16
+          for (int i = lo; i < hi; ++i) {
+            const uint64_t w = ld_relaxed_gpu_u64(rr + i);
+            tags &= w;
+            mx = fmaxf(mx, d1_value(w));
+          }
+          if (!(tags & kD1Tag)) {
+            // an entry was not there yet: the range again, waiting for each
+            mx = -INFINITY;
+            for (int i = lo; i < hi && good; ++i) {
+              float v;
+              good = d1_entry(rr, i, v, &sh.abort_flag, a.status, a.limit_ns);
+              mx = fmaxf(mx, v);
+            }
+          }
+          if (good && mx > m + kTau) {
+            for (int t = jc; t <= j; ++t) {
+              float M = -INFINITY;
+#pragma unroll
+              for (int i = 0; i < kSubPerTile; ++i) M = fmaxf(M, d1_value(ld_relaxed_gpu_u64(rr + t * kSubPerTile + i)));
+              m = (M > m + kTau) ? M : m;
+            }
+          }
+          sh.mcs[row] = m;
         }
+        if (!good) sh.abort_flag = 1u;
         jc = j + 1;
         mbar_arrive(&sh.ep_bar);
         if (!__all_sync(0xffffffffu, mbar_wait<false>(&sh.ep_bar, (epc++) & 1u, wc))) { ok = false; break; }

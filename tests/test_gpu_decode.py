@@ -37,7 +37,9 @@ def test_few_rows_bitwise_equal_to_packed_batch(H, V, cuda_device):
     h, w, y = random_inputs(300, H, V, seed=H + V)
     h, w, y = h.to(cuda_device), w.to(cuda_device), y.to(cuda_device)
     packed_lp, packed_lse = _lp(h, w, y, cuda_device)          # 300 rows: the cluster kernel
-    for rows in ([0], [5, 17, 299], list(range(128)), list(range(172, 300))):
+    # 1, 3, 12 and 20 rows keep their hidden rows resident (one, two or four 8-row atoms); 128 rows
+    # stream them with every stage
+    for rows in ([0], [5, 17, 299], list(range(128)), list(range(172, 300)), list(range(40, 52)), list(range(7, 27))):
         r = torch.tensor(rows, device=cuda_device)
         lp, lse = _lp(h[r].contiguous(), w, y[r].contiguous(), cuda_device)   # <= 128 rows: every SM
         assert torch.equal(lp, packed_lp[r]), f"logprob bits differ (H={H}, V={V}, {len(rows)} rows)"
