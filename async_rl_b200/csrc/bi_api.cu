@@ -467,18 +467,19 @@ int logprob_decode(const uint16_t* hidden, const uint16_t* w_lm, const int32_t* 
                    int32_t V, float* logprob, float* lse, int32_t* dev_status, uint8_t* ws, const WsLayout& L,
                    const DevInfo* di, cudaStream_t s) {
   const LmPlan pl = plan_lm(H, di);
-  if (pl.C == 0 || pl.C > 8 || !di->coop || pl.NZ % bi::kD1Sub != 0) return kDecodeUnsupported;
+  if (pl.C == 0 || pl.C > 8 || !di->coop || pl.NZ % 64 != 0) return kDecodeUnsupported;
+  const int sub = bi::d1_sub(pl.NZ);
   const int nvz = (V + pl.NZ - 1) / pl.NZ;
   const size_t zsm = bi::zscan_smem(nvz, pl.NZ);
   if (zsm > kZscanSmemMax) return kDecodeUnsupported;
   // hidden rows kept resident in 1 KB atoms of 8 rows when few (the ring then carries W only)
   int ag = T <= 8 ? 1 : (T <= 16 ? 2 : (T <= 32 ? 4 : 0));
-  if (ag > 0 && bi::d1_a_bytes(ag, H / 64) + 4 * bi::kD1WBytes + 4096 > bi::kD1Smem) ag = 0;
+  if (ag > 0 && bi::d1_a_bytes(ag, H / 64) + 4 * bi::d1_stage_bytes(ag, sub) + 4096 > bi::kD1Smem) ag = 0;
   CUtensorMap tm_h, tm_w64;
-  if (!make_map(&tm_h, hidden, T, H, ag > 0 ? 8 * ag : 128) || !make_map(&tm_w64, w_lm, V, H, bi::kD1Sub))
+  if (!make_map(&tm_h, hidden, T, H, ag > 0 ? 8 * ag : 128) || !make_map(&tm_w64, w_lm, V, H, sub))
     return BI_ERR_CUDA;
-  const int nsub = nvz * (pl.NZ / bi::kD1Sub);
-  const int G = nsub < di->sms ? nsub : di->sms;  // >= NZ / 64 sub-tiles: every wait has a finite target
+  const int nsub = nvz * (pl.NZ / sub);
+  const int G = nsub < di->sms ? nsub : di->sms;  // >= NZ / sub sub-tiles: every wait has a finite target
   bi::D1Args d{};
   d.T = T;
   d.V = V;

@@ -21,12 +21,12 @@ constexpr int kZtThreads = 192;   // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 // ---------------------------------------------------------------------------------------------
 // Single pass (k_lm_decode1): one cooperative launch, one CTA per SM, W read once.
 //
-// The vocabulary is cut into 64-column sub-tiles (an NZ-wide tile of the cluster kernel is NZ / 64
+// The vocabulary is cut into 128-column sub-tiles (an NZ-wide tile of the cluster kernel is NZ / 128
 // of them; a logit column's value does not depend on the N of the instruction that computes it,
 // only on its row of A, its row of B and the K order, which are the cluster kernel's).  Sub-tile
 // s is handled by CTA s mod G in round s div G, which spreads the vocabulary evenly over the SMs.
-// Per round a CTA computes its sub-tile's logits into one of eight TMEM buffers, takes the row
-// maxima over the valid columns and stores each as a tagged 64-bit word.  Five rounds later it
+// Per round a CTA computes its sub-tile's logits into one of four TMEM buffers, takes the row
+// maxima over the valid columns and stores each as a tagged 64-bit word.  Two rounds later it
 // forms the sub-tile's 32-column chunk sums: each row's reference chain is first advanced up to
 // this tile, as the cluster kernel's producers pass it on, from the maxima of every sub-tile of the
 // tiles up to this one, each read (and waited for, bounded, should its writer not have stored it
@@ -78,13 +78,15 @@ __device__ __forceinline__ bool d1_entry(const uint64_t* rr, int i, float& v, vo
   }
 }
 
-constexpr int kD1Sub = 64;     // columns of a sub-tile (one MMA of N = 64)
+// Columns of a sub-tile (one MMA of that N): 128 where it divides the tile width NZ, else 64.  A
+// narrower MMA costs the issuing thread about as much as a wide one, so sub-tiles are as wide as
+// the balance over the SMs allows.
+__host__ __device__ constexpr int d1_sub(int nz) { return nz % 128 == 0 ? 128 : 64; }
 constexpr int kD1MaxStages = 24;
-constexpr int kD1Buf = 8;      // logit buffers in TMEM (8 x 64 columns)
-constexpr int kD1Lag = 5;      // rounds between a sub-tile's maxima and its chunk sums: a round's sums
-                               // need every CTA's maxima of at most the next round, so the waits
-                               // have three rounds of slack
-constexpr int kD1WBytes = kD1Sub * 128;  // W rows [64 x 64]
+constexpr int kD1MaxBuf = 8;   // logit buffers in TMEM: 512 / sub-tile width
+// Rounds between a sub-tile's maxima and its chunk sums (buffers - 2): a round's sums need every
+// CTA's maxima of at most the next round.
+__host__ __device__ constexpr int d1_lag(int sub) { return 512 / sub - 2; }
 constexpr int kD1Smem = kLmSmemLimit;     // the ring takes what the resident rows leave
 
 // Hidden rows, the A operand of every sub-tile, are either streamed with each stage (kAG = 0: a
@@ -94,11 +96,12 @@ constexpr int kD1Smem = kLmSmemLimit;     // the ring takes what the resident ro
 // rows give logits of rows past T, which nothing reads; the windows overlap, so the rows cost
 // (KB - 1) kAG KB + 16 KB instead of KB x 16 KB, and every stage of the ring carries W only.
 __host__ __device__ constexpr int d1_a_bytes(int kag, int kb) { return kag == 0 ? 0 : ((kb - 1) * kag + 16) * 1024; }
-__host__ __device__ constexpr int d1_stage_bytes(int kag) { return kag == 0 ? kAUnitBytes + kD1WBytes : kD1WBytes; }
+// A stage: W rows [sub x 64] (and the hidden rows' [128 x 64] box when they are not resident).
+__host__ __device__ constexpr int d1_stage_bytes(int kag, int sub) { return (kag == 0 ? kAUnitBytes : 0) + sub * 128; }
 
 struct D1Shared {
   uint64_t full[kD1MaxStages], empty[kD1MaxStages];
-  uint64_t z_full[kD1Buf], z_empty[kD1Buf];
+  uint64_t z_full[kD1MaxBuf], z_empty[kD1MaxBuf];
   uint64_t a_full, mma_done, ep_bar;
   float mcs[kDecodeRows];  // each row's reference after tile jc - 1
   uint32_t tmem_base;
@@ -108,7 +111,7 @@ struct D1Shared {
 struct D1Args {
   int64_t T;          // real rows (<= 128)
   int32_t V, nvz, KB;
-  int32_t nsub;       // sub-tiles: nvz * NZ / 64
+  int32_t nsub;       // sub-tiles: nvz * NZ / sub-tile width
   int32_t rounds;     // ceil(nsub / gridDim.x)
   uint64_t* smax;     // [T][nsub] row maxima of each sub-tile over its valid columns, tagged (zero at launch)
   float* mref;        // [nvz][T] reference of each row at each step
@@ -122,11 +125,14 @@ struct D1Args {
 template <int kNZ, int kAG>
 __global__ void __launch_bounds__(kZtThreads, 1)
     k_lm_decode1(const __grid_constant__ CUtensorMap tm_h, const __grid_constant__ CUtensorMap tm_w, D1Args a) {
-  // tm_h: hidden [T][H], box {64, kAG ? 8 kAG : 128}; tm_w: W [V][H], box {64, 64}; both 128-byte
-  // swizzled
+  // tm_h: hidden [T][H], box {64, kAG ? 8 kAG : 128}; tm_w: W [V][H], box {64, sub-tile width};
+  // both 128-byte swizzled
+  constexpr int kD1Sub = d1_sub(kNZ);
+  constexpr int kD1Buf = 512 / kD1Sub;
+  constexpr int kD1Lag = d1_lag(kD1Sub);
   constexpr int kSubPerTile = kNZ / kD1Sub;
   constexpr int kChunks = kNZ / 32;
-  constexpr int kStageBytes = d1_stage_bytes(kAG);
+  constexpr int kStageBytes = d1_stage_bytes(kAG, kD1Sub);
   extern __shared__ __align__(1024) uint8_t dsmem[];
   constexpr int kShBytes = static_cast<int>((sizeof(D1Shared) + 1023) / 1024 * 1024);
   D1Shared& sh = *reinterpret_cast<D1Shared*>(dsmem + kD1Smem - kShBytes);
@@ -211,7 +217,7 @@ __global__ void __launch_bounds__(kZtThreads, 1)
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
-      // the cluster kernel's instruction sequence per 64-column chunk of K, with N = 64
+      // the cluster kernel's instruction sequence per 64-column chunk of K, with N = sub-tile width
       constexpr uint32_t idesc = idesc_bf16(128, kD1Sub, false, false);
       constexpr uint64_t sb = static_cast<uint64_t>(kStageBytes >> 4);
       const uint64_t dk0 = sdesc_k_sw128(kAG == 0 ? ring : abase);
@@ -365,7 +371,8 @@ __global__ void __launch_bounds__(kZtThreads, 1)
       if (warp_rows) {
         if (real && sub % kSubPerTile == 0) a.mref[static_cast<int64_t>(j) * a.T + row] = mc;
         const float mn2 = (real ? mc : 0.f) * kLog2e;
-        float* cs_out = a.csum + (static_cast<int64_t>(real ? row : 0) * a.nvz + j) * kChunks + (sub % kSubPerTile) * 2;
+        float* cs_out = a.csum + (static_cast<int64_t>(real ? row : 0) * a.nvz + j) * kChunks +
+                        (sub % kSubPerTile) * (kD1Sub / 32);
 #pragma unroll 1
         for (int c = 0; c < kD1Sub / 32; ++c) {
           uint32_t v[32];
