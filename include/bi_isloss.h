@@ -158,9 +158,9 @@ BI_API size_t bi_workspace_bytes_pstore(int64_t T, int32_t H, int32_t V, int32_t
  * A row gets identical bits whether it is scored alone (T = 1, decode style) or packed.  Packed
  * batches run on the cluster kernel (one cluster sweeps the vocabulary for each 128-row tile).
  * With 1 <= T <= 128 and a workspace of bi_workspace_bytes(T, H, V, 0) bytes the rows are scored
- * on every SM instead, in one cooperative pass over W: the logits of 64-column sub-tiles with the
+ * on every SM instead, in one cooperative pass over W: the logits of 128-column sub-tiles with the
  * cluster kernel's per-column instruction sequence give the row maxima, every CTA advances the
- * reference chain once the maxima of the tiles it needs are published, forms the 32-column partial
+ * reference chain once the maxima of the tiles it needs are stored, forms the 32-column partial
  * sums against each step's reference, and a per-row combine follows the cluster kernel's class
  * order, which reproduces its bits ("Zero Mismatch, Simple Async RL", section "Alignment permits a
  * simpler learning path").  Without cooperative launch support the rows go to the cluster kernel,
