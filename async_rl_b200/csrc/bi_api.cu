@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <array>
 #include <cmath>
 #include <cstdint>
@@ -36,11 +37,12 @@ thread_local uint64_t g_force_timeout_ns = 0;
 // ---------------------------------------------------------------------------------------------
 enum KernelKind : int { kKPrep, kKRowmap, kKZeroRows, kKGather, kKLmFwd, kKLmFwdDH, kKLmDW, kKDwRows,
                         kKDwStream, kKSeqGate, kKRowParts, kKReduce, kKD3Partial, kKGemm, kKRmsNorm, kKLmZscan,
-                        kKLmDecode1, kNumKinds };
+                        kKLmDecode1, kKD1Zero, kNumKinds };
 const char* const kKindNames[kNumKinds] = {"k_prep", "k_rowmap", "k_zero_prompt_rows", "k_gather_rows",
                                            "k_lm_fwd", "k_lm_fwd_dh", "k_lm_dw", "k_dw_rows", "k_dw_stream",
                                            "k_seq_gate", "k_row_parts", "k_reduce_parts", "k_d3_partial",
-                                           "k_gemm_pair", "k_rmsnorm", "k_lm_zscan", "k_lm_decode1"};
+                                           "k_gemm_pair", "k_rmsnorm", "k_lm_zscan", "k_lm_decode1",
+                                           "k_d1_zero"};
 static_assert(sizeof(bi::D3Out) == sizeof(bi_d3), "device-written diagnostics match the ABI struct");
 struct Pending {
   int kind;
@@ -110,6 +112,23 @@ constexpr size_t kFinBytes = static_cast<size_t>(kMaxSms) * 2 * 384 * sizeof(flo
 // references ([ceil(V / 128)][T] fp32, enough for any tile width NZ >= 128), 32-column partial
 // sums ([T][V / 32 + 8] fp32 at most), the target logits ([T] fp32) and the row maxima of
 // 64-column sub-tiles ([T][V / 64 + 4] tagged 64-bit words at most).  Nothing of size T x V.
+bool split_ok(int32_t H, int c);
+int logit_cols(int Hs);
+
+// Sub-tiles of the all-SM decode pass for the widest plan any valid split of H gives (the plan
+// chosen on a device is one of them).
+size_t decode_subtiles_max(int32_t H, int32_t V) {
+  size_t n = 0;
+  for (int c = 1; c <= bi::kMaxCluster; ++c) {
+    if (!split_ok(H, c)) continue;
+    const int nz = logit_cols(H / c);
+    if (nz < 64) continue;
+    const size_t ns = static_cast<size_t>((V + nz - 1) / nz) * static_cast<size_t>(nz / bi::d1_sub(nz));
+    n = ns > n ? ns : n;
+  }
+  return n;
+}
+
 WsLayout ws_layout(int64_t T, int32_t H, int32_t V, int32_t R, bool store, bool decode = false) {
   WsLayout L{};
   const size_t t = static_cast<size_t>(T > 0 ? T : 1);
@@ -159,7 +178,7 @@ WsLayout ws_layout(int64_t T, int32_t H, int32_t V, int32_t R, bool store, bool 
     L.zmref = take(t * ntile * 4);
     L.zcsum = take(t * (static_cast<size_t>(V + 31) / 32 + 8) * 4);
     L.zy = take(t * 4);
-    L.zsmax = take(t * (static_cast<size_t>(V + 63) / 64 + 4) * 8);
+    L.zsmax = take(t * decode_subtiles_max(H, V) * 8);
   }
   L.total = o;
   return L;
@@ -479,6 +498,7 @@ int logprob_decode(const uint16_t* hidden, const uint16_t* w_lm, const int32_t* 
   if (!make_map(&tm_h, hidden, T, H, ag > 0 ? 8 * ag : 128) || !make_map(&tm_w64, w_lm, V, H, sub))
     return BI_ERR_CUDA;
   const int nsub = nvz * (pl.NZ / sub);
+  if (static_cast<size_t>(nsub) > decode_subtiles_max(H, V)) return kDecodeUnsupported;  // not held by L.zsmax
   const int G = nsub < di->sms ? nsub : di->sms;  // >= NZ / sub sub-tiles: every wait has a finite target
   bi::D1Args d{};
   d.T = T;
@@ -494,8 +514,14 @@ int logprob_decode(const uint16_t* hidden, const uint16_t* w_lm, const int32_t* 
   d.y = targets;
   d.status = dev_status;
   d.limit_ns = kWaitLimitNs;
-  // the tagged maxima start untagged: a reader waits for its writer's tag
-  if (cudaMemsetAsync(d.smax, 0, static_cast<size_t>(T) * nsub * 8, s) != cudaSuccess) return BI_ERR_CUDA;
+  // the status word and the tagged maxima start at zero (a reader waits for its writer's tag)
+  {
+    ProfScope ps(kKD1Zero, s);
+    const int64_t nz = T * static_cast<int64_t>(nsub);
+    const unsigned zb = static_cast<unsigned>(std::min<int64_t>((nz + 255) / 256, 4 * di->sms));
+    bi::k_d1_zero<<<zb, 256, 0, s>>>(d.smax, nz, dev_status);
+    if (cudaGetLastError() != cudaSuccess) return BI_ERR_CUDA;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(G), 1, 1);
   cfg.blockDim = dim3(bi::kZtThreads, 1, 1);
@@ -519,14 +545,28 @@ int logprob_decode(const uint16_t* hidden, const uint16_t* w_lm, const int32_t* 
 #undef BI_D1_LAUNCH
   }
   if (e != cudaSuccess) return BI_ERR_CUDA;
+  // the combine as a programmatic dependent of the pass: its launch overlaps the pass, and it waits
+  // for the pass's completion before reading (a plain launch where the attribute is refused)
   ProfScope ps(kKLmZscan, s);
-  const unsigned rows = static_cast<unsigned>(T);
-  switch (pl.NZ) {
-    case 256: bi::k_lm_zscan<256><<<rows, bi::kZsThreads, zsm, s>>>(d.csum, d.mref, d.zy, targets, T, V, nvz, pl.C, logprob, lse, dev_status); break;
-    case 192: bi::k_lm_zscan<192><<<rows, bi::kZsThreads, zsm, s>>>(d.csum, d.mref, d.zy, targets, T, V, nvz, pl.C, logprob, lse, dev_status); break;
-    default:  bi::k_lm_zscan<128><<<rows, bi::kZsThreads, zsm, s>>>(d.csum, d.mref, d.zy, targets, T, V, nvz, pl.C, logprob, lse, dev_status); break;
+  cudaLaunchConfig_t zc = {};
+  zc.gridDim = dim3(static_cast<unsigned>(T), 1, 1);
+  zc.blockDim = dim3(bi::kZsThreads, 1, 1);
+  zc.dynamicSmemBytes = zsm;
+  zc.stream = s;
+  cudaLaunchAttribute zattr[1];
+  zattr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  zattr[0].val.programmaticStreamSerializationAllowed = 1;
+  zc.attrs = zattr;
+  zc.numAttrs = 1;
+  auto* zk = pl.NZ == 256 ? bi::k_lm_zscan<256> : (pl.NZ == 192 ? bi::k_lm_zscan<192> : bi::k_lm_zscan<128>);
+  const int32_t Cz = pl.C;
+  e = cudaLaunchKernelEx(&zc, zk, d.csum, d.mref, d.zy, targets, T, V, nvz, Cz, logprob, lse, dev_status);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    zc.numAttrs = 0;
+    e = cudaLaunchKernelEx(&zc, zk, d.csum, d.mref, d.zy, targets, T, V, nvz, Cz, logprob, lse, dev_status);
   }
-  return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+  return e == cudaSuccess ? BI_OK : BI_ERR_CUDA;
 }
 
 }  // namespace
@@ -645,15 +685,16 @@ bi_status bi_logprob_fwd(const uint16_t* hidden, const uint16_t* w_lm, const int
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const DevInfo* di = device_info();
   if (!di) return BI_ERR_CUDA;
-  if (cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s) != cudaSuccess) return BI_ERR_CUDA;
-  if (T == 0) return BI_OK;
-  // a few rows: the same bits from every SM when the workspace holds their logits
+  // a few rows: the same bits from every SM when the workspace holds their logits (that path
+  // zeroes the status word itself, in the launch that zeroes its tagged maxima)
   const WsLayout Ld = ws_layout(T, H, V, 0, false, true);
-  if (Ld.decode && ws_bytes >= Ld.total && force == 0) {
+  if (T > 0 && Ld.decode && ws_bytes >= Ld.total && force == 0) {
     const int r = logprob_decode(hidden, w_lm, targets, T, H, V, logprob, lse, dev_status, static_cast<uint8_t*>(ws),
                                  Ld, di, s);
     if (r != kDecodeUnsupported) return static_cast<bi_status>(r);
   }
+  if (cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s) != cudaSuccess) return BI_ERR_CUDA;
+  if (T == 0) return BI_OK;
   float* fin = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + L.fin);
   return logprob_forward(hidden, w_lm, targets, T, H, V, logprob, lse, dev_status, fin, force, di, s);
 }

@@ -143,6 +143,8 @@ __global__ void __launch_bounds__(kZtThreads, 1)
   const int lane = threadIdx.x & 31;
   const int G = static_cast<int>(gridDim.x);
   const int b = static_cast<int>(blockIdx.x);
+  // the combine kernel may be launched now; it waits for this grid's completion before reading
+  pdl_launch_dependents();
   if (threadIdx.x == 0) {
     for (int i = 0; i < kD1MaxStages; ++i) {
       mbar_init(&sh.full[i], 1);
@@ -411,7 +413,16 @@ __global__ void __launch_bounds__(kZtThreads, 1)
   }
 }
 
+// The status word and the tagged maxima zeroed in one launch: a maximum's reader waits for its
+// writer's tag, so the words must start untagged.
+__global__ void k_d1_zero(uint64_t* __restrict__ smax, int64_t n, int32_t* __restrict__ status) {
+  const int64_t i0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i0 == 0) *status = 0;
+  for (int64_t i = i0; i < n; i += static_cast<int64_t>(gridDim.x) * blockDim.x) smax[i] = 0;
+}
+
 constexpr int kZsThreads = 256;
+constexpr int kZsBatch = 8;    // loads in flight per thread while staging
 
 // Dynamic shared memory of k_lm_zscan: one row's chunk sums and references.
 __host__ __device__ constexpr size_t zscan_smem(int nvz, int nz) {
@@ -432,10 +443,27 @@ __global__ void __launch_bounds__(kZsThreads)
   float* mr = zs + static_cast<int64_t>(nvz) * kChunks;      // [nvz]
   __shared__ float cls[2 * 8];  // [8] class reference, [8] class sum
   const int64_t t = blockIdx.x;
+  // launched as a programmatic dependent of k_lm_decode1: its sums are read only once it completed
+  pdl_wait_primary();
   if (t >= T) return;
   const float* crow = csum + t * static_cast<int64_t>(nvz) * kChunks;
-  for (int i = threadIdx.x; i < nvz * kChunks; i += kZsThreads) cs[i] = crow[i];
-  for (int j = threadIdx.x; j < nvz; j += kZsThreads) mr[j] = mref[static_cast<int64_t>(j) * T + t];
+  // staged in batches of kZsBatch independent loads per thread, so that a batch costs one L2 round
+  // trip rather than one per element
+  const int ncs = nvz * kChunks;
+#pragma unroll 1
+  for (int base = 0; base < ncs + nvz; base += kZsThreads * kZsBatch) {
+    float v[kZsBatch];
+#pragma unroll
+    for (int u = 0; u < kZsBatch; ++u) {
+      const int i = base + u * kZsThreads + static_cast<int>(threadIdx.x);
+      v[u] = i < ncs ? __ldcg(crow + i) : (i < ncs + nvz ? __ldcg(mref + static_cast<int64_t>(i - ncs) * T + t) : 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < kZsBatch; ++u) {
+      const int i = base + u * kZsThreads + static_cast<int>(threadIdx.x);
+      if (i < ncs + nvz) zs[i] = v[u];  // cs, then mr right after it
+    }
+  }
   __syncthreads();
   // class k: its steps in order, rescaled at each change of reference
   if (static_cast<int>(threadIdx.x) < C) {

@@ -102,6 +102,7 @@ def test_decode_workload_line():
     line = _run(["--workload", "decode", "--steps", "20", "--warmup", "3"], timeout=900)
     for k in REQUIRED + ("roofline", "clocks", "gpu_launches", "cluster_kernel_ms", "rows_128_ms"):
         assert k in line, k
-    # two launches per one-row call: the single pass over W on every SM, then the combine
-    assert line["gpu_launches"] == 2 * 20 and line["value"] < line["cluster_kernel_ms"]
+    # three launches per one-row call: zeroing of the status and the tagged maxima, the single
+    # pass over W on every SM, then the combine
+    assert line["gpu_launches"] == 3 * 20 and line["value"] < line["cluster_kernel_ms"]
     assert 0 < line["roofline"]["frac"] < 2 and line["e2e"]["h2d_bytes_per_step"] > 0
