@@ -15,6 +15,13 @@
 
 namespace bi {
 
+// Programmatic dependent launch (sm_90+): a kernel launched with programmatic stream
+// serialization may start while the previous kernel of the stream runs; it must wait for that
+// kernel's completion (and its memory) before touching its results.  Without the launch attribute
+// both instructions are no-ops.
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait_primary() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 constexpr int kDecodeRows = 128;  // rows one tile holds: the largest T this path serves
 constexpr int kZtThreads = 192;   // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 

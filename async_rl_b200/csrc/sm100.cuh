@@ -107,13 +107,6 @@ __device__ __forceinline__ bool mbar_test_acq_cluster(uint64_t* bar, uint32_t pa
   return ok != 0;
 }
 
-// Programmatic dependent launch (sm_90+): a kernel launched with programmatic stream
-// serialization may start while the previous kernel of the stream runs; it must wait for that
-// kernel's completion (and its memory) before touching its results.  Without the launch attribute
-// both instructions are no-ops.
-__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-__device__ __forceinline__ void pdl_wait_primary() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-
 // Bounded wait state shared by all roles of a CTA.  A wait that runs longer than `limit_ns`
 // records BI_ERR_TIMEOUT in the global status, raises the CTA's abort flag and returns false;
 // a wait also returns false as soon as another role (or a peer CTA) raised the abort flag.
