@@ -134,9 +134,11 @@ typedef struct {
  * copy of the scored hidden rows (T H bf16), per-response coefficients and a fixed-size scratch for
  * the tiles the cluster passes between its CTAs; dW recomputes the logits tile by tile.
  * For bi_logprob_fwd with 1 <= T <= 128 rows (decode-style scoring) it also holds what the all-SM
- * path keeps: row maxima of 64-column sub-tiles, each step's reference and 32-column partial sums
- * of e^{z - m} (about 4 T V / 18 bytes at most), so that the call runs on every SM instead of one
- * cluster; the bits are the same either way. */
+ * path keeps: each row's maximum over every 128-column sub-tile (64-column where 128 does not
+ * divide the logit-tile width; one 8-byte word each), each step's reference and the 32-column
+ * partial sums of e^{z - m} (about 4 T V / 18 bytes at H = 1536, V = 151936: 1/18 of the rows'
+ * fp32 logits), so that the call runs on every SM instead of one cluster; the bits are the same
+ * either way. */
 BI_API size_t bi_workspace_bytes(int64_t T, int32_t H, int32_t V, int32_t R);
 
 /* Smallest workspace accepted.  For bi_is_loss_fwd_bwd it equals bi_workspace_bytes.  For R = 0 it
