@@ -264,7 +264,7 @@ int query_clusters(int C) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(C, 1, 1);
   cfg.blockDim = dim3(bi::LmThreads<kMode>::value, 1, 1);
-  cfg.dynamicSmemBytes = bi::LmTile<256, 256>::smem;
+  cfg.dynamicSmemBytes = bi::LmTile<kMode, 256, 256>::smem;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = C;
@@ -296,13 +296,13 @@ bool set_lm_attributes() {
 #define BI_SET_ATTR(NZ_, HS_)                                                                                  \
   ok = ok && cudaFuncSetAttribute(bi::k_lm_cluster<bi::kModeFwd, NZ_, HS_>,                                   \
                                   cudaFuncAttributeMaxDynamicSharedMemorySize,                                \
-                                  bi::LmTile<NZ_, HS_>::smem) == cudaSuccess;                                 \
+                                  bi::LmTile<bi::kModeFwd, NZ_, HS_>::smem) == cudaSuccess;                   \
   ok = ok && cudaFuncSetAttribute(bi::k_lm_cluster<bi::kModeFwdDH, NZ_, HS_>,                                 \
                                   cudaFuncAttributeMaxDynamicSharedMemorySize,                                \
-                                  bi::LmTile<NZ_, HS_>::smem) == cudaSuccess;                                 \
+                                  bi::LmTile<bi::kModeFwdDH, NZ_, HS_>::smem) == cudaSuccess;                 \
   ok = ok && cudaFuncSetAttribute(bi::k_lm_cluster<bi::kModeDW, NZ_, HS_>,                                    \
                                   cudaFuncAttributeMaxDynamicSharedMemorySize,                                \
-                                  bi::LmTile<NZ_, HS_>::smem) == cudaSuccess;
+                                  bi::LmTile<bi::kModeDW, NZ_, HS_>::smem) == cudaSuccess;
   BI_LM_CONFIGS(BI_SET_ATTR)
 #undef BI_SET_ATTR
 #define BI_SET_DW_ATTR(HS_)                                                                                     \
@@ -401,7 +401,7 @@ template <int kMode, int kNZ, int kHS>
 bi_status launch_lm(const CUtensorMap& tm_stat, const CUtensorMap& tm_zb, const CUtensorMap& tm_sl,
                     const CUtensorMap& tm_dz, const bi::LmArgs& a, int64_t units_upper, const DevInfo* di,
                     cudaStream_t s) {
-  const int smem = bi::LmTile<kNZ, kHS>::smem;
+  const int smem = bi::LmTile<kMode, kNZ, kHS>::smem;
   const int maxc = di->max_clusters[kMode][a.C];
   if (maxc <= 0) return BI_ERR_CUDA;
   int64_t ncl = units_upper < maxc ? units_upper : maxc;

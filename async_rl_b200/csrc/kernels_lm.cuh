@@ -130,25 +130,33 @@ struct LmShared {
   uint32_t rflag[kMaxSlots];       // rescale needed at the step of this slot (written by its producer)
   uint32_t wvote[4];               // per-warp rescale votes of this CTA's epilogue
   uint32_t rs_slot;                // slot of the pending rescale request (or kRsNone / kRsStop)
-  float mref[128];                 // reference sent by the previous producer
-  float col_lse2[kMaxNZ];          // kModeDW: per-column lse * log2(e)
-  float col_g[kMaxNZ];             // kModeDW: per-column g
-  int32_t col_y[kMaxNZ];           // kModeDW: per-column target (INT32_MIN: column not valid)
   uint32_t tmem_base;
   volatile uint32_t abort_flag;
 };
 
-constexpr int kLmSharedBytes = static_cast<int>((sizeof(LmShared) + 127) / 128 * 128);
+// Arrays of one mode only, right after LmShared: the forward modes' reference received from the
+// previous producer ([128] fp32), kModeDW's per-column parameters of the streamed rows of a step
+// (lse * log2(e), g, target: [NZ] each).  Sized per mode so that the ring keeps every byte the
+// other mode's arrays would take (at Hs = 320 that is the difference between 3 and 4 stages).
+template <int kMode, int kNZ>
+struct LmAux {
+  static constexpr int bytes = (kMode == kModeDW) ? kNZ * 12 : 128 * 4;
+};
+
 constexpr int kLmSmemLimit = 232448;  // per-block opt-in shared memory on sm_100
 
 // Stage geometry of one compiled tiling: a stage holds one A unit (128 x 64) and the larger of
-// the logit-phase B tile (NZ x 64) and the slice tile (64 x Hs).
-template <int kNZ, int kHS>
+// the logit-phase B tile (NZ x 64) and the slice tile (64 x Hs); LmShared and the mode's arrays
+// follow the ring.
+template <int kMode, int kNZ, int kHS>
 struct LmTile {
   static constexpr int stage_bytes = ((kAUnitBytes + (kNZ > kHS ? kNZ : kHS) * 128) + 1023) / 1024 * 1024;
-  static constexpr int fit = (kLmSmemLimit - kLmSharedBytes) / stage_bytes;
+  static constexpr int shared_bytes =
+      static_cast<int>(((sizeof(LmShared) + 15) / 16 * 16 + static_cast<size_t>(LmAux<kMode, kNZ>::bytes) + 127) / 128 *
+                       128);
+  static constexpr int fit = (kLmSmemLimit - shared_bytes) / stage_bytes;
   static constexpr int nstages = fit < kMaxStages ? fit : kMaxStages;
-  static constexpr int smem = nstages * stage_bytes + kLmSharedBytes;
+  static constexpr int smem = nstages * stage_bytes + shared_bytes;
   static_assert(nstages >= 2, "pipeline needs at least two stages");
   static_assert(kHS % 64 == 0 && kNZ % 64 == 0 && kHS + kNZ <= 512 && kNZ <= 256, "tile does not fit tensor memory");
 };
@@ -184,6 +192,10 @@ struct StreamPos {
 
 // Everything one CTA of the cluster needs to know about its place in the work.
 struct LmCtx {
+  float* mref;                     // forward modes: [128] reference sent by the previous producer
+  float* col_lse2;                 // kModeDW: [NZ] per-column lse * log2(e)
+  float* col_g;                    // kModeDW: [NZ] per-column g
+  int32_t* col_y;                  // kModeDW: [NZ] per-column target (INT32_MIN: column not valid)
   uint32_t C, rank, cl, ncl, nslot;
   int64_t rows, total;
   int steps, nunits, KB, slice0;
@@ -236,8 +248,8 @@ __device__ __forceinline__ void lm_tma_role(LmShared& sh, const LmArgs& a, const
     tma_prefetch_desc(m.sl);
     tma_prefetch_desc(m.dz);
   }
-  constexpr uint32_t nst = static_cast<uint32_t>(LmTile<kNZ, kHS>::nstages);
-  constexpr uint32_t sbytes = static_cast<uint32_t>(LmTile<kNZ, kHS>::stage_bytes);
+  constexpr uint32_t nst = static_cast<uint32_t>(LmTile<kMode, kNZ, kHS>::nstages);
+  constexpr uint32_t sbytes = static_cast<uint32_t>(LmTile<kMode, kNZ, kHS>::stage_bytes);
   constexpr uint32_t zbytes = kAUnitBytes + kNZ * 128;
   constexpr uint32_t obytes = kAUnitBytes + kHS * 128;
   constexpr int nkc = kNZ / 64;
@@ -319,14 +331,14 @@ __device__ __forceinline__ bool rs_handshake(LmShared& sh, const LmArgs& a, uint
 template <int kMode, int kNZ, int kHS>
 __device__ __forceinline__ void lm_mma_role(LmShared& sh, const LmArgs& a, const LmCtx& x, uint32_t tmem) {
   using ZB = ZBuf<kMode, kNZ>;
-  constexpr uint32_t nst = static_cast<uint32_t>(LmTile<kNZ, kHS>::nstages);
+  constexpr uint32_t nst = static_cast<uint32_t>(LmTile<kMode, kNZ, kHS>::nstages);
   constexpr uint32_t idesc_z = idesc_bf16(128, kNZ, false, false);
   constexpr int n1 = kHS < 256 ? kHS : 256;  // slice update: one MMA of n1 columns, one of n2
   constexpr int n2 = kHS - n1;
   constexpr uint32_t idesc_o1 = idesc_bf16(128, n1, false, true);
   constexpr uint32_t idesc_o2 = idesc_bf16(128, n2 > 0 ? n2 : 64, false, true);
   constexpr int nkc = kNZ / 64;
-  constexpr uint64_t sb_desc = static_cast<uint64_t>(LmTile<kNZ, kHS>::stage_bytes >> 4);
+  constexpr uint64_t sb_desc = static_cast<uint64_t>(LmTile<kMode, kNZ, kHS>::stage_bytes >> 4);
   const uint64_t dk0 = sdesc_k_sw128(x.ring_base);                                // A operands
   const uint64_t dkb0 = sdesc_k_sw128(x.ring_base + kAUnitBytes);                 // logit-phase B
   const uint64_t dmb0 = sdesc_mn_sw128(x.ring_base + kAUnitBytes, kSlUnitBytes);  // slice B
@@ -553,13 +565,13 @@ __device__ __forceinline__ void lm_fwd_epilogue_role(LmShared& sh, const LmArgs&
       if (p.j > 0) {
         if (!ep_wait<true>(sh, a, x.C, &sh.mref_full, mrc & 1u)) break;
         ++mrc;
-        mprev = sh.mref[row];
+        mprev = x.mref[row];
         if (et == 0) mbar_arrive_expect_tx(&sh.mref_full, 128 * 4);  // arm the next delivery
       }
       const float mnew = (M > mprev + kTau) ? M : mprev;
       if (p.j < x.steps - 1) {
         const uint32_t nxt = (p.modc + 1u == x.C) ? 0u : p.modc + 1u;
-        st_async_u32(mapa_shared(smem_u32(&sh.mref[row]), nxt), __float_as_uint(mnew),
+        st_async_u32(mapa_shared(smem_u32(&x.mref[row]), nxt), __float_as_uint(mnew),
                      mapa_shared(smem_u32(&sh.mref_full), nxt));
       }
       // this CTA's partial sum follows its own latest reference
@@ -806,9 +818,9 @@ __device__ __forceinline__ void lm_dw_epilogue_role(LmShared& sh, const LmArgs& 
       for (int cc = et; cc < kNZ; cc += 128) {
         const int64_t tt = static_cast<int64_t>(p.j) * kNZ + cc;
         const bool tv = tt < x.rows;
-        sh.col_lse2[cc] = tv ? a.lse_c[tt] * kLog2e : 0.f;
-        sh.col_g[cc] = tv ? a.g_c[tt] : 0.f;
-        sh.col_y[cc] = tv ? a.y[tt] : INT32_MIN;
+        x.col_lse2[cc] = tv ? a.lse_c[tt] * kLog2e : 0.f;
+        x.col_g[cc] = tv ? a.g_c[tt] : 0.f;
+        x.col_y[cc] = tv ? a.y[tt] : INT32_MIN;
       }
       mbar_arrive(&sh.ep_bar);
       if (!ep_wait<false>(sh, a, x.C, &sh.ep_bar, (epc++) & 1u)) break;
@@ -829,10 +841,10 @@ __device__ __forceinline__ void lm_dw_epilogue_role(LmShared& sh, const LmArgs& 
 #pragma unroll
         for (int q = 0; q < 32; ++q) {
           const int tc = c * 32 + q;
-          const float pr = ex2_approx(fmaf(__uint_as_float(v[q]), kLog2e, -sh.col_lse2[tc]));
-          const int32_t yc = sh.col_y[tc];
+          const float pr = ex2_approx(fmaf(__uint_as_float(v[q]), kLog2e, -x.col_lse2[tc]));
+          const int32_t yc = x.col_y[tc];
           const float oh = (static_cast<int64_t>(yc) == vrow) ? 1.f : 0.f;
-          d[q] = (v_ok && yc != INT32_MIN) ? sh.col_g[tc] * (oh - pr) : 0.f;
+          d[q] = (v_ok && yc != INT32_MIN) ? x.col_g[tc] * (oh - pr) : 0.f;
         }
         store_bf16x32_sectors(dzrow + c * 32, d);
       }
@@ -853,11 +865,17 @@ __global__ void __launch_bounds__(LmThreads<kMode>::value, 1)
     k_lm_cluster(const __grid_constant__ CUtensorMap tm_stat, const __grid_constant__ CUtensorMap tm_zb,
                  const __grid_constant__ CUtensorMap tm_sl, const __grid_constant__ CUtensorMap tm_dz, LmArgs a) {
   extern __shared__ __align__(1024) uint8_t dsmem[];
-  LmShared& sh = *reinterpret_cast<LmShared*>(dsmem + LmTile<kNZ, kHS>::nstages * LmTile<kNZ, kHS>::stage_bytes);
+  using Tile = LmTile<kMode, kNZ, kHS>;
+  LmShared& sh = *reinterpret_cast<LmShared*>(dsmem + Tile::nstages * Tile::stage_bytes);
+  uint8_t* aux = dsmem + Tile::nstages * Tile::stage_bytes + (sizeof(LmShared) + 15) / 16 * 16;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   LmCtx x;
+  x.mref = reinterpret_cast<float*>(aux);                  // forward modes
+  x.col_lse2 = reinterpret_cast<float*>(aux);              // kModeDW (the two never coexist)
+  x.col_g = x.col_lse2 + kNZ;
+  x.col_y = reinterpret_cast<int32_t*>(x.col_g + kNZ);
   x.C = static_cast<uint32_t>(a.C);
   x.rank = cluster_ctarank();
   x.cl = cluster_id_x();
