@@ -494,9 +494,11 @@ int logprob_decode(const uint16_t* hidden, const uint16_t* w_lm, const int32_t* 
   // hidden rows kept resident in 1 KB atoms of 8 rows when few (the ring then carries W only)
   int ag = T <= 8 ? 1 : (T <= 16 ? 2 : (T <= 32 ? 4 : 0));
   if (ag > 0 && bi::d1_a_bytes(ag, H / 64) + 4 * bi::d1_stage_bytes(ag, sub) + 4096 > bi::kD1Smem) ag = 0;
+  // streamed hidden rows: a box of T rows rounded up to 8 (whole 1 KB atoms of the swizzle), so
+  // that no stage carries rows past T
+  const int a_rows = ag > 0 ? 8 * ag : static_cast<int>(std::min<int64_t>(128, (T + 7) / 8 * 8));
   CUtensorMap tm_h, tm_w64;
-  if (!make_map(&tm_h, hidden, T, H, ag > 0 ? 8 * ag : 128) || !make_map(&tm_w64, w_lm, V, H, sub))
-    return BI_ERR_CUDA;
+  if (!make_map(&tm_h, hidden, T, H, a_rows) || !make_map(&tm_w64, w_lm, V, H, sub)) return BI_ERR_CUDA;
   const int nsub = nvz * (pl.NZ / sub);
   if (static_cast<size_t>(nsub) > decode_subtiles_max(H, V)) return kDecodeUnsupported;  // not held by L.zsmax
   const int G = nsub < di->sms ? nsub : di->sms;  // >= NZ / sub sub-tiles: every wait has a finite target
@@ -506,6 +508,7 @@ int logprob_decode(const uint16_t* hidden, const uint16_t* w_lm, const int32_t* 
   d.nvz = nvz;
   d.KB = H / 64;
   d.nsub = nsub;
+  d.a_rows = a_rows;
   d.rounds = (nsub + G - 1) / G;
   d.smax = reinterpret_cast<uint64_t*>(ws + L.zsmax);
   d.mref = reinterpret_cast<float*>(ws + L.zmref);

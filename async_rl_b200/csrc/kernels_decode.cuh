@@ -57,11 +57,18 @@ __device__ __forceinline__ uint64_t ld_relaxed_gpu_u64(const uint64_t* p) {
 constexpr uint64_t kD1Tag = uint64_t{1} << 32;
 __device__ __forceinline__ float d1_value(uint64_t w) { return __uint_as_float(static_cast<uint32_t>(w)); }
 
-// The value of entry i of a row, waiting (bounded) until its writer has stored it.  Returns false
+// Where row `row`'s maximum of sub-tile `sub` lives: row-major for up to 8 rows (a warp walks one
+// row, its lanes over consecutive sub-tiles), sub-tile-major beyond (each row's owner thread walks
+// the sub-tiles, and a warp's 32 rows of one sub-tile are one 256-byte line).
+__device__ __forceinline__ int64_t d1_slot(int64_t T, int nsub, int row, int sub) {
+  return T <= 8 ? static_cast<int64_t>(row) * nsub + sub : static_cast<int64_t>(sub) * T + row;
+}
+
+// The value of the entry at p, waiting (bounded) until its writer has stored it.  Returns false
 // on a timeout or an abort.
-__device__ __forceinline__ bool d1_entry(const uint64_t* rr, int i, float& v, volatile uint32_t* abort_flag,
+__device__ __forceinline__ bool d1_entry(const uint64_t* p, float& v, volatile uint32_t* abort_flag,
                                          int32_t* status, uint64_t limit_ns) {
-  uint64_t w = ld_relaxed_gpu_u64(rr + i);
+  uint64_t w = ld_relaxed_gpu_u64(p);
   if (w & kD1Tag) {
     v = d1_value(w);
     return true;
@@ -69,7 +76,7 @@ __device__ __forceinline__ bool d1_entry(const uint64_t* rr, int i, float& v, vo
   const uint64_t t0 = globaltimer_ns();
   uint32_t spins = 0;
   while (true) {
-    w = ld_relaxed_gpu_u64(rr + i);
+    w = ld_relaxed_gpu_u64(p);
     if (w & kD1Tag) {
       v = d1_value(w);
       return true;
@@ -119,8 +126,10 @@ struct D1Args {
   int64_t T;          // real rows (<= 128)
   int32_t V, nvz, KB;
   int32_t nsub;       // sub-tiles: nvz * NZ / sub-tile width
+  int32_t a_rows;     // rows of the streamed hidden-row box (kAG = 0): T rounded up to 8, <= 128
   int32_t rounds;     // ceil(nsub / gridDim.x)
-  uint64_t* smax;     // [T][nsub] row maxima of each sub-tile over its valid columns, tagged (zero at launch)
+  uint64_t* smax;     // [T][nsub] (T <= 8) or [nsub][T] row maxima of each sub-tile over its valid
+                      // columns, tagged (zero at launch): d1_slot
   float* mref;        // [nvz][T] reference of each row at each step
   float* csum;        // [T][nvz][NZ / 32] chunk sums
   float* zy;          // [T] target logits
@@ -146,6 +155,10 @@ __global__ void __launch_bounds__(kZtThreads, 1)
   const int a_bytes = d1_a_bytes(kAG, a.KB);
   const int nst_i = (kD1Smem - kShBytes - a_bytes) / kStageBytes;
   const uint32_t nst = static_cast<uint32_t>(nst_i < kD1MaxStages ? nst_i : kD1MaxStages);
+  // bytes a stage receives: W rows, and the real hidden rows (rounded up to 8) when they are
+  // streamed; the MMA's rows past them read whatever the stage held and give logits of rows past
+  // T, which nothing reads
+  const uint32_t stage_tx = static_cast<uint32_t>((kAG == 0 ? a.a_rows * 128 : 0) + kD1Sub * 128);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int G = static_cast<int>(gridDim.x);
@@ -200,7 +213,7 @@ __global__ void __launch_bounds__(kZtThreads, 1)
 #pragma unroll 1
         for (int kb = 0; kb < a.KB; ++kb) {
           if (!mbar_wait<false>(&sh.empty[stage], phase ^ 1u, wc)) { ok = false; break; }
-          mbar_arrive_expect_tx(&sh.full[stage], static_cast<uint32_t>(kStageBytes));
+          mbar_arrive_expect_tx(&sh.full[stage], stage_tx);
           const uint32_t dst = ring + stage * kStageBytes;
           if (kAG == 0) {
             tma_load_2d(dst, &tm_h, &sh.full[stage], kb * 64, 0);
@@ -291,7 +304,7 @@ __global__ void __launch_bounds__(kZtThreads, 1)
               for (int q = 0; q < 32; ++q)
                 if (vb + q < a.V) M = fmaxf(M, __uint_as_float(v[q]));
             }
-            if (real) st_relaxed_gpu_u64(a.smax + static_cast<int64_t>(row) * a.nsub + sub, kD1Tag | __float_as_uint(M));
+            if (real) st_relaxed_gpu_u64(a.smax + d1_slot(a.T, a.nsub, row, sub), kD1Tag | __float_as_uint(M));
           }
         }
       }
@@ -319,7 +332,7 @@ __global__ void __launch_bounds__(kZtThreads, 1)
             float mx = -INFINITY;
             for (int i = lo + lane; i < hi; i += 32) {
               float v;
-              good = good && d1_entry(rr, i, v, &sh.abort_flag, a.status, a.limit_ns);
+              good = good && d1_entry(rr + i, v, &sh.abort_flag, a.status, a.limit_ns);
               mx = fmaxf(mx, v);
             }
             if (!__all_sync(0xffffffffu, good)) { good = false; break; }
@@ -342,13 +355,14 @@ __global__ void __launch_bounds__(kZtThreads, 1)
             if (lane == 0) sh.mcs[r] = m;
           }
         } else if (real) {
-          const uint64_t* rr = a.smax + static_cast<int64_t>(row) * a.nsub;
+          const uint64_t* rr = a.smax + row;  // entry of sub-tile i at rr + i T
+          const int64_t Tr = a.T;
           float m = sh.mcs[row];
           float mx = -INFINITY;
           uint64_t tags = kD1Tag;
 #pragma unroll 16
           for (int i = lo; i < hi; ++i) {
-            const uint64_t w = ld_relaxed_gpu_u64(rr + i);
+            const uint64_t w = ld_relaxed_gpu_u64(rr + i * Tr);
             tags &= w;
             mx = fmaxf(mx, d1_value(w));
           }
@@ -357,7 +371,7 @@ __global__ void __launch_bounds__(kZtThreads, 1)
             mx = -INFINITY;
             for (int i = lo; i < hi && good; ++i) {
               float v;
-              good = d1_entry(rr, i, v, &sh.abort_flag, a.status, a.limit_ns);
+              good = d1_entry(rr + i * Tr, v, &sh.abort_flag, a.status, a.limit_ns);
               mx = fmaxf(mx, v);
             }
           }
@@ -365,7 +379,8 @@ __global__ void __launch_bounds__(kZtThreads, 1)
             for (int t = jc; t <= j; ++t) {
               float M = -INFINITY;
 #pragma unroll
-              for (int i = 0; i < kSubPerTile; ++i) M = fmaxf(M, d1_value(ld_relaxed_gpu_u64(rr + t * kSubPerTile + i)));
+              for (int i = 0; i < kSubPerTile; ++i)
+                M = fmaxf(M, d1_value(ld_relaxed_gpu_u64(rr + (t * kSubPerTile + i) * Tr)));
               m = (M > m + kTau) ? M : m;
             }
           }
