@@ -442,11 +442,14 @@ bi_status logprob_forward(const uint16_t* hidden, const uint16_t* w_lm, const in
                           uint64_t force_timeout_ns, const DevInfo* di, cudaStream_t s) {
   const LmPlan pl = plan_lm(H, di);
   if (pl.C == 0) return BI_ERR_UNSUPPORTED_SHAPE;
+  // fewer than 128 rows: one unit, whose hidden-row box holds the real rows only (rounded up to 8)
+  const int a_rows = T < 128 ? static_cast<int>((T + 7) / 8 * 8) : 128;
   CUtensorMap tm_h, tm_wz, tm_w64;
-  if (!make_map(&tm_h, hidden, T, H, 128) || !make_map(&tm_wz, w_lm, V, H, pl.NZ) ||
+  if (!make_map(&tm_h, hidden, T, H, a_rows) || !make_map(&tm_wz, w_lm, V, H, pl.NZ) ||
       !make_map(&tm_w64, w_lm, V, H, 64))
     return BI_ERR_CUDA;
   bi::LmArgs a{};
+  a.a_rows = a_rows;
   a.H = H;
   a.V = V;
   a.C = pl.C;

@@ -73,6 +73,10 @@ struct LmArgs {
   int32_t Hs;              // H / C
   int32_t NZ;              // streamed rows per step
   int64_t T;               // rows of the hidden-state tensor maps (upper bound)
+  int32_t a_rows;          // rows of the stationary operand's logit-phase box: 0 for 128; fewer (a
+                           // multiple of 8) only when one unit holds every row, which the rows
+                           // past it then never see: the MMA's rows beyond read stale shared memory
+                           // and give logits of rows past T, which nothing reads
   const int64_t* d_rows;   // number of valid rows on the device (nullptr: T)
   int32_t nvz;             // ceil(V / NZ)
   int32_t nv128;           // ceil(V / 128)
@@ -250,7 +254,7 @@ __device__ __forceinline__ void lm_tma_role(LmShared& sh, const LmArgs& a, const
   }
   constexpr uint32_t nst = static_cast<uint32_t>(LmTile<kMode, kNZ, kHS>::nstages);
   constexpr uint32_t sbytes = static_cast<uint32_t>(LmTile<kMode, kNZ, kHS>::stage_bytes);
-  constexpr uint32_t zbytes = kAUnitBytes + kNZ * 128;
+  const uint32_t zbytes = static_cast<uint32_t>((a.a_rows > 0 ? a.a_rows : 128) * 128 + kNZ * 128);
   constexpr uint32_t obytes = kAUnitBytes + kHS * 128;
   constexpr int nkc = kNZ / 64;
   uint32_t stage = 0, phase = 0;
