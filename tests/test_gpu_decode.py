@@ -37,9 +37,11 @@ def test_few_rows_bitwise_equal_to_packed_batch(H, V, cuda_device):
     h, w, y = random_inputs(300, H, V, seed=H + V)
     h, w, y = h.to(cuda_device), w.to(cuda_device), y.to(cuda_device)
     packed_lp, packed_lse = _lp(h, w, y, cuda_device)          # 300 rows: the cluster kernel
-    # 1, 3, 12 and 20 rows keep their hidden rows resident (one, two or four 8-row atoms); 128 rows
-    # stream them with every stage
-    for rows in ([0], [5, 17, 299], list(range(128)), list(range(172, 300)), list(range(40, 52)), list(range(7, 27))):
+    # 1, 3, 9, 12 and 20 rows keep their hidden rows resident (one, two or four 8-row atoms); 33,
+    # 40, 100 and 128 rows stream them with every stage, in a box of the rows rounded up to 8.
+    # Past 8 rows the sub-tile maxima are stored sub-tile-major.
+    for rows in ([0], [5, 17, 299], list(range(128)), list(range(172, 300)), list(range(40, 52)), list(range(7, 27)),
+                 list(range(60, 69)), list(range(200, 233)), list(range(3, 43)), list(range(150, 250))):
         r = torch.tensor(rows, device=cuda_device)
         lp, lse = _lp(h[r].contiguous(), w, y[r].contiguous(), cuda_device)   # <= 128 rows: every SM
         assert torch.equal(lp, packed_lp[r]), f"logprob bits differ (H={H}, V={V}, {len(rows)} rows)"
@@ -66,14 +68,16 @@ def test_few_rows_with_moving_reference_bitwise_equal_to_packed_batch(cuda_devic
         assert torch.equal(lp, packed_lp[r]) and torch.equal(lse, packed_lse[r])
 
 
-def test_few_rows_with_minimum_workspace_take_the_cluster_kernel(cuda_device):
+@pytest.mark.parametrize("T", [5, 100])
+def test_few_rows_with_minimum_workspace_take_the_cluster_kernel(T, cuda_device):
     """A workspace without room for the all-SM path's partial sums is accepted (the cluster
-    kernel scores the rows); the bits are the same."""
-    h, w, y = random_inputs(5, 1536, 8192, seed=3)
+    kernel scores the rows, loading a hidden-row box of the rows rounded up to 8); the bits are
+    the same."""
+    h, w, y = random_inputs(T, 1536, 8192, seed=3)
     h, w, y = h.to(cuda_device), w.to(cuda_device), y.to(cuda_device)
     fast, _ = _lp(h, w, y, cuda_device)
-    small = torch.empty(bi.workspace_bytes(5, 1536, 8192, 0, minimal=True), dtype=torch.uint8, device=cuda_device)
-    assert small.numel() < bi.workspace_bytes(5, 1536, 8192, 0)
+    small = torch.empty(bi.workspace_bytes(T, 1536, 8192, 0, minimal=True), dtype=torch.uint8, device=cuda_device)
+    assert small.numel() < bi.workspace_bytes(T, 1536, 8192, 0)
     lp, _, st = bi.logprob_fwd(h, w, y, ws=small)
     torch.cuda.synchronize()
     bi.check_status(st)
