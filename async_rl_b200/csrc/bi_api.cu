@@ -494,9 +494,16 @@ int logprob_decode(const uint16_t* hidden, const uint16_t* w_lm, const int32_t* 
   const int nvz = (V + pl.NZ - 1) / pl.NZ;
   const size_t zsm = bi::zscan_smem(nvz, pl.NZ);
   if (zsm > kZscanSmemMax) return kDecodeUnsupported;
-  // hidden rows kept resident in 1 KB atoms of 8 rows when few (the ring then carries W only)
+  // hidden rows kept resident in 1 KB atoms of 8 rows when few (the ring then carries W only).
+  // The pass then also leaves room for the combine's block where four ring stages still fit, so
+  // that the block is resident (waiting on the pass) before the pass ends: 228 KB of shared
+  // memory per SM, 1 KB of it reserved per resident block.
+  constexpr size_t kSmPerSm = 233472, kPerBlock = 1024;
+  const int smem_lean = static_cast<int>((kSmPerSm - kPerBlock - (zsm + 64 + kPerBlock)) / 1024 * 1024);
+  auto fits = [&](int g, int smem) { return bi::d1_a_bytes(g, H / 64) + 4 * bi::d1_stage_bytes(g, sub) + 4096 <= smem; };
   int ag = T <= 8 ? 1 : (T <= 16 ? 2 : (T <= 32 ? 4 : 0));
-  if (ag > 0 && bi::d1_a_bytes(ag, H / 64) + 4 * bi::d1_stage_bytes(ag, sub) + 4096 > bi::kD1Smem) ag = 0;
+  if (ag > 0 && !fits(ag, bi::kD1Smem)) ag = 0;
+  const int d1_smem = (ag > 0 && smem_lean < bi::kD1Smem && fits(ag, smem_lean)) ? smem_lean : bi::kD1Smem;
   // streamed hidden rows: a box of T rows rounded up to 8 (whole 1 KB atoms of the swizzle), so
   // that no stage carries rows past T
   const int a_rows = ag > 0 ? 8 * ag : static_cast<int>(std::min<int64_t>(128, (T + 7) / 8 * 8));
@@ -512,6 +519,7 @@ int logprob_decode(const uint16_t* hidden, const uint16_t* w_lm, const int32_t* 
   d.KB = H / 64;
   d.nsub = nsub;
   d.a_rows = a_rows;
+  d.smem = d1_smem;
   d.rounds = (nsub + G - 1) / G;
   d.smax = reinterpret_cast<uint64_t*>(ws + L.zsmax);
   d.mref = reinterpret_cast<float*>(ws + L.zmref);
@@ -531,7 +539,7 @@ int logprob_decode(const uint16_t* hidden, const uint16_t* w_lm, const int32_t* 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(G), 1, 1);
   cfg.blockDim = dim3(bi::kZtThreads, 1, 1);
-  cfg.dynamicSmemBytes = static_cast<size_t>(bi::kD1Smem);
+  cfg.dynamicSmemBytes = static_cast<size_t>(d.smem);
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeCooperative;

@@ -127,6 +127,7 @@ struct D1Args {
   int32_t V, nvz, KB;
   int32_t nsub;       // sub-tiles: nvz * NZ / sub-tile width
   int32_t a_rows;     // rows of the streamed hidden-row box (kAG = 0): T rounded up to 8, <= 128
+  int32_t smem;       // dynamic shared memory of the launch (<= kD1Smem)
   int32_t rounds;     // ceil(nsub / gridDim.x)
   uint64_t* smax;     // [T][nsub] (T <= 8) or [nsub][T] row maxima of each sub-tile over its valid
                       // columns, tagged (zero at launch): d1_slot
@@ -151,9 +152,9 @@ __global__ void __launch_bounds__(kZtThreads, 1)
   constexpr int kStageBytes = d1_stage_bytes(kAG, kD1Sub);
   extern __shared__ __align__(1024) uint8_t dsmem[];
   constexpr int kShBytes = static_cast<int>((sizeof(D1Shared) + 1023) / 1024 * 1024);
-  D1Shared& sh = *reinterpret_cast<D1Shared*>(dsmem + kD1Smem - kShBytes);
+  D1Shared& sh = *reinterpret_cast<D1Shared*>(dsmem + a.smem - kShBytes);
   const int a_bytes = d1_a_bytes(kAG, a.KB);
-  const int nst_i = (kD1Smem - kShBytes - a_bytes) / kStageBytes;
+  const int nst_i = (a.smem - kShBytes - a_bytes) / kStageBytes;
   const uint32_t nst = static_cast<uint32_t>(nst_i < kD1MaxStages ? nst_i : kD1MaxStages);
   // bytes a stage receives: W rows, and the real hidden rows (rounded up to 8) when they are
   // streamed; the MMA's rows past them read whatever the stage held and give logits of rows past
