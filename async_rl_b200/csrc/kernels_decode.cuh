@@ -57,11 +57,13 @@ __device__ __forceinline__ uint64_t ld_relaxed_gpu_u64(const uint64_t* p) {
 constexpr uint64_t kD1Tag = uint64_t{1} << 32;
 __device__ __forceinline__ float d1_value(uint64_t w) { return __uint_as_float(static_cast<uint32_t>(w)); }
 
-// Where row `row`'s maximum of sub-tile `sub` lives: row-major for up to 8 rows (a warp walks one
-// row, its lanes over consecutive sub-tiles), sub-tile-major beyond (each row's owner thread walks
-// the sub-tiles, and a warp's 32 rows of one sub-tile are one 256-byte line).
+// Where row `row`'s maximum of sub-tile `sub` lives: row-major for up to 32 rows (a warp walks up
+// to 8 rows, its lanes over consecutive sub-tiles), sub-tile-major beyond (each row's owner
+// thread walks the sub-tiles, and a warp's 32 rows of one sub-tile are one 256-byte line).
+constexpr int kD1WarpRows = 32;    // up to this many rows: row-major maxima, 8 rows per epilogue warp
+constexpr int kD1LaneEntries = 6;  // entries per lane per row loaded at once (a round's range is ~G)
 __device__ __forceinline__ int64_t d1_slot(int64_t T, int nsub, int row, int sub) {
-  return T <= 8 ? static_cast<int64_t>(row) * nsub + sub : static_cast<int64_t>(sub) * T + row;
+  return T <= kD1WarpRows ? static_cast<int64_t>(row) * nsub + sub : static_cast<int64_t>(sub) * T + row;
 }
 
 // The value of the entry at p, waiting (bounded) until its writer has stored it.  Returns false
@@ -129,7 +131,7 @@ struct D1Args {
   int32_t a_rows;     // rows of the streamed hidden-row box (kAG = 0): T rounded up to 8, <= 128
   int32_t smem;       // dynamic shared memory of the launch (<= kD1Smem)
   int32_t rounds;     // ceil(nsub / gridDim.x)
-  uint64_t* smax;     // [T][nsub] (T <= 8) or [nsub][T] row maxima of each sub-tile over its valid
+  uint64_t* smax;     // [T][nsub] (T <= 32) or [nsub][T] row maxima of each sub-tile over its valid
                       // columns, tagged (zero at launch): d1_slot
   float* mref;        // [nvz][T] reference of each row at each step
   float* csum;        // [T][nvz][NZ / 32] chunk sums
@@ -318,42 +320,92 @@ __global__ void __launch_bounds__(kZtThreads, 1)
       if (jc <= j) {
         // advance every row's chain over tiles jc .. j, as the cluster kernel's producers pass the
         // reference on.  The range's largest sub-tile maximum is checked first: only when it could
-        // raise the reference are the tiles walked in order.  Few rows: a warp per row (coalesced
-        // loads, the ordered walk 32 tiles at a time over the lanes by shuffles).  Many rows: each
-        // row's owner thread alone, its loads independent of one another.
+        // raise the reference are the tiles walked in order.  Up to 32 rows: a warp per group of
+        // rows (coalesced loads, the ordered walk 32 tiles at a time over the lanes by shuffles).
+        // More rows: each row's owner thread alone, its loads independent of one another.
         // (each entry is waited for until its writer has stored it: by the schedule it nearly
         // always has, the entries a round needs being at least two rounds old)
         const int lo = jc * kSubPerTile, hi = (j + 1) * kSubPerTile;
         bool good = true;
-        if (a.T <= 8) {
+        if (a.T <= kD1WarpRows) {
+          // up to 8 rows per warp (rows ew, ew + 4, ...): every lane loads all its entries of all
+          // its rows before anything waits (one round trip), and only a lane that found one of
+          // them not yet written loads its entries again, waiting for each
           const int ew = warp - 2;  // 0..3
-          for (int r = ew; r < static_cast<int>(a.T); r += 4) {
-            const uint64_t* rr = a.smax + static_cast<int64_t>(r) * a.nsub;
-            float m = sh.mcs[r];
-            float mx = -INFINITY;
-            for (int i = lo + lane; i < hi; i += 32) {
-              float v;
-              good = good && d1_entry(rr + i, v, &sh.abort_flag, a.status, a.limit_ns);
-              mx = fmaxf(mx, v);
-            }
-            if (!__all_sync(0xffffffffu, good)) { good = false; break; }
+          float mxr[8];
+          uint64_t tags = kD1Tag;
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-            if (mx > m + kTau) {
-              for (int base = jc; base <= j; base += 32) {
-                float Ml = -INFINITY;
-                if (base + lane <= j) {
+          for (int q = 0; q < 8; ++q) {
+            mxr[q] = -INFINITY;
+            const int r = ew + 4 * q;
+            if (r < static_cast<int>(a.T)) {
+              const uint64_t* rr = a.smax + static_cast<int64_t>(r) * a.nsub;
 #pragma unroll
-                  for (int i = 0; i < kSubPerTile; ++i) Ml = fmaxf(Ml, d1_value(ld_relaxed_gpu_u64(rr + (base + lane) * kSubPerTile + i)));
+              for (int k = 0; k < kD1LaneEntries; ++k) {
+                const int i = lo + lane + 32 * k;
+                if (i < hi) {
+                  const uint64_t w = ld_relaxed_gpu_u64(rr + i);
+                  tags &= w;
+                  mxr[q] = fmaxf(mxr[q], d1_value(w));
                 }
-                const int nt = (j - base + 1) < 32 ? (j - base + 1) : 32;
-                for (int l = 0; l < nt; ++l) {
-                  const float M = __shfl_sync(0xffffffffu, Ml, l);
-                  m = (M > m + kTau) ? M : m;
+              }
+              for (int i = lo + lane + 32 * kD1LaneEntries; i < hi; i += 32) {  // a wider range than a round's
+                const uint64_t w = ld_relaxed_gpu_u64(rr + i);
+                tags &= w;
+                mxr[q] = fmaxf(mxr[q], d1_value(w));
+              }
+            }
+          }
+          if (!(tags & kD1Tag)) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              mxr[q] = -INFINITY;
+              const int r = ew + 4 * q;
+              if (r < static_cast<int>(a.T)) {
+                const uint64_t* rr = a.smax + static_cast<int64_t>(r) * a.nsub;
+                for (int i = lo + lane; i < hi && good; i += 32) {
+                  float v;
+                  good = d1_entry(rr + i, v, &sh.abort_flag, a.status, a.limit_ns);
+                  mxr[q] = fmaxf(mxr[q], v);
                 }
               }
             }
-            if (lane == 0) sh.mcs[r] = m;
+          }
+          if (!__all_sync(0xffffffffu, good)) {
+            good = false;
+          } else {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const int r = ew + 4 * q;
+              if (r >= static_cast<int>(a.T)) break;  // warp-uniform
+              const uint64_t* rr = a.smax + static_cast<int64_t>(r) * a.nsub;
+              float m = sh.mcs[r];
+              float mx = mxr[q];
+#pragma unroll
+              for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+              if (mx > m + kTau) {
+                for (int base = jc; base <= j; base += 32) {
+                  const bool has = base + lane <= j;
+                  float Ml = -INFINITY;
+                  if (has) {
+#pragma unroll
+                    for (int i = 0; i < kSubPerTile; ++i) Ml = fmaxf(Ml, d1_value(ld_relaxed_gpu_u64(rr + (base + lane) * kSubPerTile + i)));
+                  }
+                  // the tiles in order: the first whose maximum raises the reference sets it, and
+                  // the search goes on past it with the new reference (the same decisions as one
+                  // tile at a time, one ballot per raise)
+                  int from = 0;
+                  while (true) {
+                    const uint32_t up = __ballot_sync(0xffffffffu, has && lane >= from && Ml > m + kTau);
+                    if (up == 0u) break;
+                    const int l = __ffs(static_cast<int>(up)) - 1;
+                    m = __shfl_sync(0xffffffffu, Ml, l);
+                    from = l + 1;
+                  }
+                }
+              }
+              if (lane == 0) sh.mcs[r] = m;
+            }
           }
         } else if (real) {
           const uint64_t* rr = a.smax + row;  // entry of sub-tile i at rr + i T

@@ -62,7 +62,7 @@ def test_few_rows_with_moving_reference_bitwise_equal_to_packed_batch(cuda_devic
     w = (w.float() * ramp).to(torch.bfloat16)
     h, w, y = h.to(cuda_device), w.to(cuda_device), y.to(cuda_device)
     packed_lp, packed_lse = _lp(h, w, y, cuda_device)
-    for rows in ([3], list(range(100, 228))):
+    for rows in ([3], list(range(10, 30)), list(range(40, 72)), list(range(100, 228))):
         r = torch.tensor(rows, device=cuda_device)
         lp, lse = _lp(h[r].contiguous(), w, y[r].contiguous(), cuda_device)
         assert torch.equal(lp, packed_lp[r]) and torch.equal(lse, packed_lse[r])
