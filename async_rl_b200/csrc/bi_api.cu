@@ -497,9 +497,9 @@ int logprob_decode(const uint16_t* hidden, const uint16_t* w_lm, const int32_t* 
   // hidden rows kept resident in 1 KB atoms of 8 rows when few (the ring then carries W only).
   // The pass then also leaves room for the combine's block where four ring stages still fit, so
   // that the block is resident (waiting on the pass) before the pass ends: 228 KB of shared
-  // memory per SM, 1 KB of it reserved per resident block.
-  constexpr size_t kSmPerSm = 233472, kPerBlock = 1024;
-  const int smem_lean = static_cast<int>((kSmPerSm - kPerBlock - (zsm + 64 + kPerBlock)) / 1024 * 1024);
+  // memory per SM, 1 KB of it reserved per resident block, and up to 1 KB of the combine's own.
+  constexpr size_t kSmPerSm = 233472, kPerBlock = 1024, kZsStatic = 1024;
+  const int smem_lean = static_cast<int>((kSmPerSm - kPerBlock - (zsm + kZsStatic + kPerBlock)) / 1024 * 1024);
   auto fits = [&](int g, int smem) { return bi::d1_a_bytes(g, H / 64) + 4 * bi::d1_stage_bytes(g, sub) + 4096 <= smem; };
   int ag = T <= 8 ? 1 : (T <= 16 ? 2 : (T <= 32 ? 4 : 0));
   if (ag > 0 && !fits(ag, bi::kD1Smem)) ag = 0;

@@ -497,7 +497,7 @@ __global__ void k_d1_zero(uint64_t* __restrict__ smax, int64_t n, int32_t* __res
 }
 
 constexpr int kZsThreads = 256;
-constexpr int kZsBatch = 8;    // loads in flight per thread while staging
+constexpr int kZsBatch = 24;   // loads in flight per thread while staging (one batch at V = 151936)
 
 // Dynamic shared memory of k_lm_zscan: one row's chunk sums and references.
 __host__ __device__ constexpr size_t zscan_smem(int nvz, int nz) {
