@@ -230,6 +230,12 @@ def cpu_oracle_sample(b, logmu_host, nrows):
             "sample": f"first {nrows} rows of the {CONFIG} batch (fwd + loss + dH + dW in fp64 NumPy), {dt:.1f} s"}
 
 
+def loss_workload(spec, T):
+    """The loss step's workload name, the same in both arms' `config`."""
+    return (f"{CONFIG}: H={spec.H} V={spec.V}, {spec.groups}x{spec.per_group} responses "
+            f"U[{spec.len_lo},{spec.len_hi}] rows, T={T} scored rows per rank")
+
+
 def run_reference(args):
     """--impl reference: the fp64 CPU oracle on the machine's host cores, a bounded slice per step."""
     rank, world, _ = dist_env()
@@ -251,9 +257,11 @@ def run_reference(args):
     line = {"impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": f"{CONFIG}: H=1536 V=151936, {nrows}-row slice per step on host cores"},
+            "config": {"workload": loss_workload(b.spec, b.n_rows), "global_batch_tokens": int(b.n_rows),
+                       "parallelism": "dp1"},
             "cpu_baseline": {"value": val, "unit": UNIT, "cores": r["cores"], "kind": "oracle",
-                             "sample": f"first {nrows} rows of the {CONFIG} batch per step"},
+                             "sample": f"first {nrows} rows of that batch per step (fwd + loss + dH + dW in "
+                                       f"fp64 NumPy), throughput scaled to tokens/s"},
             "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -486,8 +494,7 @@ def run_ours(args):
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": f"{CONFIG}: H={H} V={V}, {spec.groups}x{spec.per_group} responses "
-                                   f"U[{spec.len_lo},{spec.len_hi}] rows, T={T} scored rows per rank",
+            "config": {"workload": loss_workload(spec, T),
                        "global_batch_tokens": int(total_tokens), "parallelism": f"dp{world}",
                        "path": "default: no T x V array in device memory (dW recomputes the logits)",
                        "workspace_gb": ws.numel() / 1e9,
@@ -523,6 +530,12 @@ DENSE_METRIC = "batch-invariant RMSNorm + bf16 GEMM (gate/up) TFLOP/s at M76239 
 DENSE_CPU_ROWS = 32768
 
 
+def dense_workload():
+    """The dense step's workload name, the same in both arms' `config`."""
+    return (f"dense: RMSNorm [{DENSE_M}, {DENSE_K}] then Y = X W^T, W [{DENSE_N}, {DENSE_K}] "
+            f"(1.5B shape gate/up)")
+
+
 def run_dense_reference(args):
     """--impl reference --workload dense: the fp64 oracle on the machine's host cores, a bounded slice
     of rows per step (rank 0 only)."""
@@ -545,10 +558,9 @@ def run_dense_reference(args):
                       "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
                       "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
                       "data": "synthetic",
-                      "config": {"workload": f"dense: RMSNorm + GEMM, {rows}-row slice of [{M}, {K}] x [{N}, {K}]^T "
-                                             "per step on host cores"},
+                      "config": {"workload": dense_workload()},
                       "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                                       "sample": f"{rows} rows per step"},
+                                       "sample": f"{rows} rows of [{M}, {K}] per step (fp64 RMSNorm + GEMM)"},
                       "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),
           flush=True)
 
@@ -663,7 +675,7 @@ def run_dense(args):
     line = {"metric": DENSE_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": f"dense: RMSNorm [{M}, {K}] then Y = X W^T, W [{N}, {K}] (1.5B shape gate/up)",
+            "config": {"workload": dense_workload(),
                        "parallelism": f"replicas{world}",
                        "l2": "inputs larger than L2 (x 0.23 GB, y 1.37 GB); no flush"},
             "roofline": {"bound": "tensor", "kernel": "k_gemm_pair", "achieved": g_tf, "peak": peak_tf,
@@ -691,6 +703,11 @@ def run_dense(args):
 DECODE_METRIC = "decode-style logprob scoring latency, one row per call, at H1536 V151936"
 
 
+def decode_workload(H, V):
+    """The decode line's workload name, the same in both arms' `config`."""
+    return f"decode: 1 row per bi_logprob_fwd call, H={H} V={V}"
+
+
 def run_decode_reference(args):
     """--impl reference --workload decode: the fp64 oracle scoring one row per step on the host cores."""
     rank, world, _ = dist_env()
@@ -715,7 +732,7 @@ def run_decode_reference(args):
                       "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
                       "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
                       "data": "synthetic",
-                      "config": {"workload": "decode: 1 row per call, H=1536 V=151936, fp64 oracle on host cores"},
+                      "config": {"workload": decode_workload(1536, 151936)},
                       "cpu_baseline": {"value": ms, "unit": "ms per call", "cores": int(cores), "kind": "oracle",
                                        "sample": "one row per step"},
                       "e2e": {"value": ms, "unit": "ms per call", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),
@@ -798,7 +815,7 @@ def run_decode(args):
     line = {"metric": DECODE_METRIC, "value": ms, "unit": "ms per call", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": False, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": f"decode: 1 row per bi_logprob_fwd call, H={H} V={V}, all-SM path",
+            "config": {"workload": decode_workload(H, V),
                        "parallelism": f"replicas{world}", "l2": "W 0.47 GB exceeds L2; no flush"},
             "rows_128_ms": ms_128, "cluster_kernel_ms": ms_cluster,
             "roofline": {"bound": "hbm", "kernel": wk, "achieved": w_bytes / (zt_ms * 1e-3) / 1e9,
