@@ -134,6 +134,25 @@ def test_loss_odd_shapes(cuda_device):
     _loss_case(b, cuda_device)
 
 
+@pytest.mark.parametrize("case", ["all_prompt", "no_rows"])
+def test_loss_without_scored_rows(case, cuda_device):
+    """No scored token at all (every row a prompt row, or no rows): the loss and both gradients are
+    exactly zero, D3 counts nothing, the status is clean ("Zero Mismatch, Simple Async RL", section
+    "Alignment permits a simpler learning path": a response contributes its token mean, an empty
+    one nothing)."""
+    lengths = [5, 7, 3, 9, 2, 4, 6, 8] if case == "all_prompt" else [0] * 8
+    spec = spec_for("tiny", groups=2, per_group=4, len_lo=0, len_hi=9, prompt_len=16 if case == "all_prompt" else 0)
+    b = make_batch(spec, lengths=lengths).to(cuda_device)
+    mu = torch.full((b.n_rows,), -6.0, dtype=torch.float32, device=cuda_device)
+    out = bi.is_loss_fwd_bwd(b.hidden, b.w, b.targets, mu, b.rewards, b.resp_offsets, b.group_offsets,
+                             b.prompt_lens, 0.0)
+    torch.cuda.synchronize()
+    bi.check_status(out.status)
+    assert float(out.loss.item()) == 0.0
+    assert not bool(out.grad_w.any()) and not bool(out.grad_hidden.any())
+    assert out.d3()["count"] == 0
+
+
 def test_loss_cluster_split_h2048(cuda_device):
     """H = 2048: eight CTAs share each tile (256 columns each)."""
     spec = spec_for("tiny", H=2048, V=3000, groups=2, per_group=2, len_lo=40, len_hi=150)
