@@ -7,8 +7,9 @@
 // alone or packed.  The cluster kernel gives a one-row call the same bits as a packed one, but it
 // sweeps the whole vocabulary on one cluster.  Here the same arithmetic is spread over the GPU:
 // k_lm_decode1 reads W once on every SM and leaves per-sub-tile row maxima, each step's reference
-// and 32-column partial sums (about 1/20 of the logits); k_lm_zscan combines them per row in the
-// cluster kernel's order.
+// and 32-column partial sums (about 1/18 of the rows' fp32 logits); k_lm_zscan combines them per
+// row in the cluster kernel's order.  A call launches k_d1_zero (status word and maxima), then
+// k_lm_decode1 (cooperative), then k_lm_zscan as a programmatic dependent of it.
 #pragma once
 
 #include "kernels_lm.cuh"
