@@ -934,15 +934,16 @@ bi_status bi_d3_stats(const float* learner_logprob, const float* rollout_logprob
   const size_t nred = static_cast<size_t>((T > 0 ? T : 1) + bi::kRedBlock - 1) / bi::kRedBlock;
   if (!ws || ws_bytes < nred * sizeof(RedPart) || (reinterpret_cast<uintptr_t>(ws) & 255u)) return BI_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s) != cudaSuccess) return BI_ERR_CUDA;
   RedPart* parts = static_cast<RedPart*>(ws);
+  // one partial per kD3BlockRows rows (the workspace holds one per kRedBlock rows, more than that)
+  const size_t nblk = static_cast<size_t>((T > 0 ? T : 1) + bi::kD3BlockRows - 1) / bi::kD3BlockRows;
   {
     ProfScope ps(kKD3Partial, s);
-    bi::k_d3_partial<<<static_cast<unsigned>(nred), bi::kRedBlock, 0, s>>>(learner_logprob, rollout_logprob, mask, T,
-                                                                           parts);
+    bi::k_d3_partial<<<static_cast<unsigned>(nblk), bi::kRedBlock, 0, s>>>(learner_logprob, rollout_logprob, mask, T,
+                                                                           parts, dev_status);
   }
   ProfScope ps(kKReduce, s);
-  bi::k_reduce_parts<<<1, 1024, 0, s>>>(parts, static_cast<int>(nred), nullptr, 0, nullptr,
+  bi::k_reduce_parts<<<1, 1024, 0, s>>>(parts, static_cast<int>(nblk), nullptr, 0, nullptr,
                                         reinterpret_cast<bi::D3Out*>(out), dev_status);
   return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
 }

@@ -223,17 +223,66 @@ __global__ void k_row_parts(const float* __restrict__ tl_c, const float* __restr
   if (threadIdx.x == 0) parts[blockIdx.x] = b;
 }
 
-// One thread per row of bi_d3_stats.
+// bi_d3_stats: one block partial per kD3BlockRows rows.  A thread sums its rows in a fixed order
+// (four consecutive rows per step, kD3Steps steps kRedBlock x 4 rows apart, so that every step of
+// the block reads 4 KB of each input contiguously) before the block reduction, whose cost would
+// otherwise outweigh the 9 bytes a row brings in.
+constexpr int kD3Steps = 8;
+constexpr int kD3BlockRows = kRedBlock * 4 * kD3Steps;
+
+__device__ __forceinline__ void acc_token(RedPart& v, float delta, float d3) {
+  const double dd = static_cast<double>(delta);
+  v.d3sum += static_cast<double>(d3);
+  v.d3max = max_keep_nan(v.d3max, d3);
+  v.k1sum -= dd;
+  v.k2sum += 0.5 * dd * dd;
+  v.count += 1;
+  v.nonfinite += isfinite(d3) ? 0 : 1;
+}
+
 __global__ void k_d3_partial(const float* __restrict__ lp, const float* __restrict__ mu,
-                             const uint8_t* __restrict__ mask, int64_t T, RedPart* parts) {
-  const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+                             const uint8_t* __restrict__ mask, int64_t T, RedPart* parts, int32_t* status) {
+  // the status word starts at BI_OK here; only k_reduce_parts, launched after this kernel, raises it
+  if (blockIdx.x == 0 && threadIdx.x == 0) *status = 0;
+  const int64_t base = static_cast<int64_t>(blockIdx.x) * kD3BlockRows;
+  // 16-byte loads where the arrays allow them (the API takes any float pointers)
+  const bool vec = ((reinterpret_cast<uintptr_t>(lp) | reinterpret_cast<uintptr_t>(mu)) & 15u) == 0 &&
+                   (mask == nullptr || (reinterpret_cast<uintptr_t>(mask) & 3u) == 0);
   RedPart v = red_zero();
-  if (t < T && (mask == nullptr || mask[t] != 0)) {
-    const float delta = lp[t] - mu[t];
-    add_token(v, delta, expm1f(delta) - delta);
+#pragma unroll
+  for (int k = 0; k < kD3Steps; ++k) {
+    const int64_t t0 = base + (static_cast<int64_t>(k) * kRedBlock + threadIdx.x) * 4;
+    float a[4], b[4];
+    uint32_t m[4] = {1u, 1u, 1u, 1u};
+    if (vec && t0 + 3 < T) {
+      const float4 av = *reinterpret_cast<const float4*>(lp + t0);
+      const float4 bv = *reinterpret_cast<const float4*>(mu + t0);
+      a[0] = av.x; a[1] = av.y; a[2] = av.z; a[3] = av.w;
+      b[0] = bv.x; b[1] = bv.y; b[2] = bv.z; b[3] = bv.w;
+      if (mask != nullptr) {
+        const uint32_t mw = *reinterpret_cast<const uint32_t*>(mask + t0);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) m[e] = (mw >> (8 * e)) & 0xffu;
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const bool in = t0 + e < T;
+        a[e] = in ? lp[t0 + e] : 0.f;
+        b[e] = in ? mu[t0 + e] : 0.f;
+        m[e] = in ? (mask != nullptr ? mask[t0 + e] : 1u) : 0u;
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (m[e] != 0u) {
+        const float delta = a[e] - b[e];
+        acc_token(v, delta, expm1f(delta) - delta);
+      }
+    }
   }
-  const RedPart b = block_reduce(v);
-  if (threadIdx.x == 0) parts[blockIdx.x] = b;
+  const RedPart r = block_reduce(v);
+  if (threadIdx.x == 0) parts[blockIdx.x] = r;
 }
 
 // One block per response (sequence-gate variant).  rho_i = mean of delta over the response's

@@ -7,7 +7,7 @@ forward logits + log-softmax + target gather, IS weight, D3, advantages, loss, d
 Inputs (hidden 0.2 GB, W 0.47 GB) are larger than the 126 MB L2, so no flush is needed between
 steps.  Prints one JSON line (rank 0).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload loss|dense]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload loss|dense|decode|d3]
 
 The default line runs the path that never writes anything of size T x V to device memory: the
 fused forward + dH kernel, then the dW kernel that recomputes the logits tile by tile.  The opt-in
@@ -29,6 +29,9 @@ Y = X W^T with W [8960, 1536] (bi_rmsnorm + bi_gemm_bf16); ranks are independent
 --workload decode times decode-style scoring (not the default line): one bi_logprob_fwd call per
 step on one row of the 1.5B head (the all-SM path: one pass over W on every SM, then the
 per-row combine), with the cluster kernel's latency beside it.
+
+--workload d3 times bi_d3_stats (not the default line): the D3 statistic and the KL estimators of
+2^24 tokens' learner and rollout log-probabilities with a mask, an HBM-bound reduction, in GB/s.
 """
 from __future__ import annotations
 
@@ -64,9 +67,9 @@ def parse():
     ap.add_argument("--small", action="store_true",
                     help="profiling case: same head, 4 responses of 1408 rows (T=5632: two full rounds of "
                          "22 clusters); not a bench line")
-    ap.add_argument("--workload", choices=["loss", "dense", "decode"], default="loss",
+    ap.add_argument("--workload", choices=["loss", "dense", "decode", "d3"], default="loss",
                     help="loss: the fused LM-head step (default line); dense: RMSNorm + linear layer; "
-                         "decode: one-row logprob scoring latency")
+                         "decode: one-row logprob scoring latency; d3: bi_d3_stats over 2^24 tokens")
     ap.add_argument("--dry-run", action="store_true",
                     help="CPU check of the multi-rank plumbing (gloo, tiny workload, no GPU kernels)")
     ap.add_argument("--no-pstore", action="store_true", help="skip the opt-in P-store comparison key")
@@ -830,6 +833,141 @@ def run_decode(args):
         print(json.dumps(line), flush=True)
 
 
+D3_T = 1 << 24
+D3_METRIC = "bi_d3_stats (D3 and the KL estimators) GB/s over 16,777,216 tokens"
+D3_BYTES_PER_TOKEN = 9  # fp32 learner and rollout log-probabilities, u8 mask
+
+
+def d3_workload():
+    """The D3 line's workload name, the same in both arms' `config`."""
+    return f"d3: bi_d3_stats over {D3_T} tokens (fp32 log pi and log mu, u8 mask scoring 80%)"
+
+
+def d3_cpu_sample(lp, mu, mask, rows):
+    """The fp64 oracle's D3 statistics over the first `rows` tokens: (seconds, cores)."""
+    from oracle import isloss_oracle as orc
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max((d.get("num_threads", 1) for d in threadpool_info()), default=os.cpu_count())
+    except Exception:  # pragma: no cover
+        cores = os.cpu_count()
+    t0 = time.perf_counter()
+    orc.d3_stats(lp[:rows], mu[:rows], mask[:rows])
+    return time.perf_counter() - t0, int(cores)
+
+
+def run_d3_reference(args):
+    """--impl reference --workload d3: the fp64 oracle on the host cores, a 2^21-token slice per step."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    from workloads import logprob_pair_inputs
+    rows = 1 << 21
+    lp, mu, mask = logprob_pair_inputs(rows, seed=1234)
+    times, cores = [], 1
+    for i in range(args.warmup + args.steps):
+        dt, cores = d3_cpu_sample(lp, mu, mask, rows)
+        if i >= args.warmup:
+            times.append(dt)
+    sec = statistics.mean(times)
+    val = D3_BYTES_PER_TOKEN * rows / sec / 1e9
+    print(json.dumps({"impl": "reference", "metric": D3_METRIC, "value": val, "unit": "GB/s", "n_gpus": world,
+                      "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sec,
+                      "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                      "data": "synthetic", "config": {"workload": d3_workload()},
+                      "cpu_baseline": {"value": val, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                                       "sample": f"the first {rows} tokens per step (fp64 NumPy)"},
+                      "e2e": {"value": val, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),
+          flush=True)
+
+
+def run_d3(args):
+    """--workload d3: bi_d3_stats over 2^24 tokens, HBM-bound; GB/s of algorithmic bytes."""
+    rank, world, local = dist_env()
+    import async_rl_b200 as bi
+    from async_rl_b200.build import build
+    from workloads import logprob_pair_inputs
+
+    if rank == 0:
+        build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    T = D3_T
+    lp, mu, mask = logprob_pair_inputs(T, seed=1234 + rank, device=dev)
+    ws = bi.make_workspace(T, 64, 1, 0, dev)
+    nbytes = D3_BYTES_PER_TOKEN * T
+
+    def call(a, b, m):
+        return bi.d3_stats(a, b, m, ws=ws)
+
+    for _ in range(args.warmup):
+        call(lp, mu, mask)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        raw, st = call(lp, mu, mask)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    bi.profile_reset()
+    bi.profile_enable(True)
+    for _ in range(args.steps):
+        raw, st = call(lp, mu, mask)
+    torch.cuda.synchronize()
+    bi.profile_enable(False)
+    clk = clocks.stop()
+    prof = bi.profile_read()
+    bi.check_status(st)
+    # end to end: the three arrays copied in from pinned memory and the 40-byte result read back
+    lph, muh, mh = lp.cpu().pin_memory(), mu.cpu().pin_memory(), mask.cpu().pin_memory()
+    rawh = torch.empty(40, dtype=torch.uint8).pin_memory()
+    lpd, mud, md = torch.empty_like(lp), torch.empty_like(mu), torch.empty_like(mask)
+    torch.cuda.synchronize()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record()
+    for _ in range(args.steps):
+        lpd.copy_(lph, non_blocking=True)
+        mud.copy_(muh, non_blocking=True)
+        md.copy_(mh, non_blocking=True)
+        raw, st = call(lpd, mud, md)
+        rawh.copy_(raw, non_blocking=True)
+    f1.record()
+    torch.cuda.synchronize()
+    ems = f0.elapsed_time(f1) / args.steps
+    cpu = None
+    if rank == 0 and not args.no_cpu_baseline:
+        rows = 1 << 21
+        sec, cores = d3_cpu_sample(lph, muh, mh, rows)
+        cpu = {"value": D3_BYTES_PER_TOKEN * rows / sec / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+               "sample": f"the first {rows} tokens (fp64 NumPy), {sec:.2f} s"}
+    peaks, peak_src = measured_peaks()
+    kp = prof.get("k_d3_partial", (float("nan"), 1))
+    kp_ms = kp[0] / max(kp[1], 1)
+    achieved = nbytes / (kp_ms * 1e-3) / 1e9
+    line = {"metric": D3_METRIC, "value": nbytes / (ms * 1e-3) / 1e9 * world, "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": d3_workload(), "parallelism": f"replicas{world}",
+                       "l2": "inputs 151 MB, larger than L2; no flush"},
+            "roofline": {"bound": "hbm", "kernel": "k_d3_partial", "achieved": achieved,
+                         "peak": float(peaks.get("hbm_gbs")), "unit": "GB/s",
+                         "frac": achieved / float(peaks.get("hbm_gbs")), "traffic": None,
+                         "peak_source": f"{peak_src} hbm_gbs", "algorithmic_bytes_per_launch": nbytes},
+            "kernels": {k: {"ms_per_launch": v[0] / max(v[1], 1), "launches": v[1]} for k, v in prof.items()},
+            "gpu_launches": int(sum(v[1] for v in prof.values())), "clocks": clk,
+            "e2e": {"value": nbytes / (ems * 1e-3) / 1e9 * world, "unit": "GB/s", "h2d_bytes_per_step": nbytes,
+                    "d2h_bytes_per_step": 40,
+                    "h2d": "pinned host arrays in, the 40-byte result out, every call"}}
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     relaunch_if_needed(args)
@@ -846,6 +984,11 @@ def main():
             run_dense_reference(args)
         else:
             run_dense(args)
+    elif args.workload == "d3":
+        if args.impl == "reference":
+            run_d3_reference(args)
+        else:
+            run_d3(args)
     elif args.impl == "reference":
         run_reference(args)
     else:

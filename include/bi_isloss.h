@@ -229,7 +229,9 @@ BI_API bi_status bi_is_loss_fwd_bwd(const uint16_t* hidden, const uint16_t* w_lm
 /* D3 statistics from two logprob arrays ("Zero Mismatch", "Only one probability gap ..."):
  *   learner_logprob [T] float, rollout_logprob [T] float, mask [T] uint8 (may be NULL: all rows;
  *   otherwise rows with mask != 0).  out [1] bi_d3 in device memory.  Sets BI_ERR_NONFINITE in
- *   *dev_status when a term is non-finite. */
+ *   *dev_status when a term is non-finite.  The terms are summed in float64 in a fixed order:
+ *   per block of 8192 rows, then over the blocks (16-byte loads when the two arrays are 16-byte
+ *   aligned and the mask 4-byte aligned, element loads otherwise, with the same sums). */
 BI_API bi_status bi_d3_stats(const float* learner_logprob, const float* rollout_logprob,
                       const uint8_t* mask, int64_t T, bi_d3* out, int32_t* dev_status, void* ws,
                       size_t ws_bytes, void* stream);

@@ -220,3 +220,17 @@ def norm_inputs(M: int, H: int, seed: int, device="cpu"):
     x.mul_(torch.rand((M, 1), generator=gen, device=device) * 19.95 + 0.05)
     g = 1.0 + 0.1 * torch.randn((H,), generator=gen, device=device)
     return x.to(torch.bfloat16), g.to(torch.bfloat16)
+
+
+def logprob_pair_inputs(T: int, seed: int, device="cpu"):
+    """(learner log-probs, rollout log-probs, mask) for the D3 statistics: learner log pi ~
+    N(-8, 2^2), rollout log mu = log pi + N(0, 0.05^2) with 1% of the tokens moved by a further
+    N(0, 1) (mismatch spikes), and a mask that scores 80% of the tokens; fp32, fp32, u8."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    lp = torch.randn(T, generator=gen, device=device) * 2.0 - 8.0
+    mu = lp + torch.randn(T, generator=gen, device=device) * 0.05
+    spikes = torch.randperm(T, generator=gen, device=device)[: max(1, T // 100)]
+    mu[spikes] += torch.randn(spikes.shape[0], generator=gen, device=device)
+    mask = (torch.rand(T, generator=gen, device=device) < 0.8).to(torch.uint8)
+    return lp.float(), mu.float(), mask
