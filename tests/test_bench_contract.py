@@ -106,3 +106,21 @@ def test_decode_workload_line():
     # pass over W on every SM, then the combine
     assert line["gpu_launches"] == 3 * 20 and line["value"] < line["cluster_kernel_ms"]
     assert 0 < line["roofline"]["frac"] < 2 and line["e2e"]["h2d_bytes_per_step"] > 0
+
+
+def test_d3_reference_arm_line():
+    line = _run(["--impl", "reference", "--workload", "d3", "--steps", "1", "--warmup", "0"], timeout=600)
+    for k in REQUIRED:
+        assert k in line, k
+    assert line["impl"] == "reference" and line["unit"] == "GB/s" and line["value"] > 0
+
+
+@pytest.mark.gpu
+def test_d3_workload_line():
+    line = _run(["--workload", "d3", "--steps", "10", "--warmup", "3"], timeout=900)
+    for k in REQUIRED + ("roofline", "clocks", "gpu_launches", "cpu_baseline"):
+        assert k in line, k
+    # two launches per call: the block partials, then their fixed-order sum
+    assert line["gpu_launches"] == 2 * 10
+    assert line["roofline"]["bound"] == "hbm" and 0 < line["roofline"]["frac"] < 2
+    assert line["e2e"]["h2d_bytes_per_step"] == 9 * (1 << 24)
