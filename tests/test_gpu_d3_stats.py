@@ -76,3 +76,23 @@ def test_d3_stats_empty_and_fully_masked(cuda_device):
     lp, mu, _ = _inputs(300, seed=4)
     got, st = _run(lp, mu, torch.zeros(300, dtype=torch.uint8), cuda_device)
     assert st == 0 and got["count"] == 0 and got["mean"] == 0.0 and got["max"] == 0.0
+
+
+def test_d3_stats_unaligned_arrays_give_the_same_sums(cuda_device):
+    """Arrays starting 4 bytes (and the mask 1 byte) past an alignment boundary take the kernel's
+    element loads instead of its 16-byte loads; the sums, formed in the same order, are the same
+    bits, and both agree with the oracle."""
+    T = 70001
+    lp, mu, mask = _inputs(T + 1, seed=33)
+    lpd, mud, md = lp.to(cuda_device), mu.to(cuda_device), mask.to(cuda_device)
+    # the same T values, once 16-byte aligned (fresh copies) and once at an offset of one element
+    a_lp, a_mu, a_m = lpd[1:].clone(), mud[1:].clone(), md[1:].clone()
+    u_lp, u_mu, u_m = lpd[1:], mud[1:], md[1:]
+    assert u_lp.data_ptr() % 16 != 0 and u_m.data_ptr() % 4 != 0
+    ga, sa = _run(a_lp, a_mu, a_m, cuda_device)
+    gu, su = _run(u_lp, u_mu, u_m, cuda_device)
+    assert sa == su == 0
+    assert ga == gu
+    ref = orc.d3_stats(lp[1:].double().numpy(), mu[1:].double().numpy(), mask[1:].numpy())
+    assert gu["count"] == ref["count"]
+    assert abs(gu["mean"] - ref["mean"]) <= 1e-4 * abs(ref["mean"])
