@@ -230,14 +230,13 @@ __global__ void k_row_parts(const float* __restrict__ tl_c, const float* __restr
 constexpr int kD3Steps = 8;
 constexpr int kD3BlockRows = kRedBlock * 4 * kD3Steps;
 
+// One token into a thread's running sums (the counts are kept by the caller in 32 bits).
 __device__ __forceinline__ void acc_token(RedPart& v, float delta, float d3) {
   const double dd = static_cast<double>(delta);
   v.d3sum += static_cast<double>(d3);
   v.d3max = max_keep_nan(v.d3max, d3);
   v.k1sum -= dd;
   v.k2sum += 0.5 * dd * dd;
-  v.count += 1;
-  v.nonfinite += isfinite(d3) ? 0 : 1;
 }
 
 __global__ void k_d3_partial(const float* __restrict__ lp, const float* __restrict__ mu,
@@ -249,6 +248,7 @@ __global__ void k_d3_partial(const float* __restrict__ lp, const float* __restri
   const bool vec = ((reinterpret_cast<uintptr_t>(lp) | reinterpret_cast<uintptr_t>(mu)) & 15u) == 0 &&
                    (mask == nullptr || (reinterpret_cast<uintptr_t>(mask) & 3u) == 0);
   RedPart v = red_zero();
+  int32_t cnt = 0, nonfin = 0;  // at most kD3BlockRows / kRedBlock tokens per thread
 #pragma unroll
   for (int k = 0; k < kD3Steps; ++k) {
     const int64_t t0 = base + (static_cast<int64_t>(k) * kRedBlock + threadIdx.x) * 4;
@@ -277,10 +277,15 @@ __global__ void k_d3_partial(const float* __restrict__ lp, const float* __restri
     for (int e = 0; e < 4; ++e) {
       if (m[e] != 0u) {
         const float delta = a[e] - b[e];
-        acc_token(v, delta, expm1f(delta) - delta);
+        const float d3 = expm1f(delta) - delta;
+        acc_token(v, delta, d3);
+        cnt += 1;
+        nonfin += isfinite(d3) ? 0 : 1;
       }
     }
   }
+  v.count = cnt;
+  v.nonfinite = nonfin;
   const RedPart r = block_reduce(v);
   if (threadIdx.x == 0) parts[blockIdx.x] = r;
 }
